@@ -1,0 +1,377 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees with
+a fact fixed by the pages or by mathematics:
+
+* the pages' printed examples (``tests/golden``): block tables, the
+  block-size-4 worked example, capacity figures;
+* special cases that reduce to a library routine: numpy's binary16 and
+  torch's bfloat16 conversions; dense, unpaged attention written with
+  numpy matmul on the logical (position-ordered) rows;
+* closed forms: a context of one token returns that token's V exactly;
+  identical keys give the mean of V; split-context partial results merge
+  to the unsplit result (log-sum-exp identity);
+* brute force on tiny inputs with ``math.fsum``;
+* invariances: relabelling physical blocks, poison in slots never read.
+
+``test_oracle_pins.py`` runs every pin against the oracle;
+``test_oracle_mutants.py`` compiles copies of the oracle with a planted
+mistake and checks that some pin fails for each.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import oracle
+import synth
+from conftest import read_golden
+from oracle.allocator_model import BlockManagerModel
+
+NAN_BITS = {"f16": 0x7E00, "bf16": 0x7FC0}
+
+
+# --------------------------------------------------------------------------- library decoders
+def lib_f64(bits: np.ndarray, dtype: str) -> np.ndarray:
+    """Widen 16-bit patterns with library routines (numpy / torch), not the oracle."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    if dtype == "f16":
+        return bits.view(np.float16).astype(np.float64)
+    t = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+def _same(a, b):
+    return np.array_equal(np.isnan(a), np.isnan(b)) and np.array_equal(a[~np.isnan(a)],
+                                                                       b[~np.isnan(b)])
+
+
+def pin_f16_decoder():
+    allbits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    assert _same(oracle.widen(allbits, "f16"), lib_f64(allbits, "f16")), "binary16 decode"
+
+
+def pin_bf16_decoder():
+    allbits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    assert _same(oracle.widen(allbits, "bf16"), lib_f64(allbits, "bf16")), "bfloat16 decode"
+
+
+# --------------------------------------------------------------------------- slots (pages)
+def _check_table_fixture(bs, ranges, physical, n_positions):
+    row = np.array(physical, dtype=np.int32)
+    for (lb, lo, hi) in ranges:
+        for t in range(lo, min(hi, n_positions - 1) + 1):
+            s = oracle.slot(row, t, bs)
+            assert s // bs == physical[lb], f"token {t}: block {s // bs} != {physical[lb]}"
+            assert s % bs == t - lo, f"token {t}: offset {s % bs} != {t - lo}"
+
+
+def pin_worked_example_slots():
+    g = read_golden("worked_example_bs4.txt")
+    bs = int(g["block_size"][0][0])
+    physical = [int(x) for x in g["physical"][0]]
+    ranges = [(int(v[0]), int(v[2]), int(v[3])) for v in g["logical_block"]]
+    _check_table_fixture(bs, ranges, physical, n_positions=12)
+    # the 11th token (index 10) still lands in logical block 2
+    nth, lb = (int(x) for x in g["nth_token_in_logical_block"][0])
+    assert oracle.slot(np.array(physical, np.int32), nth - 1, bs) // bs == physical[lb]
+
+
+def pin_bs16_tables():
+    g = read_golden("block_tables_bs16.txt")
+    bs = int(g["block_size"][0][0])
+    ranges = [(int(v[0]), int(v[2]), int(v[3])) for v in g["logical_block"]]
+    for key in ("table_A", "table_section5"):
+        physical = [int(x) for x in g[key][0]]
+        _check_table_fixture(bs, ranges, physical, n_positions=48)
+
+
+# --------------------------------------------------------------------------- placement
+def place_numpy(batch, include_new=True, poison=True):
+    """Independent placement of a batch's logical rows into fresh pools by numpy
+    indexing: position t of sequence b goes to block table[b][t // bs], offset
+    t % bs. Unwritten entries hold NaN patterns when ``poison`` is set."""
+    shape = (batch.num_blocks, batch.num_kv_heads, batch.block_size, batch.head_dim)
+    fill = NAN_BITS[batch.dtype] if poison else 0
+    kp = np.full(shape, fill, dtype=np.uint16)
+    vp = np.full(shape, fill, dtype=np.uint16)
+    bs = batch.block_size
+    for b in range(batch.num_seqs):
+        n = int(batch.context_lens[b]) - (0 if include_new else 1)
+        if n <= 0:
+            continue
+        t = np.arange(n)
+        blocks = batch.block_tables[b][t // bs]
+        rows = batch.rows(b)
+        kp[blocks, :, t % bs, :] = batch.k[rows][:n]
+        vp[blocks, :, t % bs, :] = batch.v[rows][:n]
+    return kp, vp
+
+
+def dense_reference(batch):
+    """Unpaged attention on the logical rows with numpy fp64 matmuls; query head h
+    uses KV head h // (Hq / Hkv) (np.repeat = contiguous groups)."""
+    G = batch.num_q_heads // batch.num_kv_heads
+    out = np.zeros((batch.num_seqs, batch.num_q_heads, batch.head_dim))
+    q = lib_f64(batch.q, batch.dtype)
+    for b in range(batch.num_seqs):
+        n = int(batch.context_lens[b])
+        if n == 0:
+            continue
+        K = np.repeat(lib_f64(batch.k[batch.rows(b)], batch.dtype), G, axis=1)
+        V = np.repeat(lib_f64(batch.v[batch.rows(b)], batch.dtype), G, axis=1)
+        for h in range(batch.num_q_heads):
+            s = (K[:, h, :] @ q[b, h]) * float(batch.scale)
+            w = np.exp(s - s.max())
+            out[b, h] = (w @ V[:, h, :]) / w.sum()
+    return out
+
+
+def oracle_out(batch, kp=None, vp=None):
+    if kp is None:
+        kp, vp = place_numpy(batch)
+    return oracle.decode(batch.q, kp, vp, batch.block_tables, batch.context_lens, batch.scale,
+                         batch.dtype)
+
+
+def small_batches():
+    """Small paged batches over the shapes that matter: GQA and MHA, both
+    dtypes, block sizes 4..32, lengths 1, block-aligned and ragged."""
+    return [
+        synth.small_random(11, 5, [1, 4, 5, 17, 40], 4, 2, 16, 4, 80, "f16"),
+        synth.small_random(12, 4, [3, 16, 31, 33], 8, 2, 32, 16, 16, "bf16"),
+        synth.small_random(13, 3, [64, 9, 1], 6, 6, 8, 32, 12, "f16"),
+        synth.small_random(14, 2, [100, 7], 4, 1, 24, 8, 40, "bf16"),
+        synth.tiny(),
+    ]
+
+
+def pin_dense(batches=None, tol=1e-12):
+    for batch in batches or small_batches():
+        got = oracle_out(batch)
+        ref = dense_reference(batch)
+        err = np.max(np.abs(got - ref)) if got.size else 0.0
+        assert err <= tol, f"{batch.name}: paged oracle vs dense numpy differ by {err}"
+
+
+def pin_len1_returns_v():
+    batch = synth.small_random(21, 6, [1] * 6, 8, 4, 16, 4, 64, "bf16")
+    got = oracle_out(batch)
+    G = batch.num_q_heads // batch.num_kv_heads
+    for b in range(batch.num_seqs):
+        v = lib_f64(batch.v[batch.seq_start[b]], batch.dtype)  # [Hkv, D]
+        for h in range(batch.num_q_heads):
+            assert np.array_equal(got[b, h], v[h // G]), "length-1 context must return V"
+
+
+def pin_identical_keys_mean_v():
+    batch = synth.small_random(22, 3, [5, 19, 37], 4, 4, 16, 8, 20, "f16")
+    for b in range(batch.num_seqs):
+        r = batch.rows(b)
+        batch.k[r] = batch.k[r][0:1]  # every key row of the sequence equal to its first
+    got = oracle_out(batch)
+    for b in range(batch.num_seqs):
+        V = lib_f64(batch.v[batch.rows(b)], batch.dtype)  # [n, H, D]
+        for h in range(batch.num_q_heads):
+            for d in range(batch.head_dim):
+                mean = math.fsum(V[:, h, d]) / V.shape[0]
+                assert abs(got[b, h, d] - mean) <= 1e-14, "identical keys must average V"
+
+
+def pin_bruteforce_fsum():
+    batch = synth.small_random(23, 3, [2, 6, 11], 4, 2, 8, 4, 12, "bf16")
+    got = oracle_out(batch)
+    G = batch.num_q_heads // batch.num_kv_heads
+    q = lib_f64(batch.q, batch.dtype).tolist()
+    for b in range(batch.num_seqs):
+        K = lib_f64(batch.k[batch.rows(b)], batch.dtype).tolist()
+        V = lib_f64(batch.v[batch.rows(b)], batch.dtype).tolist()
+        n = len(K)
+        for h in range(batch.num_q_heads):
+            g = h // G
+            s = [float(batch.scale) * math.fsum(q[b][h][d] * K[t][g][d]
+                                                for d in range(batch.head_dim)) for t in range(n)]
+            m = max(s)
+            w = [math.exp(x - m) for x in s]
+            den = math.fsum(w)
+            for d in range(batch.head_dim):
+                ref = math.fsum(w[t] * V[t][g][d] for t in range(n)) / den
+                assert abs(got[b, h, d] - ref) <= 1e-13, "brute force disagrees"
+
+
+def pin_relabel():
+    batch = synth.small_random(24, 4, [13, 30, 2, 47], 4, 2, 16, 8, 40, "f16")
+    kp, vp = place_numpy(batch)
+    base = oracle_out(batch, kp, vp)
+    perm = np.random.default_rng(5).permutation(batch.num_blocks)
+    kp2, vp2 = np.empty_like(kp), np.empty_like(vp)
+    kp2[perm] = kp
+    vp2[perm] = vp
+    tables = perm[batch.block_tables].astype(np.int32)
+    got = oracle.decode(batch.q, kp2, vp2, tables, batch.context_lens, batch.scale, batch.dtype)
+    assert np.array_equal(got, base), "relabelling physical blocks changed the output"
+
+
+def pin_poison():
+    batch = synth.small_random(25, 4, [3, 17, 16, 9], 8, 2, 16, 8, 24, "bf16")
+    clean = oracle_out(batch, *place_numpy(batch, poison=False))
+    dirty = oracle_out(batch, *place_numpy(batch, poison=True))
+    assert np.all(np.isfinite(dirty)), "poison in unread slots reached the output"
+    assert np.array_equal(clean, dirty), "unread slots changed the output"
+
+
+def pin_partition_merge():
+    for batch in small_batches()[:4]:
+        kp, vp = place_numpy(batch)
+        full = oracle_out(batch, kp, vp)
+        ref_scores = _dense_scores(batch)
+        for pt in (1, 3, 16, 64, 512):
+            out, pm, pl, _ = oracle.decode_partitioned(batch.q, kp, vp, batch.block_tables,
+                                                       batch.context_lens, batch.scale,
+                                                       batch.dtype, pt, return_partials=True)
+            err = np.max(np.abs(out - full))
+            assert err <= 1e-12, f"partition {pt}: merged result off by {err}"
+            for b in range(batch.num_seqs):
+                n = int(batch.context_lens[b])
+                for h in range(batch.num_q_heads):
+                    for p in range(-(-n // pt)):
+                        s = ref_scores[b][h][p * pt:(p + 1) * pt]
+                        assert abs(pm[b, h, p] - s.max()) <= 1e-12, "partition max"
+                        assert abs(pl[b, h, p] - np.exp(s - s.max()).sum()) <= 1e-11, "partition sum"
+
+
+def _dense_scores(batch):
+    G = batch.num_q_heads // batch.num_kv_heads
+    q = lib_f64(batch.q, batch.dtype)
+    res = []
+    for b in range(batch.num_seqs):
+        K = lib_f64(batch.k[batch.rows(b)], batch.dtype)
+        res.append([(K[:, h // G, :] @ q[b, h]) * float(batch.scale)
+                    for h in range(batch.num_q_heads)])
+    return res
+
+
+# --------------------------------------------------------------------------- write / copy
+def pin_reshape_layout():
+    """Write the worked example's 10 tokens (block size 4, blocks 8, 3, 15) at the
+    oracle's slots; each row must sit at pool[physical, head, offset, :]."""
+    g = read_golden("worked_example_bs4.txt")
+    bs = int(g["block_size"][0][0])
+    physical = [int(x) for x in g["physical"][0]]
+    ranges = [(int(v[0]), int(v[2]), int(v[3])) for v in g["logical_block"]]
+    n, H, D = int(g["num_tokens"][0][0]), 2, 4
+    rng = np.random.default_rng(0)
+    k_new = rng.integers(0, 1 << 16, size=(n + 1, H, D), dtype=np.uint64).astype(np.uint16)
+    v_new = rng.integers(0, 1 << 16, size=(n + 1, H, D), dtype=np.uint64).astype(np.uint16)
+    # the example's 10 tokens, then a padding token (slot -1), then a token at slot 0
+    slots = np.append(oracle.slots_for(np.array(physical, np.int32), range(n), bs), [-1, 0])
+    k_new = np.concatenate([k_new, k_new[:1]])
+    v_new = np.concatenate([v_new, v_new[:1]])
+    kc = oracle.empty_pool(16, H, bs, D)
+    vc = oracle.empty_pool(16, H, bs, D)
+    oracle.reshape_and_cache(k_new, v_new, slots, kc, vc)
+    written = np.zeros(kc.shape[:3], dtype=bool)
+    assert np.array_equal(kc[0, :, 0, :], k_new[-1]) and np.array_equal(vc[0, :, 0, :], v_new[-1])
+    written[0, :, 0] = True
+    for (lb, lo, hi) in ranges:
+        for t in range(lo, min(hi, n - 1) + 1):
+            assert np.array_equal(kc[physical[lb], :, t - lo, :], k_new[t]), f"K token {t}"
+            assert np.array_equal(vc[physical[lb], :, t - lo, :], v_new[t]), f"V token {t}"
+            written[physical[lb], :, t - lo] = True
+    assert not kc[~written].any() and not vc[~written].any(), "write touched other slots"
+
+
+def pin_copy_blocks():
+    rng = np.random.default_rng(1)
+    shape = (12, 3, 8, 16)
+    kc = rng.integers(0, 1 << 16, size=shape, dtype=np.uint64).astype(np.uint16)
+    vc = rng.integers(0, 1 << 16, size=shape, dtype=np.uint64).astype(np.uint16)
+    k0, v0 = kc.copy(), vc.copy()
+    pairs = np.array([[3, 7], [0, 11], [5, 5]], dtype=np.int64)
+    oracle.copy_blocks(kc, vc, pairs)
+    exp_k, exp_v = k0.copy(), v0.copy()
+    for s, d in pairs:
+        exp_k[d] = k0[s]
+        exp_v[d] = v0[s]
+    assert np.array_equal(kc, exp_k) and np.array_equal(vc, exp_v), "copy_blocks"
+
+
+# --------------------------------------------------------------------------- block manager
+def pin_allocator_worked_example():
+    g = read_golden("worked_example_bs4.txt")
+    bs = int(g["block_size"][0][0])
+    n = int(g["num_tokens"][0][0])
+    m = BlockManagerModel(32, bs)
+    m.add_seq(0, n)
+    assert len(m.block_table(0)) == int(g["blocks_needed"][0][0])
+    nth, lb = (int(x) for x in g["nth_token_in_logical_block"][0])
+    # tokens n+1 .. nth-ish: the 11th and 12th tokens still go into logical block 2
+    for pos in range(n, 12):
+        slot, src, dst = m.append_slot(0)
+        assert slot // bs == m.block_table(0)[lb] and src == dst == -1
+    assert len(m.block_table(0)) == 3
+    new_at = int(g["nth_token_needs_new_block"][0][0])
+    assert m.lens[0] == new_at - 1
+    m.append_slot(0)
+    assert len(m.block_table(0)) == 4, "the 13th token must take a new block"
+    before = m.num_free()
+    m.free_seq(0)
+    returned = m.num_free() - before
+    assert returned in [int(x) for x in g["blocks_returned"][0]] and m.num_free() == 32
+
+
+def pin_allocator_capacity():
+    g = read_golden("capacity_figures.txt")
+    val = lambda k: int(g[k][0][0])  # noqa: E731
+    m = BlockManagerModel(4096, 16)
+    m.add_seq(1, val("request_tokens"))
+    assert len(m.block_table(1)) == val("request_blocks")
+    free, used, wasted = m.stats()
+    assert used == val("request_tokens") and 16 - wasted == val("request_last_block_fill")
+    assert wasted * val("llama31_8b_kv_bytes_per_token") == val("request_waste_bytes")
+    worst = 0
+    for n in range(1, 600):
+        mm = BlockManagerModel(64, 16)
+        mm.add_seq(0, n)
+        worst = max(worst, mm.stats()[2])
+    assert worst == val("max_waste_tokens_bs16")
+    rng = np.random.default_rng(2)
+    mm = BlockManagerModel(1 << 18, 16)
+    lens = rng.integers(1, 2000, size=2000)
+    for i, n in enumerate(lens):
+        mm.add_seq(i, int(n))
+    avg = mm.stats()[2] / len(lens)
+    assert abs(avg - val("avg_waste_tokens_bs16")) <= 0.75, f"average waste {avg}"
+
+
+def pin_allocator_cow():
+    """Reference-count trace of sharing and copy-on-write."""
+    m = BlockManagerModel(16, 4)
+    m.add_seq(0, 6)                    # blocks: one full, one holding 2 of 4
+    for c in (1, 2, 3):
+        m.fork(0, c)
+    shared = m.block_table(0)
+    assert all(m.ref[b] == 4 for b in shared), "fork adds one reference per block"
+    slot, src, dst = m.append_slot(1)  # writes into the shared, partly filled block
+    assert src == shared[1] and dst not in shared
+    assert m.ref[src] == 3 and m.ref[dst] == 1 and m.block_table(1)[1] == dst
+    assert slot == dst * 4 + 2
+    for c in (2, 3):
+        _, s2, _ = m.append_slot(c)
+        assert s2 == shared[1]
+    assert m.ref[shared[1]] == 1
+    slot0, s0, _ = m.append_slot(0)   # now the sole owner: writes in place
+    assert s0 == -1 and slot0 == shared[1] * 4 + 2
+    for c in (0, 1, 2, 3):
+        m.free_seq(c)
+    assert m.num_free() == 16 and all(r == 0 for r in m.ref)
+
+
+ALL_ORACLE_PINS = [
+    pin_f16_decoder, pin_bf16_decoder, pin_worked_example_slots, pin_bs16_tables, pin_dense,
+    pin_len1_returns_v, pin_identical_keys_mean_v, pin_bruteforce_fsum, pin_relabel, pin_poison,
+    pin_partition_merge, pin_reshape_layout, pin_copy_blocks,
+]
+ALL_MODEL_PINS = [pin_allocator_worked_example, pin_allocator_capacity, pin_allocator_cow]

@@ -1,0 +1,59 @@
+"""Plant one plausible mistake at a time in a copy of the oracle's C source and
+check that at least one pin catches it. This shows the pins constrain every
+part of the oracle: decoders, slot arithmetic, pool layout, scores, softmax,
+head grouping, the split-context merge, and the write / copy routines."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import pins
+
+MUTANTS = {
+    "scale_dropped": ("s[t] = scale * dot;", "s[t] = dot;"),
+    "group_by_modulo": ("int g = h / group;", "int g = h % num_kv_heads;"),
+    "slot_without_block_size": ("return (int64_t)table_row[logical_block] * block_size + offset;",
+                                "return (int64_t)table_row[logical_block] + offset;"),
+    "slot_offset_shifted": ("int64_t offset = pos % block_size;",
+                            "int64_t offset = (pos + 1) % block_size;"),
+    "pool_transposed": ("* block_size + offset) * head_dim + d;",
+                        "* head_dim + d) * block_size + offset;"),
+    "no_normalisation": ("out[d] /= denom;", "out[d] /= 1.0;"),
+    "softmax_sign": ("double w = exp(s[t] - m);", "double w = exp(m - s[t]);"),
+    "dot_drops_last": ("for (int d = 0; d < head_dim; ++d)\n            dot += q[d]",
+                       "for (int d = 0; d < head_dim - 1; ++d)\n            dot += q[d]"),
+    "v_is_k": ("out[d] += w * V[(size_t)t * head_dim + d];",
+               "out[d] += w * K[(size_t)t * head_dim + d];"),
+    "merge_unweighted": ("L += exp(m[p] - M) * l[p];", "L += l[p];"),
+    "partition_drops_tail": ("int t1 = t0 + partition_tokens < n ? t0 + partition_tokens : n;",
+                             "int t1 = t0 + partition_tokens < n ? t0 + partition_tokens : n - 1;"),
+    "f16_bias": ("mag = ldexp((double)(1024 + f), e - 25);", "mag = ldexp((double)(1024 + f), e - 24);"),
+    "bf16_bias": ("mag = ldexp((double)(128 + f), e - 134);", "mag = ldexp((double)(128 + f), e - 133);"),
+    "write_skips_slot0": ("if (slot < 0)\n            continue;", "if (slot <= 0)\n            continue;"),
+    "copy_k_only": ("v_cache[(size_t)dst * block_elems + i] = v_cache[(size_t)src * block_elems + i];",
+                    ";"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(oracle.SRC).read()
+    assert old in src, f"anchor of mutant {name} not found in oracle.c"
+    mutated = src.replace(old, new)
+    c_path = os.path.join(tmp_path, "oracle_mutant.c")
+    so_path = os.path.join(tmp_path, "liboracle_mutant.so")
+    with open(c_path, "w") as f:
+        f.write(mutated)
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-ffp-contract=off", "-fPIC", "-shared", "-std=c11",
+                    "-o", so_path, c_path, "-lm"], check=True)
+    caught = []
+    with oracle.using(so_path):
+        for pin in pins.ALL_ORACLE_PINS:
+            try:
+                pin()
+            except Exception as e:  # noqa: BLE001 -- any failure of a pin counts
+                caught.append((pin.__name__, type(e).__name__))
+                break
+    assert caught, f"no pin caught the planted mistake {name}"
