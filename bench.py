@@ -1,0 +1,584 @@
+#!/usr/bin/env python
+"""Benchmark: paged decode attention on B200 -- KV GB/s, % of HBM peak, query tokens/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload llama8b|long_skew|mixed|shared_prompt] [--block-size BS]
+
+A step is one pass of the whole hot path over one batch: the slot-indexed
+write of every sequence's new K/V (pa_reshape_and_cache), copy-on-write block
+copies where the workload has them (pa_copy_blocks), and paged decode
+attention with its split-context merge (pa_decode). The default workload is
+the Llama-3.1-8B-shaped single-layer batch: 64 sequences, 32 q / 8 KV heads,
+head_dim 128, bf16, 16-token blocks, lengths uniform in [128, 2048], a
+65,536-block pool. Four such batches with disjoint blocks live in the pool and
+steps rotate through them, so each step reads KV that is not in L2 (1.1 GB of
+KV across the four versus a 126 MB L2).
+
+Timing: each step's write and decode are replayed as CUDA graphs; CUDA events
+on the launching stream bracket the K timed steps (after W warm-up steps, with
+a barrier and a device synchronise on both sides) and the decode of every step.
+With N > 1 (torchrun, one process per GPU) every rank runs its own batches --
+the sequences shard across GPUs with no exchange -- and the slowest rank's
+time is used. ``e2e`` repeats the measurement with the step's inputs in pinned
+host memory, copied in and the output copied out inside every step.
+
+``--impl reference`` times the fp64 CPU oracle on the same workload instead
+(a bounded sample of sequences per step), on the host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from paged_kv_cache_370_b200.accounting import (decode_step_bytes, new_token_bytes,  # noqa: E402
+                                                split_scratch_bytes)
+
+METRIC = "paged decode attention: KV GB/s and % of B200 HBM peak; query tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_370_b200", "csrc", "pa_decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pa_decode_llama8b_traffic.md")
+
+
+# ------------------------------------------------------------------------------------- setup
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b",
+                    choices=["llama8b", "long_skew", "mixed", "shared_prompt"])
+    ap.add_argument("--block-size", type=int, default=16, help="block size of the mixed workload")
+    ap.add_argument("--variants", type=int, default=4, help="batches rotated (llama8b)")
+    ap.add_argument("--partition-tokens", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic():
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current decode source; else None."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    src = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_sha or not m_bytes or m_sha.group(1) != src:
+        return None
+    return int(m_bytes.group(1))
+
+
+# ---------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons for one GPU."""
+
+    FIELDS = ("timestamp,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id: str | None):
+        self.bus_id = (bus_id or "").lower()
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.bus_id and not parts[1].lower().endswith(self.bus_id[-12:]):
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        used = inside or [s for s in self.samples if t0 - 1.0 <= s[0] <= t1 + 1.0]
+        if not used:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in used for i, v in enumerate(s[3]) if v == "Active"})
+        return {"sm_mhz": float(np.median([s[1] for s in used])),
+                "sm_max_mhz": float(max(s[2] for s in used)), "reasons": reasons,
+                "samples": len(used), "samples_in_timed_region": len(inside)}
+
+
+# ------------------------------------------------------------------------------- workloads
+def make_batches(args, rank):
+    """Host-side batches of the workload for one rank (seeded per rank)."""
+    seed_shift = 1_000_003 * rank
+    if args.workload == "llama8b":
+        return [synth.llama8b(seed=synth.SEED_BASE + 2 + seed_shift, variant=v,
+                              num_variants=args.variants) for v in range(args.variants)]
+    if args.workload == "long_skew":
+        return [synth.long_skew(seed=synth.SEED_BASE + 3 + seed_shift)]
+    if args.workload == "mixed":
+        return [synth.mixed_sweep(args.block_size, seed=synth.SEED_BASE + 5 + seed_shift)]
+    return None  # shared_prompt is built through the block manager
+
+
+def workload_config(args, batches, pt):
+    if args.workload == "llama8b":
+        b = batches[0]
+        return {"workload": "Llama-3.1-8B-shaped single-layer paged decode",
+                "num_seqs": b.num_seqs, "num_q_heads": b.num_q_heads,
+                "num_kv_heads": b.num_kv_heads, "head_dim": b.head_dim,
+                "block_size": b.block_size, "context_lens": "uniform [128, 2048]",
+                "num_blocks": b.num_blocks, "partition_tokens": pt,
+                "batches_rotated": len(batches),
+                "l2": f"inputs larger than L2: {len(batches)} rotating batches, "
+                      f"{sum(decode_step_bytes(x.context_lens, 32, 8, 128, 16)['kv'] for x in batches) / 1e9:.2f} GB of KV",
+                "timing": "CUDA graphs replayed back to back; CUDA events on the stream"}
+    if args.workload == "long_skew":
+        return {"workload": "long-context skew decode", "num_seqs": 8, "num_q_heads": 32,
+                "num_kv_heads": 8, "head_dim": 128, "block_size": 16,
+                "context_lens": "uniform [8192, 32768]", "partition_tokens": pt,
+                "l2": "inputs larger than L2 (671 MB KV per step)"}
+    if args.workload == "mixed":
+        return {"workload": "mixed serving batch", "num_seqs": 256, "num_q_heads": 32,
+                "num_kv_heads": 8, "head_dim": 128, "block_size": args.block_size,
+                "context_lens": "log-uniform [16, 4096]", "partition_tokens": pt,
+                "l2": "inputs larger than L2 (~770 MB KV per step)"}
+    return {"workload": "OPT-13B-shaped shared-prompt decode with copy-on-write",
+            "num_seqs": 64, "num_q_heads": 40, "num_kv_heads": 40, "head_dim": 128,
+            "block_size": 16, "prompts": 16, "prompt_len": 512, "fork": 4,
+            "partition_tokens": pt, "l2": "shared prompt blocks hit in L2 by design"}
+
+
+def to_dev(bits, dtype, torch, device):
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device)
+    return t.view(torch.bfloat16 if dtype == "bf16" else torch.float16)
+
+
+def device_steps(args, batches, torch, device):
+    """Place the batches into one device pool and return (steps, byte counts, pool)."""
+    from paged_kv_cache_370_b200 import abi
+    from paged_kv_cache_370_b200.step import DecodeStep
+    if batches is None:
+        return shared_prompt_steps(args, torch, device)
+    b0 = batches[0]
+    shape = (b0.num_blocks, b0.num_kv_heads, b0.block_size, b0.head_dim)
+    tdt = torch.bfloat16 if b0.dtype == "bf16" else torch.float16
+    kc = torch.zeros(shape, dtype=tdt, device=device)
+    vc = torch.zeros(shape, dtype=tdt, device=device)
+    steps, infos = [], []
+    for b in batches:
+        slots = abi.pa_slot_mapping(b.block_tables, b.context_lens, b.block_size)
+        hist, new = b.history_rows(), b.new_token_rows()
+        k_all, v_all = to_dev(b.k, b.dtype, torch, device), to_dev(b.v, b.dtype, torch, device)
+        hidx = torch.from_numpy(hist).to(device)
+        abi.pa_reshape_and_cache(k_all[hidx].contiguous(), v_all[hidx].contiguous(),
+                                 torch.from_numpy(slots[hist]).to(device), kc, vc)
+        nidx = torch.from_numpy(new).to(device)
+        step = DecodeStep(k_cache=kc, v_cache=vc, q=to_dev(b.q, b.dtype, torch, device),
+                          k_new=k_all[nidx].contiguous(), v_new=v_all[nidx].contiguous(),
+                          slot_mapping=torch.from_numpy(slots[new]).to(device),
+                          block_tables=torch.from_numpy(b.block_tables).to(device),
+                          context_lens=torch.from_numpy(b.context_lens).to(device),
+                          max_context_len=b.max_context_len, scale=float(b.scale),
+                          partition_tokens=args.partition_tokens)
+        del k_all, v_all
+        steps.append(step)
+        infos.append(_byte_info(b.context_lens, b.num_q_heads, b.num_kv_heads, b.head_dim,
+                                b.block_size, step.partition, b.num_seqs))
+    torch.cuda.synchronize()
+    return steps, infos
+
+
+def _byte_info(lens, hq, hkv, d, bs, pt, ntok):
+    return {"decode": decode_step_bytes(lens, hq, hkv, d, bs),
+            "scratch": split_scratch_bytes(lens, hq, d, pt),
+            "write": new_token_bytes(ntok, hkv, d), "lens": np.asarray(lens)}
+
+
+def shared_prompt_steps(args, torch, device):
+    from paged_kv_cache_370_b200 import abi
+    from paged_kv_cache_370_b200.step import DecodeStep
+    s = synth.shared_prompt()
+    mgr = abi.BlockManager(s.num_blocks, s.block_size)
+    shape = (s.num_blocks, s.num_heads, s.block_size, s.head_dim)
+    kc = torch.zeros(shape, dtype=torch.float16, device=device)
+    vc = torch.zeros(shape, dtype=torch.float16, device=device)
+    slots, rows_k, rows_v = [], [], []
+    for i in range(s.num_prompts):
+        p0, p1, p2, p3 = (4 * i + j for j in range(4))
+        mgr.add_seq(p0, s.prompt_len)
+        slots.extend(mgr.seq_slots(p0, 0, s.prompt_len).tolist())
+        rows_k.append(s.prompt_k[i])
+        rows_v.append(s.prompt_v[i])
+        mgr.fork(p0, p1)
+        mgr.fork(p0, p2)
+        for _ in range(int(s.n_before_fork[i])):
+            slots.append(mgr.append_slot(p1)[0])
+        rows_k.append(s.gen_k[i][1])
+        rows_v.append(s.gen_v[i][1])
+        mgr.fork(p1, p3)
+        for seq, j, n in ((p0, 0, s.n_after[i, 0]), (p2, 2, s.n_after[i, 1])):
+            for _ in range(int(n)):
+                slots.append(mgr.append_slot(seq)[0])
+            rows_k.append(s.gen_k[i][j])
+            rows_v.append(s.gen_v[i][j])
+    abi.pa_reshape_and_cache(to_dev(np.concatenate(rows_k), "f16", torch, device),
+                             to_dev(np.concatenate(rows_v), "f16", torch, device),
+                             torch.tensor(slots, dtype=torch.int64, device=device), kc, vc)
+    new_slots, pairs = [], []
+    ids = [4 * i + j for i in range(s.num_prompts) for j in range(4)]
+    for sid in ids:
+        slot, src, dst = mgr.append_slot(sid)
+        new_slots.append(slot)
+        if src >= 0:
+            pairs.append((src, dst))
+    tables, lens = mgr.fill_tables(ids, 48, pad=0)
+    step = DecodeStep(k_cache=kc, v_cache=vc, q=to_dev(s.q, "f16", torch, device),
+                      k_new=to_dev(s.new_k, "f16", torch, device),
+                      v_new=to_dev(s.new_v, "f16", torch, device),
+                      slot_mapping=torch.tensor(new_slots, dtype=torch.int64, device=device),
+                      block_tables=torch.from_numpy(tables).to(device),
+                      context_lens=torch.from_numpy(lens).to(device),
+                      max_context_len=int(lens.max()), scale=float(s.scale),
+                      partition_tokens=args.partition_tokens,
+                      copy_pairs=torch.tensor(pairs, dtype=torch.int64, device=device))
+    torch.cuda.synchronize()
+    info = _byte_info(lens, 40, 40, 128, 16, step.partition, len(ids))
+    info["copy"] = 2 * 2 * len(pairs) * 40 * 16 * 128 * 2
+    return [step], [info]
+
+
+# ------------------------------------------------------------------------------ timing (GPU)
+def rank_aggregate(ms: float, nbytes: float, dist, device=None):
+    """Whole-job numbers: the slowest rank's time and the bytes all ranks moved."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    b = torch.tensor([nbytes], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(b.item())
+
+
+def capture(fn, torch):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm the launch path outside capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def run_ours(args, rank, world, local, dist):
+    import torch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    batches = make_batches(args, rank)
+    steps, infos = device_steps(args, batches, torch, device)
+    pt = steps[0].partition
+    # graphs: [copies + write] and [decode (+ merge)] per batch
+    g_write = [capture(lambda s=s: (s.copy(), s.write()), torch) for s in steps]
+    g_dec = [capture(lambda s=s: s.attend(), torch) for s in steps]
+    V = len(steps)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    for i in range(args.warmup):
+        g_write[i % V].replay()
+        g_dec[i % V].replay()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    props = torch.cuda.get_device_properties(device)
+    bus = getattr(props, "pci_bus_id", None)
+    bus_str = None
+    if isinstance(bus, int):
+        bus_str = f"{getattr(props, 'pci_domain_id', 0):08x}:{bus:02x}:" \
+                  f"{getattr(props, 'pci_device_id', 0):02x}.0"
+    sampler = ClockSampler(bus_str)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    t0 = time.time()
+    for i in range(K):
+        e = ev[i]
+        e[0].record(stream)
+        g_write[i % V].replay()
+        e[1].record(stream)
+        g_dec[i % V].replay()
+        e[2].record(stream)
+    barrier()
+    t1 = time.time()
+    time.sleep(0.2)
+    sampler.stop()
+    total_ms = ev[0][0].elapsed_time(ev[K - 1][2])
+    dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    wr_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    step_bytes = [infos[i % V]["decode"]["total"] for i in range(K)]
+    total_ms_max, all_bytes = rank_aggregate(total_ms, float(sum(step_bytes)), dist, device)
+    ms_per_step = total_ms_max / K
+    gbs = all_bytes / (total_ms_max * 1e-3) / 1e9
+    q_tok = sum(len(infos[i % V]["lens"]) for i in range(K)) * world / (total_ms_max * 1e-3)
+
+    peak, peak_kind = measured_peaks()
+    dec_avg_ms = float(np.mean(dec_ms))
+    dec_bytes = float(np.mean(step_bytes))
+    achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
+    traffic = recorded_traffic() if args.workload == "llama8b" else None
+    launches = sum(s.launches() for s in (steps[i % V] for i in range(K)))
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, steps, infos, torch, device, dist, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and batches is not None:
+        cpu = cpu_baseline(batches[0], args.cpu_seconds)
+    clocks = sampler.summary(t0, t1)
+    res = {
+        "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype":
+            "bf16" if (batches and batches[0].dtype == "bf16") else "f16",
+        "data": "synthetic (seeded N(0,1) K/V/q, random block tables)",
+        "config": workload_config(args, batches, pt),
+        "query_tokens_per_s": round(q_tok, 1),
+        "pct_of_hbm_measured": round(100 * gbs / world / peak, 2),
+        "pct_of_hbm_nominal_8tbs": round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
+        "roofline": {"bound": "hbm", "kernel": "pa_decode (partition kernel + LSE merge)",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": int(dec_bytes),
+                     "avg_launch_ms": round(dec_avg_ms, 5),
+                     "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4)},
+        "kernel_ms": {"write(+copy)": round(float(np.mean(wr_ms)), 5),
+                      "decode": round(dec_avg_ms, 5)},
+        "extra_bytes_per_step": {"split_scratch": int(np.mean([infos[i % V]["scratch"]
+                                                               for i in range(K)])),
+                                 "kv_write": int(infos[0]["write"]),
+                                 "copy_on_write": int(infos[0].get("copy", 0))},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        res["e2e"] = e2e
+    if cpu is not None:
+        res["cpu_baseline"] = cpu
+    return res
+
+
+def run_e2e(args, steps, infos, torch, device, dist, world):
+    """The same steps fed from pinned host buffers, output copied back, graph-replayed."""
+    from paged_kv_cache_370_b200.step import HostDecodeStep
+    hsteps = []
+    for s in steps:
+        hsteps.append(HostDecodeStep(k_cache=s.k_cache, v_cache=s.v_cache, q=s.q, k_new=s.k_new,
+                                     v_new=s.v_new, slot_mapping=s.slot_mapping,
+                                     block_tables=s.block_tables, context_lens=s.context_lens,
+                                     max_context_len=s.max_context_len, scale=s.scale,
+                                     partition_tokens=s.partition_tokens,
+                                     copy_pairs=s.copy_pairs))
+    graphs = [capture(h.run, torch) for h in hsteps]
+    V = len(graphs)
+    for i in range(args.warmup):
+        graphs[i % V].replay()
+    K = args.steps
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(K):
+        graphs[i % V].replay()
+    b.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    my_bytes = sum(infos[i % V]["decode"]["total"] for i in range(K))
+    ms, total = rank_aggregate(a.elapsed_time(b), float(my_bytes), dist, device)
+    return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms / K, 5),
+            "h2d_bytes_per_step": int(np.mean([hsteps[i % V].h2d_bytes for i in range(K)])),
+            "d2h_bytes_per_step": int(hsteps[0].d2h_bytes),
+            "how": "pinned host inputs copied in and output copied out every step, "
+                   "graph-replayed through the library's HostDecodeStep"}
+
+
+# --------------------------------------------------------------------------- CPU (oracle)
+def _oracle_setup(batch):
+    import oracle
+    shape = (batch.num_blocks, batch.num_kv_heads, batch.block_size, batch.head_dim)
+    kp = np.zeros(shape, dtype=np.uint16)
+    vp = np.zeros(shape, dtype=np.uint16)
+    oracle.place_history(batch, kp, vp, include_new=True)
+    return kp, vp
+
+
+def _oracle_pass(batch, kp, vp, seqs, threads=0):
+    import oracle
+    return oracle.decode(np.ascontiguousarray(batch.q[seqs]), kp, vp,
+                         np.ascontiguousarray(batch.block_tables[seqs]),
+                         np.ascontiguousarray(batch.context_lens[seqs]), batch.scale,
+                         batch.dtype, num_threads=threads)
+
+
+def cpu_baseline(batch, target_s):
+    """The oracle, as it stands, on whole sequences of the batch for about target_s seconds."""
+    import oracle
+    kp, vp = _oracle_setup(batch)
+    cores = oracle.max_threads()
+    order = np.arange(batch.num_seqs)
+    done, nbytes, t_used, passes = 0, 0, 0.0, 0
+    while t_used < target_s and passes < 64:
+        seqs = order[done % batch.num_seqs: done % batch.num_seqs + 8]
+        t = time.perf_counter()
+        _oracle_pass(batch, kp, vp, seqs)
+        t_used += time.perf_counter() - t
+        nbytes += decode_step_bytes(batch.context_lens[seqs], batch.num_q_heads,
+                                    batch.num_kv_heads, batch.head_dim,
+                                    batch.block_size)["total"]
+        done += len(seqs)
+        passes += 1
+    return {"value": round(nbytes / t_used / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{done} sequences of the batch (8 per call, {passes} calls, "
+                      f"{t_used:.1f} s), fp64, OpenMP over (sequence, q head)",
+            "query_tokens_per_s": round(done / t_used, 2)}
+
+
+def run_reference(args, rank, world):
+    import oracle
+    batches = make_batches(args, rank)
+    if batches is None:
+        return {"impl": "reference", "unavailable": "the oracle arm covers the random-table "
+                "workloads only"}
+    batch = batches[0]
+    kp, vp = _oracle_setup(batch)
+    cores = oracle.max_threads()
+    # size the per-step sample so the whole run stays within about two minutes
+    t = time.perf_counter()
+    _oracle_pass(batch, kp, vp, np.arange(1))
+    one = max(time.perf_counter() - t, 1e-4)
+    per_step_budget = 120.0 / max(1, args.steps + args.warmup)
+    nseq = int(max(1, min(batch.num_seqs, per_step_budget / one)))
+    for i in range(args.warmup):
+        _oracle_pass(batch, kp, vp, (np.arange(nseq) + i * nseq) % batch.num_seqs)
+    total_t, total_b, total_q = 0.0, 0, 0
+    for i in range(args.steps):
+        seqs = (np.arange(nseq) + i * nseq) % batch.num_seqs
+        t = time.perf_counter()
+        _oracle_pass(batch, kp, vp, seqs)
+        total_t += time.perf_counter() - t
+        total_b += decode_step_bytes(batch.context_lens[seqs], batch.num_q_heads,
+                                     batch.num_kv_heads, batch.head_dim,
+                                     batch.block_size)["total"]
+        total_q += nseq
+    gbs = total_b / total_t / 1e9
+    cfg = workload_config(args, batches, 0)
+    return {"metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "impl": "reference",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total_t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": cfg,
+            "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{nseq} of {batch.num_seqs} sequences per step"},
+            "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "query_tokens_per_s": round(total_q / total_t, 2)}
+
+
+# ------------------------------------------------------------------------------------- main
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+    dist = None
+    if world > 1:
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    try:
+        res = run_ours(args, rank, world, local, dist)
+    finally:
+        if dist is not None:
+            dist.barrier()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

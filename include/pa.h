@@ -1,0 +1,226 @@
+/*
+ * pa.h -- C ABI of the paged decode attention library (libpa370.so).
+ *
+ * What the library computes is defined by three web pages on vLLM's
+ * PagedAttention:
+ *   [P1] "大语言模型推理内存管理算法 paged attention"
+ *        (https://www.cnblogs.com/wljss/p/20424559)
+ *   [P2] "PagedAttention 核心思想解析"
+ *        (https://intelliparadigm.com/article/weixin_29574585/2267096)
+ *   [P3] "08. PagedAttention：把 KV Cache 分页管理"
+ *        (https://niuwancheng.cn/blog/docs/ai/llm-inference/08-paged-attention.html)
+ *
+ * Conventions shared by every entry point:
+ *  - Device operations take raw device pointers owned by the caller and
+ *    enqueue work on `stream` (a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream). They never synchronise the host and never
+ *    allocate device memory; split-context scratch is the caller's
+ *    `workspace`.
+ *  - Shapes and dtypes are checked on the host before any launch; a bad
+ *    argument returns PA_ERR_INVALID and launches nothing. A failed launch
+ *    returns PA_ERR_CUDA.
+ *  - Data that only the device sees (block ids, slots, lengths) is checked
+ *    by the kernels themselves: an out-of-range value skips the access that
+ *    would have used it and sets a bit in a device-side error word, which
+ *    pa_device_status() reads. A kernel never faults on such input; its
+ *    output is then undefined.
+ *  - KV pool layout (the pages fix none; this library's contract): K and V
+ *    are separate pools of shape [num_blocks][num_kv_heads][block_size]
+ *    [head_dim], row-major, elements fp16 or bf16. One (block, kv head)
+ *    tile is block_size * head_dim contiguous elements. The pools must be
+ *    16-byte aligned.
+ *  - A slot names one token position of the pool: slot = physical_block *
+ *    block_size + offset_in_block [P3, section "为什么叫 PagedAttention"].
+ *  - Query head h attends with KV head h / (num_q_heads / num_kv_heads)
+ *    (grouped-query attention [P1, section 6]).
+ */
+#ifndef PA370_H
+#define PA370_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID = -1,       /* bad argument (shape, dtype, pointer, alignment) */
+    PA_ERR_OUT_OF_BLOCKS = -2, /* allocator: not enough free blocks; nothing changed */
+    PA_ERR_STATE = -3,         /* allocator: unknown/duplicate sequence, bad reference count */
+    PA_ERR_CUDA = -4,          /* a CUDA runtime call failed */
+    PA_ERR_UNSUPPORTED = -5    /* valid but not compiled in (e.g. a head_dim/group combination) */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the device-side error word (see pa_device_status). */
+#define PA_DEVERR_BLOCK_ID 1     /* a block table entry was outside [0, num_blocks) */
+#define PA_DEVERR_SLOT 2         /* a slot was >= num_blocks * block_size */
+#define PA_DEVERR_COPY_PAIR 4    /* a copy pair named a block outside the pool */
+#define PA_DEVERR_CONTEXT_LEN 8  /* a context length exceeded the table or max_context_len */
+#define PA_DEVERR_TIMEOUT 16     /* a pipeline wait gave up (the kernel returned early) */
+
+/* ------------------------------------------------------------------------------------------
+ * pa_reshape_and_cache -- store the K and V of new tokens at their slots.
+ * [P3, section "为什么叫 PagedAttention": a new token's K and V are written to
+ * the position of the physical block it belongs to; slot = block_table[logical
+ * block] * block_size + offset, then a small GPU kernel writes each token's K/V
+ * to its slot.]
+ *
+ *   k_new, v_new   device, [num_tokens][num_kv_heads][head_dim], dtype, contiguous
+ *   slot_mapping   device, int64 [num_tokens]; a negative slot marks padding and
+ *                  is skipped; slots must be distinct (duplicates: undefined)
+ *   k_cache, v_cache  device pools (layout above), updated in place
+ * Bit-exact element copy. Returns PA_OK (num_tokens == 0 launches nothing).
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_reshape_and_cache(const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                               int num_tokens, void *k_cache, void *v_cache, int num_blocks,
+                               int num_kv_heads, int block_size, int head_dim, pa_dtype dtype,
+                               void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * pa_copy_blocks -- the device half of copy-on-write.
+ * [P2, section 2.3: when a sequence must modify a shared block, a new
+ * physical block is allocated, the original block's contents are copied
+ * into it, the block table is updated and the old block's ref_count drops;
+ * P1, section 9.]
+ *
+ *   block_pairs   device, int64 [num_pairs][2] = (src, dst) physical ids
+ * For each pair the whole block -- every KV head, every slot, K and V -- is
+ * copied bit-exactly. Destinations must be distinct and no destination may
+ * be a source of another pair (undefined otherwise); src == dst is a no-op.
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_pairs, int num_pairs,
+                         int num_blocks, int num_kv_heads, int block_size, int head_dim,
+                         pa_dtype dtype, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * pa_decode -- paged attention for one query token per sequence.
+ * [P1, section 5: out = softmax(Q K^T / sqrt(d)) V, where the kernel finds
+ * each token's logical block and maps it through the block table to the
+ * physical block holding its K/V; section 6: the formula is unchanged by
+ * paging. P3, section "它没有解决什么": each decode step reads the whole
+ * history. P2, section 2.2: scores are computed per KV block and the partial
+ * results merged.]
+ *
+ *   out            device, [num_seqs][num_q_heads][head_dim], dtype; rounded to
+ *                  nearest-even from fp32
+ *   q              device, [num_seqs][num_q_heads][head_dim], dtype
+ *   block_tables   device, int32 [num_seqs][max_blocks_per_seq]; entries past
+ *                  ceil(context_lens[b] / block_size) are never read
+ *   context_lens   device, int32 [num_seqs]; tokens of each sequence to attend
+ *                  over (including the one just written); 0 yields zeros
+ *   max_context_len  host int >= every context_lens[b] (sizes the grid; no
+ *                  device-to-host read is made)
+ *   scale          softmax scale, normally 1/sqrt(head_dim)
+ *   workspace      device scratch of at least pa_decode_workspace_size() bytes
+ *                  (same arguments), 16-byte aligned; may be NULL when that
+ *                  size is 0. Contents need no initialisation and are
+ *                  overwritten; two calls that share a workspace must not
+ *                  overlap on the device
+ *   partition_tokens  tokens per split-context partition (a positive multiple
+ *                  of 64, at most 8192), or 0 for the library's choice
+ *                  (pa_decode_default_partition)
+ * Supported: head_dim in {64, 128}; num_q_heads / num_kv_heads in {1,2,4,8};
+ * any block_size >= 1 with partition_tokens / block_size <= 4094. Sequences longer than one partition
+ * are processed as several partitions whose (max, sum, weighted V) states
+ * are merged by log-sum-exp in a second kernel on the same stream.
+ * ------------------------------------------------------------------------------------------ */
+size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                int max_context_len, int partition_tokens);
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, int max_blocks_per_seq,
+                    const int32_t *context_lens, int max_context_len, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, float scale, pa_dtype dtype, void *workspace,
+                    size_t workspace_bytes, int partition_tokens, void *stream);
+
+/* The partition size pa_decode uses for partition_tokens == 0. */
+int pa_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_len);
+
+/* ------------------------------------------------------------------------------------------
+ * pa_device_status -- read and clear the device-side error word (PA_DEVERR_*
+ * bits) after the work queued on `stream` has finished. Synchronises
+ * `stream`; meant for tests and debugging, not the hot path.
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_device_status(void *stream, int32_t *code);
+
+/* Human-readable name of a status code (static storage). */
+const char *pa_status_string(pa_status status);
+
+/* ------------------------------------------------------------------------------------------
+ * pa_slot_mapping -- host helper: the slot of every position [0, count) of
+ * each sequence, from its block table (for writing a prompt's K/V).
+ * [P3, section "为什么叫 PagedAttention", slot formula.]
+ *   block_tables  host int32 [num_seqs][max_blocks_per_seq]
+ *   counts        host int32 [num_seqs]: positions to map per sequence
+ *   slots         host int64 output, sum(counts) entries, sequence-major
+ * Returns PA_ERR_INVALID if a count exceeds the table width.
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_slot_mapping(const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *counts, int num_seqs, int block_size, int64_t *slots);
+
+/* ==========================================================================================
+ * Host-side block manager (off the hot path; not thread-safe; one per pool).
+ * [P1, sections 7-8: blocks are allocated on demand -- a new one only when the
+ * last block is full -- and returned to a free list when the request ends, for
+ * immediate reuse. P3, section "借用操作系统的办法：分页": same; section
+ * "分页还顺带解决了什么": blocks shared by several tables carry a reference
+ * count. P2, section 2.3: copy-on-write. P2, section 5.1: forking sampled
+ * sequences from a shared prompt.]
+ * Which free block is handed out is not part of the contract.
+ * ========================================================================================== */
+typedef struct pa_alloc pa_alloc;
+
+pa_status pa_alloc_create(int num_blocks, int block_size, pa_alloc **out);
+void pa_alloc_destroy(pa_alloc *a);
+
+/* New sequence holding num_tokens tokens (a prompt): ceil(num_tokens / block_size)
+ * blocks, all or none (PA_ERR_OUT_OF_BLOCKS leaves the state unchanged). */
+pa_status pa_alloc_add_seq(pa_alloc *a, int64_t seq_id, int num_tokens);
+
+/* child shares every block of parent (each block's ref_count += 1). */
+pa_status pa_alloc_fork(pa_alloc *a, int64_t parent, int64_t child);
+
+/* Reserve the slot of the sequence's next token and advance its length.
+ * Takes a new block when the last one is full. If the block to be written is
+ * shared (ref_count > 1) it is copied on write: a new block replaces it in
+ * this table, the old one loses a reference, and (*cow_src, *cow_dst) name
+ * the copy the caller must run (pa_copy_blocks) before writing the slot;
+ * otherwise both are -1. On PA_ERR_OUT_OF_BLOCKS nothing changes. */
+pa_status pa_alloc_append_slot(pa_alloc *a, int64_t seq_id, int64_t *slot, int64_t *cow_src,
+                               int64_t *cow_dst);
+
+/* Slots of existing positions [start, start + count) of a sequence. */
+pa_status pa_alloc_seq_slots(const pa_alloc *a, int64_t seq_id, int start, int count,
+                             int64_t *slots);
+
+/* Drop the sequence: each block loses a reference; blocks reaching zero go
+ * back on the free list. */
+pa_status pa_alloc_free_seq(pa_alloc *a, int64_t seq_id);
+
+/* Copy the sequence's block table into out[0 .. cap); report its block and
+ * token counts (either pointer may be NULL). PA_ERR_INVALID if cap is short. */
+pa_status pa_alloc_block_table(const pa_alloc *a, int64_t seq_id, int32_t *out, int cap,
+                               int *num_blocks, int *num_tokens);
+
+/* Fill a padded [n][max_blocks_per_seq] table and the lengths for a batch of
+ * sequences; unused entries get `pad`. */
+pa_status pa_alloc_fill_tables(const pa_alloc *a, const int64_t *seq_ids, int n,
+                               int32_t *block_tables, int max_blocks_per_seq, int32_t pad,
+                               int32_t *context_lens);
+
+pa_status pa_alloc_ref_count(const pa_alloc *a, int32_t block, int *ref_count);
+
+/* Free blocks; token slots that hold a token; allocated slots that do not
+ * (the unfilled tails of last blocks [P1, section 4; P3, section "浪费降到了多少"]). */
+pa_status pa_alloc_stats(const pa_alloc *a, int *free_blocks, int64_t *used_tokens,
+                         int64_t *wasted_tokens);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PA370_H */
