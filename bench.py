@@ -67,6 +67,8 @@ def parse_args():
     ap.add_argument("--block-size", type=int, default=16, help="block size of the mixed workload")
     ap.add_argument("--variants", type=int, default=4, help="batches rotated (llama8b)")
     ap.add_argument("--partition-tokens", type=int, default=0)
+    ap.add_argument("--pool-blocks", type=int, default=65536,
+                    help="llama8b pool size (smaller for profiler captures)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -169,7 +171,8 @@ def make_batches(args, rank):
     seed_shift = 1_000_003 * rank
     if args.workload == "llama8b":
         return [synth.llama8b(seed=synth.SEED_BASE + 2 + seed_shift, variant=v,
-                              num_variants=args.variants) for v in range(args.variants)]
+                              num_variants=args.variants, num_blocks=args.pool_blocks)
+                for v in range(args.variants)]
     if args.workload == "long_skew":
         return [synth.long_skew(seed=synth.SEED_BASE + 3 + seed_shift)]
     if args.workload == "mixed":

@@ -399,34 +399,37 @@ __global__ void __launch_bounds__(kThreads, 3)
 
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % kStages;
-    if (!mbar_wait_bounded(&full_bar[s], (i / kStages) & 1, abort_flag)) break;
+    // every lane waits; the warp then leaves together or not at all, so the
+    // warp-wide shuffles below always see all 32 lanes
+    const bool landed = mbar_wait_bounded(&full_bar[s], (i / kStages) & 1, abort_flag);
+    if (!__all_sync(0xffffffffu, landed)) break;
     const unsigned char *stage = smem + s * L::kStageBytes;
     const uint4 *Ks = reinterpret_cast<const uint4 *>(stage);
     const uint4 *Vs = reinterpret_cast<const uint4 *>(stage + kTileBytes);
     const int nvalid = min(TILE, t_end - (t_begin + i * TILE));
     const int tbase = grp * TPG;
 
-    // scores of this group's tokens (head hh), log2 units; -inf when masked
+    // scores of this group's tokens (head hh), log2 units; -inf when masked.
+    // The shuffles run for every token slot in every lane (a slot past the
+    // valid rows reads stale but in-bounds stage memory and is then masked
+    // by a select), so no shuffle is ever issued by part of a warp.
     float sc[TPG];
 #pragma unroll
     for (int j = 0; j < TPG; ++j) {
       const int t = tbase + j;
-      if (t < nvalid) {
-        float kf[CH];
-        Elem<T>::to_f32(Ks[t * (D / CH) + c], kf);
-        float part[G];
+      float kf[CH];
+      Elem<T>::to_f32(Ks[t * (D / CH) + c], kf);
+      float part[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float a = 0.f;
+      for (int h = 0; h < G; ++h) {
+        float a = 0.f;
 #pragma unroll
-          for (int e = 0; e < CH; ++e) a = fmaf(qf[h][e], kf[e], a);
-          part[h] = a;
-        }
-        HalvingSum<G, LPT / 2>::run(part, lane);
-        sc[j] = butterfly_sum<LPT / (2 * G)>(part[0]) * p.scale_log2;
-      } else {
-        sc[j] = -INFINITY;
+        for (int e = 0; e < CH; ++e) a = fmaf(qf[h][e], kf[e], a);
+        part[h] = a;
       }
+      HalvingSum<G, LPT / 2>::run(part, lane);
+      const float sj = butterfly_sum<LPT / (2 * G)>(part[0]) * p.scale_log2;
+      sc[j] = (t < nvalid) ? sj : -INFINITY;
     }
     float m_tile = sc[0];
 #pragma unroll

@@ -160,13 +160,15 @@ def tiny(seed: int = SEED_BASE + 1) -> DecodeBatch:
 
 
 def llama8b(seed: int = SEED_BASE + 2, variant: int = 0, num_variants: int = 1,
-            num_seqs: int = 64) -> DecodeBatch:
+            num_seqs: int = 64, num_blocks: int = 65536) -> DecodeBatch:
     """Llama-3.1-8B-shaped single-layer decode batch: 64 sequences, 32 q / 8 KV
     heads, head_dim 128, bf16, 16-token blocks, lengths uniform in
     [128, 2048], one 65,536-block pool. ``variant`` selects one of
     ``num_variants`` batches that draw disjoint block ids from the same
-    pool (so several batches can live in one pool at once)."""
-    bs, nb, lo, hi = 16, 65536, 128, 2048
+    pool (so several batches can live in one pool at once). A smaller
+    ``num_blocks`` shrinks the pool (for profiler captures) without changing
+    the batch's lengths or values."""
+    bs, nb, lo, hi = 16, num_blocks, 128, 2048
     width = _table_width(hi, bs)
     pool_rng = np.random.default_rng(seed)
     perm = pool_rng.permutation(nb)
