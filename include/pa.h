@@ -138,6 +138,39 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     int num_blocks, float scale, pa_dtype dtype, void *workspace,
                     size_t workspace_bytes, int partition_tokens, void *stream);
 
+/* ------------------------------------------------------------------------------------------
+ * pa_decode_static_workspace -- pa_decode for callers that cannot allocate device
+ * memory. (The pages have no counterpart: this is a deployment convenience.)
+ *
+ * Some callers have no way to obtain device scratch: code that runs where a
+ * cudaMalloc would break a memory budget or an allocator they do not own (a
+ * host framework's pooled allocator, a plug-in restricted to the buffers it is
+ * handed), or that must not allocate on a latency-critical path. This entry
+ * point takes the same arguments as pa_decode minus the workspace: the
+ * split-context scratch is a fixed device array of PA_STATIC_WORKSPACE_BYTES
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits. The caller still passes q, the pools, the tables, the lengths
+ * and the output.
+ *  - Calls that would need more scratch than PA_STATIC_WORKSPACE_BYTES (see
+ *    pa_decode_workspace_size) return PA_ERR_UNSUPPORTED and launch nothing.
+ *  - The first call on a device (made with that device current) looks up the
+ *    array's device address; make that first call before any stream capture.
+ *  - No device memory is allocated or freed, by this library or any other.
+ *  - All calls share the one array and it keeps the last call's contents. It
+ *    needs no clearing (each call writes every entry it later reads), but calls
+ *    whose work overlaps on the GPU (other streams, other host threads) race on
+ *    it: serialise them.
+ * ------------------------------------------------------------------------------------------ */
+#define PA_STATIC_WORKSPACE_BYTES (16u << 20)
+
+pa_status pa_decode_static_workspace(void *out, const void *q, const void *k_cache,
+                                     const void *v_cache, const int32_t *block_tables,
+                                     int max_blocks_per_seq, const int32_t *context_lens,
+                                     int max_context_len, int num_seqs, int num_q_heads,
+                                     int num_kv_heads, int head_dim, int block_size,
+                                     int num_blocks, float scale, pa_dtype dtype,
+                                     int partition_tokens, void *stream);
+
 /* The partition size pa_decode uses for partition_tokens == 0. */
 int pa_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_len);
 

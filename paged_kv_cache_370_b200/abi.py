@@ -32,6 +32,8 @@ PA_DEVERR_COPY_PAIR = 4
 PA_DEVERR_CONTEXT_LEN = 8
 PA_DEVERR_TIMEOUT = 16
 
+PA_STATIC_WORKSPACE_BYTES = 16 << 20
+
 
 class PAError(RuntimeError):
     def __init__(self, status: int, what: str):
@@ -55,6 +57,7 @@ def _load() -> ctypes.CDLL:
         "pa_decode_workspace_size": (sz, [i, i, i, i, i, i]),
         "pa_decode": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, P, sz, i, P]),
         "pa_decode_default_partition": (i, [i, i, i]),
+        "pa_decode_static_workspace": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P]),
         "pa_device_status": (i, [P, P]),
         "pa_status_string": (ctypes.c_char_p, [i]),
         "pa_slot_mapping": (i, [P, i, P, i, i, P]),
@@ -173,6 +176,22 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
                         _dtype_code(q), _dev_ptr(workspace, "workspace"), ws_bytes,
                         int(partition_tokens), _stream(stream))
     _check(st, "pa_decode")
+
+
+def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_lens,
+                               max_context_len, scale, partition_tokens=0, stream=None):
+    """pa_decode for callers that cannot allocate device memory: the split-context
+    scratch is the library's fixed device array (PA_STATIC_WORKSPACE_BYTES), shared
+    by every call. Raises PAError(PA_ERR_UNSUPPORTED) if the call needs more."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    st = _lib.pa_decode_static_workspace(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+        int(block_tables.shape[1]), _dev_ptr(context_lens, "context_lens"), int(max_context_len),
+        B, hq, hkv, d, bs, nb, float(scale), _dtype_code(q), int(partition_tokens),
+        _stream(stream))
+    _check(st, "pa_decode_static_workspace")
 
 
 def pa_device_status(stream=None) -> int:
