@@ -34,11 +34,13 @@
 //  * Every wait is bounded in wall-clock time; a block id or length out of
 //    range is skipped and reported in the device error word, never accessed.
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "pa.h"
 #include "pa_internal.h"
@@ -566,6 +568,412 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
 }
 
+// ===================================================================== tensor-core variant
+// pa_decode_tc_kernel: the same partition work as pa_decode_partition_kernel, with
+// the q-group x K-tile and weights x V-tile products on tensor cores.
+//  * The producer warp stages each (block, kv head) piece with 2-D TMA tensor
+//    copies (cp.async.bulk.tensor, 128-byte swizzle, no multicast) into
+//    1024-byte-aligned panels of 64 head_dim columns x 64 tokens, so ldmatrix
+//    reads them without bank conflicts.
+//  * Each consumer warp owns 16 tokens of a 64-token tile and computes
+//    S^T = K_tile . Q^T with mma.m16n8k16 (tokens are M, the GQA group padded
+//    to 8 is N, head_dim is K). Its score fragment, turned into the weights P
+//    and transposed in registers with movmatrix, is directly the B operand of
+//    O^T += V_tile^T . P (head_dim is M), so weights never touch shared memory.
+//  * Weights are rounded to the input type for the product and the running
+//    sum uses the same rounded values, so the result is an exact weighted
+//    average of V with weights perturbed by at most one rounding.
+//  * The running output is only rescaled when some head's max grew.
+// Requires a power-of-two block size >= 8 (every TMA box then starts on a
+// 1024-byte boundary and blocks align with 64-token tiles).
+namespace tc {
+
+constexpr int kTile = 64;            // tokens per stage
+constexpr int kWarps = 4;            // consumer warps, 16 tokens each
+constexpr int kThreads = (kWarps + 1) * 32;
+constexpr int kPanelBytes = kTile * 128;  // 64 columns of 2 bytes x 64 rows
+
+template <int D>
+struct Cfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kStageBytes = 2 * kPanels * kPanelBytes;  // K panels then V panels
+  static constexpr int kStages = D == 128 ? 3 : 4;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kBarOffset = kRingBytes;
+  static constexpr int kMlOffset = kBarOffset + 2 * kStages * 8;
+  static constexpr int kFlagOffset = kMlOffset + kWarps * 8 * 2 * 4;
+  static constexpr int kTableOffset = kFlagOffset + 16;
+  static constexpr int kCtasPerSm = D == 128 ? 2 : 3;
+  static size_t bytes(int table_slice) { return 1024 + kTableOffset + (size_t)table_slice * 4; }
+  static_assert(kWarps * 8 * D * 4 <= kRingBytes, "merge buffer must fit in the ring");
+};
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+template <typename T>
+struct Mma;
+
+template <>
+struct Mma<__nv_bfloat16> {
+  static __device__ __forceinline__ void run(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
+        " {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  // two floats -> packed pair (lo in the low half) and the rounded values back
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi, float &rlo, float &rhi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    rlo = __low2float(v);
+    rhi = __high2float(v);
+    return *reinterpret_cast<uint32_t *>(&v);
+  }
+};
+
+template <>
+struct Mma<__half> {
+  static __device__ __forceinline__ void run(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                             uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
+        " {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+  static __device__ __forceinline__ uint32_t pack(float lo, float hi, float &rlo, float &rhi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    rlo = __low2float(v);
+    rhi = __high2float(v);
+    return *reinterpret_cast<uint32_t *>(&v);
+  }
+};
+
+// byte address of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled panel
+__device__ __forceinline__ uint32_t swz(uint32_t panel, int row, int chunk) {
+  return panel + row * 128 + ((chunk ^ (row & 7)) << 4);
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, Cfg<D>::kCtasPerSm)
+    pa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+  using C = Cfg<D>;
+  constexpr int NS = C::kStages;
+  constexpr int KSTEPS = D / 16;
+
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  // the ring starts on a 1024-byte boundary (the 128-byte swizzle repeats every 1 KB)
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
+  uint64_t *empty_bar = full_bar + NS;
+  float *mlbuf = reinterpret_cast<float *>(smem + C::kMlOffset);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kFlagOffset);
+  int32_t *table = reinterpret_cast<int32_t *>(smem + C::kTableOffset);
+  const uint32_t ring = smem_u32(smem);
+
+  const int part = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  int len = __ldg(p.context_lens + b);
+  const int cap = p.max_blocks_per_seq * p.block_size;
+  if (len < 0 || len > cap || len > p.max_context_len) {
+    if (tid == 0 && part == 0 && kvh == 0) atomicOr(&g_decode_error, PA_DEVERR_CONTEXT_LEN);
+    len = len < 0 ? 0 : min(min(len, cap), p.max_context_len);
+  }
+  const int nparts = len > 0 ? (len + p.partition_tokens - 1) / p.partition_tokens : 1;
+  if (part >= nparts) return;
+  const int t_begin = part * p.partition_tokens;
+  const int t_end = min(len, t_begin + p.partition_tokens);
+  const int ntok = t_end - t_begin;
+  const int ntiles = (ntok + kTile - 1) / kTile;
+  const int bs = p.block_size;
+  const int box_rows = bs < kTile ? bs : kTile;
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kWarps);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  const int blk_first = t_begin / bs;
+  const int nblk = ntok > 0 ? (t_end - 1) / bs - blk_first + 1 : 0;
+  if (warp == kWarps) {
+    const int32_t *row = p.block_tables + (size_t)b * p.max_blocks_per_seq + blk_first;
+    for (int i = lane; i < nblk; i += 32) table[i] = __ldg(row + i);
+  }
+  __syncthreads();
+
+  if (warp == kWarps) {
+    // ================================================================== producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)));
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % NS;
+        if (i >= NS && !mbar_wait_bounded(&empty_bar[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
+        const int t0 = t_begin + i * kTile;
+        const int t1 = min(t0 + kTile, t_end);
+        const int blk0 = t0 / bs, blk1 = (t1 - 1) / bs;
+        uint32_t boxes = 0;
+        for (int blk = blk0; blk <= blk1; ++blk) {
+          const int phys = table[blk - blk_first];
+          if (phys < 0 || phys >= p.num_blocks) {
+            atomicOr(&g_decode_error, PA_DEVERR_BLOCK_ID);
+            continue;
+          }
+          ++boxes;
+        }
+        mbar_expect_tx_arrive(&full_bar[s], boxes * (uint32_t)(2 * C::kPanels * box_rows * 128));
+        const uint32_t stage = ring + s * C::kStageBytes;
+        for (int blk = blk0; blk <= blk1; ++blk) {
+          const int phys = table[blk - blk_first];
+          if (phys < 0 || phys >= p.num_blocks) continue;
+          // first row of the box inside its block, and where it lands in the tile
+          const int r0 = bs > kTile ? t0 - blk * bs : 0;
+          const int row = blk * bs + r0 - t0;
+          const int y = (phys * p.num_kv_heads + kvh) * bs + r0;
+#pragma unroll
+          for (int pn = 0; pn < C::kPanels; ++pn) {
+            tma_load_2d(stage + pn * kPanelBytes + row * 128, &tmap_k, pn * 64, y, &full_bar[s]);
+            tma_load_2d(stage + (C::kPanels + pn) * kPanelBytes + row * 128, &tmap_v, pn * 64, y,
+                        &full_bar[s]);
+          }
+        }
+        issued = i + 1;
+      }
+      for (int i = max(0, issued - NS); i < issued; ++i) {
+        const int s = i % NS;
+        const unsigned long long t_start = global_ns();
+        while (!mbar_try_wait(&full_bar[s], (i / NS) & 1)) {
+          if (global_ns() - t_start > kWaitLimitNs) {
+            atomicOr(&g_decode_error, PA_DEVERR_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ===================================================================== consumers
+  const int g = lane >> 2;  // fragment row group
+  const int t = lane & 3;   // thread in group: this lane's heads are 2t and 2t+1
+  const int hq0 = kvh * G;
+
+  // B operand of S^T = K . Q^T: Q^T[d][head], head = g (zero for padding heads)
+  uint32_t qb[KSTEPS][2];
+  {
+    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
+        static_cast<const T *>(p.q) + ((size_t)b * p.num_q_heads + hq0 + (g < G ? g : 0)) * D);
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      qb[kk][0] = g < G ? __ldg(qrow + (kk * 16 + 2 * t) / 2) : 0u;
+      qb[kk][1] = g < G ? __ldg(qrow + (kk * 16 + 8 + 2 * t) / 2) : 0u;
+    }
+  }
+
+  float o[KSTEPS][4];  // O^T fragments: rows d, columns heads 2t, 2t+1
+#pragma unroll
+  for (int mt = 0; mt < KSTEPS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2t, 2t+1 (log2 units)
+  float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums
+
+  const int wrow = warp * 16;  // first token of this warp in a tile
+  // per-lane ldmatrix row / chunk offsets
+  const int ld_row_k = wrow + (lane & 7) + 8 * ((lane >> 3) & 1);  // QK: A = K rows
+  const int ld_chk_k = lane >> 4;
+  const int ld_row_v = wrow + (lane & 7) + 8 * (lane >> 4);        // PV: A = V^T
+  const int ld_chk_v = (lane >> 3) & 1;
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % NS;
+    const bool landed = mbar_wait_bounded(&full_bar[s], (i / NS) & 1, abort_flag);
+    if (!__all_sync(0xffffffffu, landed)) break;
+    const uint32_t kst = ring + s * C::kStageBytes;
+    const uint32_t vst = kst + C::kPanels * kPanelBytes;
+    const int nvalid = min(kTile, t_end - (t_begin + i * kTile));
+    if (nvalid < wrow + 16) {
+      // rows past the valid tokens may hold anything (0 * NaN would poison the
+      // product): zero this warp's own V rows there before reading them
+      unsigned char *vz = smem + s * C::kStageBytes + C::kPanels * kPanelBytes;
+      for (int r = max(nvalid, wrow) + (lane >> 3); r < wrow + 16; r += 4)
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          *reinterpret_cast<uint4 *>(vz + pn * kPanelBytes + r * 128 + (lane & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+      __syncwarp();
+    }
+
+    // ---- scores: S^T[16 tokens][8 heads], two accumulators to shorten the chain
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; kk += 2) {
+      uint32_t a[4], a2[4];
+      ldsm_x4(swz(kst + (kk / 4) * kPanelBytes, ld_row_k, 2 * (kk % 4) + ld_chk_k), a);
+      ldsm_x4(swz(kst + ((kk + 1) / 4) * kPanelBytes, ld_row_k, 2 * ((kk + 1) % 4) + ld_chk_k),
+              a2);
+      Mma<T>::run(sa, a, qb[kk][0], qb[kk][1]);
+      Mma<T>::run(sb, a2, qb[kk + 1][0], qb[kk + 1][1]);
+    }
+    const bool va = wrow + g < nvalid, vb = wrow + g + 8 < nvalid;
+    const float s0 = va ? (sa[0] + sb[0]) * p.scale_log2 : -INFINITY;
+    const float s1 = va ? (sa[1] + sb[1]) * p.scale_log2 : -INFINITY;
+    const float s2 = vb ? (sa[2] + sb[2]) * p.scale_log2 : -INFINITY;
+    const float s3 = vb ? (sa[3] + sb[3]) * p.scale_log2 : -INFINITY;
+
+    // ---- online softmax over this warp's 16 tokens (max shared by the 8 lanes of a column)
+    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+    for (int off = 4; off <= 16; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m0 - mn0);
+    const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    float r0, r1, r2, r3;
+    const uint32_t x0 = Mma<T>::pack(s0 == -INFINITY ? 0.f : exp2f(s0 - mn0),
+                                     s1 == -INFINITY ? 0.f : exp2f(s1 - mn1), r0, r1);
+    const uint32_t x1 = Mma<T>::pack(s2 == -INFINITY ? 0.f : exp2f(s2 - mn0),
+                                     s3 == -INFINITY ? 0.f : exp2f(s3 - mn1), r2, r3);
+    l0 = l0 * al0 + (r0 + r2);
+    l1 = l1 * al1 + (r1 + r3);
+    if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+      for (int mt = 0; mt < KSTEPS; ++mt) {
+        o[mt][0] *= al0;
+        o[mt][1] *= al1;
+        o[mt][2] *= al0;
+        o[mt][3] *= al1;
+      }
+    }
+    // P^T fragments as the B operand: rows tokens, columns heads -> transposed in registers
+    const uint32_t pb0 = movmatrix_trans(x0);
+    const uint32_t pb1 = movmatrix_trans(x1);
+
+    // ---- O^T[d][heads] += V^T[d][tokens] . P[tokens][heads]
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt) {
+      uint32_t a[4];
+      ldsm_x4_trans(swz(vst + (mt / 4) * kPanelBytes, ld_row_v, 2 * (mt % 4) + ld_chk_v), a);
+      Mma<T>::run(o[mt], a, pb0, pb1);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+  }
+
+  // ---- per warp: complete the sums over the 8 lanes that share a head column
+#pragma unroll
+  for (int off = 4; off <= 16; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  if (g == 0) {
+    mlbuf[(warp * 8 + 2 * t) * 2] = m0;
+    mlbuf[(warp * 8 + 2 * t) * 2 + 1] = l0;
+    mlbuf[(warp * 8 + 2 * t + 1) * 2] = m1;
+    mlbuf[(warp * 8 + 2 * t + 1) * 2 + 1] = l1;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+  // ---- merge the warps in a fixed order
+  float *red = reinterpret_cast<float *>(smem);  // [warp][G][D]; the ring is idle now
+  {
+    const int h0 = 2 * t, h1 = 2 * t + 1;
+    float f0 = 0.f, f1 = 0.f;
+    if (h0 < G) {
+      float M = -INFINITY;
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h0) * 2]);
+      f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+    }
+    if (h1 < G) {
+      float M = -INFINITY;
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h1) * 2]);
+      f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+    }
+#pragma unroll
+    for (int mt = 0; mt < KSTEPS; ++mt) {
+      const int d = mt * 16 + g;
+      if (h0 < G) {
+        red[((size_t)warp * G + h0) * D + d] = o[mt][0] * f0;
+        red[((size_t)warp * G + h0) * D + d + 8] = o[mt][2] * f0;
+      }
+      if (h1 < G) {
+        red[((size_t)warp * G + h1) * D + d] = o[mt][1] * f1;
+        red[((size_t)warp * G + h1) * D + d + 8] = o[mt][3] * f1;
+      }
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+
+  const bool single = (nparts == 1);
+  for (int e0 = tid * 4; e0 < G * D; e0 += kWarps * 32 * 4) {
+    const int h = e0 / D, d = e0 % D;
+    float M = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h) * 2]);
+    float L = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = mlbuf[(w * 8 + h) * 2];
+      if (mw != -INFINITY) L += exp2f(mw - M) * mlbuf[(w * 8 + h) * 2 + 1];
+    }
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w = 0; w < kWarps; ++w) {
+      const float4 v = *reinterpret_cast<const float4 *>(red + ((size_t)w * G + h) * D + d);
+      sum.x += v.x;
+      sum.y += v.y;
+      sum.z += v.z;
+      sum.w += v.w;
+    }
+    const size_t hq = (size_t)b * p.num_q_heads + hq0 + h;
+    if (single) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      T *out = static_cast<T *>(p.out);
+      *reinterpret_cast<uint2 *>(out + hq * D + d) =
+          Elem<T>::from_f32x4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
+    } else {
+      *reinterpret_cast<float4 *>(p.ws_acc + (hq * p.max_parts + part) * D + d) = sum;
+      if (d == 0) {
+        p.ws_ml[(hq * p.max_parts + part) * 2] = M;
+        p.ws_ml[(hq * p.max_parts + part) * 2 + 1] = L;
+      }
+    }
+  }
+}
+
+}  // namespace tc
+
 // ------------------------------------------------------------------------------ merge kernel
 // One CTA per (q head, sequence), one thread per output element: combine the
 // partitions' (max, sum, weighted V) states by log-sum-exp.
@@ -600,22 +1008,110 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-template <typename T, int D, int G>
-pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, cudaStream_t stream) {
-  using L = Smem<T, D, G>;
-  const size_t smem = L::bytes(prm.table_slice);
+// ---- TMA tensor maps over a pool viewed as [num_blocks * num_kv_heads * block_size rows][D]
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+struct TmapKey {
+  const void *base;
+  long long rows;
+  int head_dim, box_rows, dtype;
+  bool operator==(const TmapKey &o) const {
+    return base == o.base && rows == o.rows && head_dim == o.head_dim && box_rows == o.box_rows &&
+           dtype == o.dtype;
+  }
+};
+
+// Encoding costs a few microseconds; the same pools come back call after call.
+bool pool_tensor_map(CUtensorMap *map, const void *base, long long rows, int head_dim,
+                     int box_rows, pa_dtype dtype) {
+  constexpr int kSlots = 16;
+  static std::mutex mu;
+  static TmapKey keys[kSlots];
+  static CUtensorMap maps[kSlots];
+  static int used = 0, next = 0;
+  const TmapKey key{base, rows, head_dim, box_rows, (int)dtype};
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (keys[i] == key) {
+      *map = maps[i];
+      return true;
+    }
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUtensorMap m;
+  if (enc(&m, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+          2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int slot = used < kSlots ? used++ : (next++ % kSlots);
+  keys[slot] = key;
+  maps[slot] = m;
+  *map = m;
+  return true;
+}
+
+bool tensor_core_block_size(int bs) { return bs >= 8 && (bs & (bs - 1)) == 0; }
+
+template <typename Kernel>
+bool ensure_smem(Kernel kernel, size_t smem, size_t (&configured)[kMaxDevices]) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
-  static size_t configured[kMaxDevices] = {};  // largest dynamic smem set per device
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
   if (smem > configured[dev]) {
-    if (cudaFuncSetAttribute(pa_decode_partition_kernel<T, D, G>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return PA_ERR_CUDA;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return false;
     configured[dev] = smem;
   }
+  return true;
+}
+
+template <typename T, int D, int G>
+pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dtype dtype,
+                        cudaStream_t stream) {
   dim3 grid((unsigned)prm.max_parts, (unsigned)prm.num_kv_heads, (unsigned)num_seqs);
-  pa_decode_partition_kernel<T, D, G><<<grid, kThreads, smem, stream>>>(prm);
+  const long long pool_rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
+  // G = 1 (one q head per kv head) leaves 7/8 of the MMA N dimension idle; the
+  // SIMT kernel measured faster there.
+  if (G > 1 && tensor_core_block_size(prm.block_size) && pool_rows <= INT32_MAX) {
+    using C = tc::Cfg<D>;
+    static size_t configured[kMaxDevices] = {};
+    const size_t smem = C::bytes(prm.table_slice);
+    const long long rows = pool_rows;
+    const int box_rows = prm.block_size < tc::kTile ? prm.block_size : tc::kTile;
+    CUtensorMap tk, tv;
+    if (!pool_tensor_map(&tk, prm.k_cache, rows, D, box_rows, dtype) ||
+        !pool_tensor_map(&tv, prm.v_cache, rows, D, box_rows, dtype))
+      return PA_ERR_CUDA;
+    if (!ensure_smem(tc::pa_decode_tc_kernel<T, D, G>, smem, configured)) return PA_ERR_CUDA;
+    tc::pa_decode_tc_kernel<T, D, G><<<grid, tc::kThreads, smem, stream>>>(tk, tv, prm);
+  } else {
+    using L = Smem<T, D, G>;
+    static size_t configured[kMaxDevices] = {};
+    const size_t smem = L::bytes(prm.table_slice);
+    if (!ensure_smem(pa_decode_partition_kernel<T, D, G>, smem, configured)) return PA_ERR_CUDA;
+    pa_decode_partition_kernel<T, D, G><<<grid, kThreads, smem, stream>>>(prm);
+  }
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (prm.max_parts > 1) {
     dim3 mgrid((unsigned)prm.num_q_heads, (unsigned)num_seqs);
@@ -629,22 +1125,22 @@ pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, cudaSt
 
 template <typename T, int D>
 pa_status dispatch_group(int group, const DecodeParams &prm, int num_seqs, void *out,
-                         cudaStream_t stream) {
+                         pa_dtype dtype, cudaStream_t stream) {
   switch (group) {
-    case 1: return launch_decode<T, D, 1>(prm, num_seqs, out, stream);
-    case 2: return launch_decode<T, D, 2>(prm, num_seqs, out, stream);
-    case 4: return launch_decode<T, D, 4>(prm, num_seqs, out, stream);
-    case 8: return launch_decode<T, D, 8>(prm, num_seqs, out, stream);
+    case 1: return launch_decode<T, D, 1>(prm, num_seqs, out, dtype, stream);
+    case 2: return launch_decode<T, D, 2>(prm, num_seqs, out, dtype, stream);
+    case 4: return launch_decode<T, D, 4>(prm, num_seqs, out, dtype, stream);
+    case 8: return launch_decode<T, D, 8>(prm, num_seqs, out, dtype, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
 
 template <typename T>
 pa_status dispatch_dim(int head_dim, int group, const DecodeParams &prm, int num_seqs, void *out,
-                       cudaStream_t stream) {
+                       pa_dtype dtype, cudaStream_t stream) {
   switch (head_dim) {
-    case 64: return dispatch_group<T, 64>(group, prm, num_seqs, out, stream);
-    case 128: return dispatch_group<T, 128>(group, prm, num_seqs, out, stream);
+    case 64: return dispatch_group<T, 64>(group, prm, num_seqs, out, dtype, stream);
+    case 128: return dispatch_group<T, 128>(group, prm, num_seqs, out, dtype, stream);
     default: return PA_ERR_UNSUPPORTED;
   }
 }
@@ -742,8 +1238,9 @@ extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, co
 
   const int group = num_q_heads / num_kv_heads;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == PA_BF16) return dispatch_dim<__nv_bfloat16>(head_dim, group, prm, num_seqs, out, st);
-  return dispatch_dim<__half>(head_dim, group, prm, num_seqs, out, st);
+  if (dtype == PA_BF16)
+    return dispatch_dim<__nv_bfloat16>(head_dim, group, prm, num_seqs, out, dtype, st);
+  return dispatch_dim<__half>(head_dim, group, prm, num_seqs, out, dtype, st);
 }
 
 pa_status pa_internal_decode_status(cudaStream_t stream, int32_t *code) {
