@@ -116,17 +116,25 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_pair
  *                  device-to-host read is made)
  *   scale          softmax scale, normally 1/sqrt(head_dim)
  *   workspace      device scratch of at least pa_decode_workspace_size() bytes
- *                  (same arguments), 16-byte aligned; may be NULL when that
- *                  size is 0. Contents need no initialisation and are
- *                  overwritten; two calls that share a workspace must not
- *                  overlap on the device
- *   partition_tokens  tokens per split-context partition (a positive multiple
- *                  of 64, at most 8192), or 0 for the library's choice
- *                  (pa_decode_default_partition)
+ *                  (same arguments, same current device), 16-byte aligned; may
+ *                  be NULL when that size is 0. Zero-fill it once before its
+ *                  first use: its first 64 KiB hold counters that every
+ *                  completed call leaves at zero (after a call that reported
+ *                  PA_DEVERR_TIMEOUT, zero-fill it again). Two calls that share
+ *                  a workspace must not overlap on the device
+ *   partition_tokens  0 for the library's choice, or a positive multiple of 64
+ *                  (at most 8192): about that many tokens of one kv head per
+ *                  CTA (smaller values split the work more finely)
  * Supported: head_dim in {64, 128}; num_q_heads / num_kv_heads in {1,2,4,8};
- * any block_size >= 1 with partition_tokens / block_size <= 4094. Sequences longer than one partition
- * are processed as several partitions whose (max, sum, weighted V) states
- * are merged by log-sum-exp in a second kernel on the same stream.
+ * any block_size >= 1 with partition_tokens / block_size <= 4094.
+ * Kernels: with 2-8 q heads per kv head and a power-of-two block_size >= 8,
+ * one persistent wave of CTAs splits all (sequence, kv head) tokens evenly
+ * (tensor cores, TMA); a sequence split between CTAs has its partial
+ * (max, sum, weighted V) states merged by log-sum-exp by the CTA that
+ * finishes last. Otherwise a SIMT kernel processes fixed partitions of
+ * partition_tokens tokens (0: pa_decode_default_partition) and a second
+ * kernel on the same stream merges them.
+
  * ------------------------------------------------------------------------------------------ */
 size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                 int max_context_len, int partition_tokens);
@@ -170,6 +178,10 @@ pa_status pa_decode_static_workspace(void *out, const void *q, const void *k_cac
                                      int num_kv_heads, int head_dim, int block_size,
                                      int num_blocks, float scale, pa_dtype dtype,
                                      int partition_tokens, void *stream);
+
+/* Kernels one pa_decode call with these arguments launches (0 if none). */
+int pa_decode_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                       int block_size, int num_blocks, int max_context_len, int partition_tokens);
 
 /* The partition size pa_decode uses for partition_tokens == 0. */
 int pa_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_len);

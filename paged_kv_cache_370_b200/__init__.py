@@ -1,19 +1,24 @@
 """Paged decode attention for NVIDIA B200 (sm_100a).
 
 The library is ``libpa370.so`` (C ABI in ``include/pa.h``): CUDA kernels for
-the paged KV write, the copy-on-write block copy and split-context decode
-attention with a log-sum-exp merge, plus a host block manager. This package
-is its Python binding; PyTorch supplies device memory and streams only.
+the paged KV write, the copy-on-write block copy and paged decode attention,
+plus a host block manager. This package is its Python binding; PyTorch
+supplies device memory and streams only.
+
+Names are resolved from ``abi`` on first use, so that ``build`` can run
+before the library exists; using any of them without the library raises.
 """
-from .abi import (  # noqa: F401
-    BlockManager,
-    OutOfBlocks,
-    PAError,
-    pa_copy_blocks,
-    pa_decode,
-    pa_decode_default_partition,
-    pa_decode_workspace_size,
-    pa_device_status,
-    pa_reshape_and_cache,
-    pa_slot_mapping,
+_EXPORTS = (
+    "BlockManager", "OutOfBlocks", "PAError", "pa_copy_blocks", "pa_decode",
+    "pa_decode_default_partition", "pa_decode_launches", "pa_decode_static_workspace",
+    "pa_decode_workspace_size", "pa_device_status", "pa_reshape_and_cache", "pa_slot_mapping",
 )
+
+__all__ = list(_EXPORTS)
+
+
+def __getattr__(name):
+    if name in _EXPORTS:
+        from . import abi
+        return getattr(abi, name)
+    raise AttributeError(f"module {__name__!r} has no attribute {name!r}")

@@ -57,6 +57,7 @@ def _load() -> ctypes.CDLL:
         "pa_decode_workspace_size": (sz, [i, i, i, i, i, i]),
         "pa_decode": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, P, sz, i, P]),
         "pa_decode_default_partition": (i, [i, i, i]),
+        "pa_decode_launches": (i, [i, i, i, i, i, i, i, i]),
         "pa_decode_static_workspace": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P]),
         "pa_device_status": (i, [P, P]),
         "pa_status_string": (ctypes.c_char_p, [i]),
@@ -156,6 +157,13 @@ def pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_
                              partition_tokens=0) -> int:
     return int(_lib.pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                              max_context_len, partition_tokens))
+
+
+def pa_decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       max_context_len, partition_tokens=0) -> int:
+    """Kernels one pa_decode call with these arguments launches."""
+    return int(_lib.pa_decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                       num_blocks, max_context_len, partition_tokens))
 
 
 def pa_decode_default_partition(num_seqs, num_kv_heads, max_context_len) -> int:

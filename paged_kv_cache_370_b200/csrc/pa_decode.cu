@@ -39,6 +39,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 #include <mutex>
 
@@ -215,6 +216,11 @@ struct DecodeParams {
   int max_parts;
   int table_slice;  // shared-memory entries reserved for a partition's block ids
   float scale_log2;  // scale * log2(e)
+  // even-split (persistent) kernel only
+  int num_seqs;
+  int grid_ctas;       // CTAs sharing the tiles
+  int *ws_counters;    // [grid_ctas] pieces finished per split segment; zero between calls
+  float *ws_pieces;    // [2 * grid_ctas][G][D + 4] partial (acc[D], max, sum, pad) per piece
 };
 
 template <int D>
@@ -569,21 +575,34 @@ __global__ void __launch_bounds__(kThreads, 3)
 }
 
 // ===================================================================== tensor-core variant
-// pa_decode_tc_kernel: the same partition work as pa_decode_partition_kernel, with
-// the q-group x K-tile and weights x V-tile products on tensor cores.
-//  * The producer warp stages each (block, kv head) piece with 2-D TMA tensor
-//    copies (cp.async.bulk.tensor, 128-byte swizzle, no multicast) into
-//    1024-byte-aligned panels of 64 head_dim columns x 64 tokens, so ldmatrix
-//    reads them without bank conflicts.
-//  * Each consumer warp owns 16 tokens of a 64-token tile and computes
-//    S^T = K_tile . Q^T with mma.m16n8k16 (tokens are M, the GQA group padded
-//    to 8 is N, head_dim is K). Its score fragment, turned into the weights P
-//    and transposed in registers with movmatrix, is directly the B operand of
-//    O^T += V_tile^T . P (head_dim is M), so weights never touch shared memory.
-//  * Weights are rounded to the input type for the product and the running
-//    sum uses the same rounded values, so the result is an exact weighted
-//    average of V with weights perturbed by at most one rounding.
-//  * The running output is only rescaled when some head's max grew.
+// pa_decode_stream_kernel: paged decode on tensor cores with an even split of the
+// whole batch over one persistent wave of CTAs.
+//  * The work is the list of (sequence, kv head) segments, each cut into tiles of
+//    64 tokens; W tiles in all. CTA c takes tiles [c*W/n, (c+1)*W/n): every CTA
+//    streams the same number of tiles (+-1) through one continuous pipeline, so
+//    neither uneven lengths nor per-partition ramp-up leave the HBM idle. The
+//    split points depend only on token counts, never on block ids or sizes.
+//  * A producer warp walks the CTA's tiles in order and stages each (block, kv
+//    head) piece with 2-D TMA tensor copies (cp.async.bulk.tensor, 128-byte
+//    swizzle, no multicast) into 1024-byte-aligned panels of 64 head_dim
+//    columns x 64 tokens; at the start of a segment it also copies the GQA
+//    group's q rows. Per-tile metadata travels with the stage.
+//  * Each consumer warp owns 16 tokens of a tile and computes S^T = K_tile . Q^T
+//    with mma.m16n8k16 (tokens are M, the GQA group padded to 8 is N, head_dim
+//    is K). The score fragment, turned into weights P and transposed in
+//    registers with movmatrix, is the B operand of O^T += V_tile^T . P (head_dim
+//    is M): weights never touch shared memory.
+//  * Weights are rounded to the input type for the product and the running sum
+//    uses the same rounded values, so the result is an exact weighted average of
+//    V with each weight perturbed by at most one rounding. The running output is
+//    rescaled only when some head's max grew.
+//  * When a CTA reaches the end of its piece of a segment, its warps merge in a
+//    fixed order. A segment wholly inside the CTA is written out directly.
+//    Otherwise the piece's (acc, max, sum) goes to the workspace and a counter
+//    per split segment is incremented; the CTA that brings it to the number of
+//    pieces merges them (in CTA order: deterministic) and resets the counter,
+//    so the counters are zero again when the kernel ends. No CTA ever waits for
+//    another.
 // Requires a power-of-two block size >= 8 (every TMA box then starts on a
 // 1024-byte boundary and blocks align with 64-token tiles).
 namespace tc {
@@ -592,21 +611,6 @@ constexpr int kTile = 64;            // tokens per stage
 constexpr int kWarps = 4;            // consumer warps, 16 tokens each
 constexpr int kThreads = (kWarps + 1) * 32;
 constexpr int kPanelBytes = kTile * 128;  // 64 columns of 2 bytes x 64 rows
-
-template <int D>
-struct Cfg {
-  static constexpr int kPanels = D / 64;
-  static constexpr int kStageBytes = 2 * kPanels * kPanelBytes;  // K panels then V panels
-  static constexpr int kStages = D == 128 ? 3 : 4;
-  static constexpr int kRingBytes = kStages * kStageBytes;
-  static constexpr int kBarOffset = kRingBytes;
-  static constexpr int kMlOffset = kBarOffset + 2 * kStages * 8;
-  static constexpr int kFlagOffset = kMlOffset + kWarps * 8 * 2 * 4;
-  static constexpr int kTableOffset = kFlagOffset + 16;
-  static constexpr int kCtasPerSm = D == 128 ? 2 : 3;
-  static size_t bytes(int table_slice) { return 1024 + kTableOffset + (size_t)table_slice * 4; }
-  static_assert(kWarps * 8 * D * 4 <= kRingBytes, "merge buffer must fit in the ring");
-};
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar) {
@@ -680,43 +684,108 @@ __device__ __forceinline__ uint32_t swz(uint32_t panel, int row, int chunk) {
   return panel + row * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
+// Per-tile schedule handed from the producer warp to the consumers with the tile.
+struct TileMeta {
+  int b, kvh, j;      // sequence, kv head, tile index inside the (sequence, kv head) segment
+  int seg_tiles;      // tiles of the segment
+  int nvalid;         // valid tokens in this tile (0..64)
+  int seg_first_x;    // global index of the segment's first tile
+  int flags;          // 1: first tile of this CTA's piece, 2: last tile of it
+  int pad;
+};
+
+template <int D, int G>
+struct Cfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kStageBytes = 2 * kPanels * kPanelBytes;  // K panels then V panels
+  static constexpr int kStages = D == 128 ? 3 : 4;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kQBytes = G * D * 2;  // the q rows of one GQA group
+  static constexpr int kQOffset = kRingBytes;
+  static constexpr int kRedOffset = kQOffset + kStages * kQBytes;
+  static constexpr int kRedBytes = kWarps * G * D * 4;
+  static constexpr int kMetaOffset = kRedOffset + kRedBytes;
+  static constexpr int kBarOffset = kMetaOffset + kStages * (int)sizeof(TileMeta);
+  static constexpr int kMlOffset = kBarOffset + 2 * kStages * 8;
+  static constexpr int kCtrlOffset = kMlOffset + kWarps * 8 * 2 * 4;
+  static constexpr int kBytes = 1024 + kCtrlOffset + 64;  // + slack to align the ring to 1 KB
+};
+
+// The CTA owning global tile x when W tiles are split evenly over n CTAs
+// (CTA c owns [c*W/n, (c+1)*W/n)).
+__device__ __forceinline__ int owner_cta(long long x, long long W, int n) {
+  return (int)(((x + 1) * n - 1) / W);
+}
+
+// Whether CTA c owns any tile (with more CTAs than tiles some own none).
+__device__ __forceinline__ bool cta_has_tiles(int c, long long W, int n) {
+  return (long long)c * W / n < (long long)(c + 1) * W / n;
+}
+
+__device__ __forceinline__ int clamp_len(int len, int cap, int max_len, bool &bad) {
+  if (len < 0 || len > cap || len > max_len) {
+    bad = true;
+    return len < 0 ? 0 : min(min(len, cap), max_len);
+  }
+  return len;
+}
+
+// tiles of one (sequence, kv head) segment; an empty sequence still gets one
+// (empty) tile so that its output is written (zeros)
+// floats per stored piece of one head: acc[D], max, sum and padding that keeps
+// every piece 16-byte aligned for vector access
+template <int D>
+constexpr int piece_stride() { return D + 4; }
+
+__device__ __forceinline__ int seg_tiles(int len) { return len > 0 ? (len + kTile - 1) / kTile : 1; }
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, Cfg<D>::kCtasPerSm)
-    pa_decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                        const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using C = Cfg<D>;
+__global__ void __launch_bounds__(kThreads, 1)
+    pa_decode_stream_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                            const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+  using C = Cfg<D, G>;
   constexpr int NS = C::kStages;
   constexpr int KSTEPS = D / 16;
+  constexpr int kPieceStride = piece_stride<D>();
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  // the ring starts on a 1024-byte boundary (the 128-byte swizzle repeats every 1 KB)
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
   uint64_t *empty_bar = full_bar + NS;
+  TileMeta *meta = reinterpret_cast<TileMeta *>(smem + C::kMetaOffset);
   float *mlbuf = reinterpret_cast<float *>(smem + C::kMlOffset);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kFlagOffset);
-  int32_t *table = reinterpret_cast<int32_t *>(smem + C::kTableOffset);
+  float *red = reinterpret_cast<float *>(smem + C::kRedOffset);
+  long long *ctrl = reinterpret_cast<long long *>(smem + C::kCtrlOffset);  // W, x0, x1
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 3);
+  volatile int *last_flag = abort_flag + 1;
   const uint32_t ring = smem_u32(smem);
 
-  const int part = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cta = blockIdx.x, nctas = p.grid_ctas;
+  const int Hkv = p.num_kv_heads, B = p.num_seqs, bs = p.block_size;
+  const int cap = p.max_blocks_per_seq * bs;
 
-  int len = __ldg(p.context_lens + b);
-  const int cap = p.max_blocks_per_seq * p.block_size;
-  if (len < 0 || len > cap || len > p.max_context_len) {
-    if (tid == 0 && part == 0 && kvh == 0) atomicOr(&g_decode_error, PA_DEVERR_CONTEXT_LEN);
-    len = len < 0 ? 0 : min(min(len, cap), p.max_context_len);
+  // ---- size the whole job (every CTA does the same scan) and take an even share
+  if (warp == kWarps) {
+    long long W = 0;
+    bool bad = false;
+    for (int base = 0; base < B; base += 32) {
+      int tiles = 0;
+      if (base + lane < B)
+        tiles = Hkv * seg_tiles(clamp_len(__ldg(p.context_lens + base + lane), cap,
+                                          p.max_context_len, bad));
+      for (int off = 16; off >= 1; off >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, off);
+      W += tiles;
+    }
+    if (__any_sync(0xffffffffu, bad) && cta == 0 && lane == 0)
+      atomicOr(&g_decode_error, PA_DEVERR_CONTEXT_LEN);
+    if (lane == 0) {
+      ctrl[0] = W;
+      ctrl[1] = (long long)cta * W / nctas;
+      ctrl[2] = (long long)(cta + 1) * W / nctas;
+    }
   }
-  const int nparts = len > 0 ? (len + p.partition_tokens - 1) / p.partition_tokens : 1;
-  if (part >= nparts) return;
-  const int t_begin = part * p.partition_tokens;
-  const int t_end = min(len, t_begin + p.partition_tokens);
-  const int ntok = t_end - t_begin;
-  const int ntiles = (ntok + kTile - 1) / kTile;
-  const int bs = p.block_size;
-  const int box_rows = bs < kTile ? bs : kTile;
-
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
@@ -725,54 +794,112 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kCtasPerSm)
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  const int blk_first = t_begin / bs;
-  const int nblk = ntok > 0 ? (t_end - 1) / bs - blk_first + 1 : 0;
-  if (warp == kWarps) {
-    const int32_t *row = p.block_tables + (size_t)b * p.max_blocks_per_seq + blk_first;
-    for (int i = lane; i < nblk; i += 32) table[i] = __ldg(row + i);
-  }
   __syncthreads();
+  const long long W = ctrl[0], x0 = ctrl[1], x1 = ctrl[2];
+  if (x0 >= x1) return;  // nothing for this CTA (uniform)
+  const int ntiles = (int)(x1 - x0);
 
   if (warp == kWarps) {
-    // ================================================================== producer
+    // ===================================================================== producer
+    // find the segment holding tile x0: sequences in order, kv heads inner
+    long long pre = 0;
+    int b = 0;
+    bool bad = false;
+    for (int base = 0; base < B; base += 32) {
+      int tiles = 0;
+      if (base + lane < B)
+        tiles = Hkv * seg_tiles(clamp_len(__ldg(p.context_lens + base + lane), cap,
+                                          p.max_context_len, bad));
+      int incl = tiles;
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      if (pre + total > x0) {
+        const unsigned hit = __ballot_sync(0xffffffffu, base + lane < B && pre + incl > x0);
+        const int first = __ffs(hit) - 1;
+        const int before = __shfl_sync(0xffffffffu, incl - tiles, first);
+        b = base + first;
+        pre += before;
+        break;
+      }
+      pre += total;
+    }
+    int len_b = clamp_len(__ldg(p.context_lens + b), cap, p.max_context_len, bad);
+    int tb = seg_tiles(len_b);
+    int kvh = (int)((x0 - pre) / tb);
+    int j = (int)((x0 - pre) % tb);
+    const int box_rows = bs < kTile ? bs : kTile;
+    const uint32_t box_bytes = 2u * C::kPanels * box_rows * 128u;
+    const int32_t *tables = p.block_tables;
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
-      int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
-        const int s = i % NS;
-        if (i >= NS && !mbar_wait_bounded(&empty_bar[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
-        const int t0 = t_begin + i * kTile;
-        const int t1 = min(t0 + kTile, t_end);
-        const int blk0 = t0 / bs, blk1 = (t1 - 1) / bs;
-        uint32_t boxes = 0;
-        for (int blk = blk0; blk <= blk1; ++blk) {
-          const int phys = table[blk - blk_first];
-          if (phys < 0 || phys >= p.num_blocks) {
-            atomicOr(&g_decode_error, PA_DEVERR_BLOCK_ID);
-            continue;
-          }
-          ++boxes;
-        }
-        mbar_expect_tx_arrive(&full_bar[s], boxes * (uint32_t)(2 * C::kPanels * box_rows * 128));
-        const uint32_t stage = ring + s * C::kStageBytes;
-        for (int blk = blk0; blk <= blk1; ++blk) {
-          const int phys = table[blk - blk_first];
-          if (phys < 0 || phys >= p.num_blocks) continue;
-          // first row of the box inside its block, and where it lands in the tile
-          const int r0 = bs > kTile ? t0 - blk * bs : 0;
-          const int row = blk * bs + r0 - t0;
-          const int y = (phys * p.num_kv_heads + kvh) * bs + r0;
-#pragma unroll
-          for (int pn = 0; pn < C::kPanels; ++pn) {
-            tma_load_2d(stage + pn * kPanelBytes + row * 128, &tmap_k, pn * 64, y, &full_bar[s]);
-            tma_load_2d(stage + (C::kPanels + pn) * kPanelBytes + row * 128, &tmap_v, pn * 64, y,
-                        &full_bar[s]);
-          }
-        }
-        issued = i + 1;
+    }
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % NS;
+      // stage free? (after a give-up the loop runs on without waiting: no early exits)
+      if (i >= NS) mbar_wait_bounded(&empty_bar[s], ((i / NS) & 1) ^ 1, abort_flag);
+      __syncwarp();
+      const int t0 = j * kTile;
+      const int nvalid = max(0, min(kTile, len_b - t0));
+      const bool seg_begin = (j == 0) || (i == 0);
+      const bool seg_end = (j == tb - 1) || (i == ntiles - 1);
+      const int nbox = nvalid > 0 ? (bs <= kTile ? (t0 + nvalid - 1) / bs - t0 / bs + 1 : 1) : 0;
+      int phys = -1;
+      bool ok = false;
+      if (lane < nbox) {
+        phys = __ldg(tables + (size_t)b * p.max_blocks_per_seq + t0 / bs + lane);
+        ok = phys >= 0 && phys < p.num_blocks;
+        if (!ok) atomicOr(&g_decode_error, PA_DEVERR_BLOCK_ID);
       }
-      for (int i = max(0, issued - NS); i < issued; ++i) {
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) {
+        TileMeta &m = meta[s];
+        m.b = b;
+        m.kvh = kvh;
+        m.j = j;
+        m.seg_tiles = tb;
+        m.nvalid = nvalid;
+        m.seg_first_x = (int)(x0 + i - j);
+        m.flags = (seg_begin ? 1 : 0) | (seg_end ? 2 : 0);
+        mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes +
+                                                (seg_begin ? (uint32_t)C::kQBytes : 0u));
+      }
+      __syncwarp();
+      const uint32_t stage = ring + s * C::kStageBytes;
+      if (ok) {
+        // box of block t0/bs + lane: whole block (bs <= 64) or a 64-row slice (bs > 64)
+        const int r0 = bs > kTile ? t0 % bs : 0;
+        const int row = bs > kTile ? 0 : lane * bs;
+        const int y = (phys * Hkv + kvh) * bs + r0;
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_2d(stage + pn * kPanelBytes + row * 128, &tmap_k, pn * 64, y, &full_bar[s]);
+          tma_load_2d(stage + (C::kPanels + pn) * kPanelBytes + row * 128, &tmap_v, pn * 64, y,
+                      &full_bar[s]);
+        }
+      }
+      if (lane == 0 && seg_begin)
+        bulk_g2s(smem + C::kQOffset + s * C::kQBytes,
+                 static_cast<const T *>(p.q) + ((size_t)b * p.num_q_heads + (size_t)kvh * G) * D,
+                 C::kQBytes, &full_bar[s]);
+      // next tile: kv heads inner, then sequences
+      if (++j == tb) {
+        j = 0;
+        if (++kvh == Hkv) {
+          kvh = 0;
+          if (++b < B) {
+            len_b = clamp_len(__ldg(p.context_lens + b), cap, p.max_context_len, bad);
+            tb = seg_tiles(len_b);
+          }
+        }
+      }
+    }
+    // do not leave while copies may still land in this CTA's shared memory
+    if (lane == 0) {
+      for (int i = max(0, ntiles - NS); i < ntiles; ++i) {
         const int s = i % NS;
         const unsigned long long t_start = global_ns();
         while (!mbar_try_wait(&full_bar[s], (i / NS) & 1)) {
@@ -786,43 +913,43 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kCtasPerSm)
     return;
   }
 
-  // ===================================================================== consumers
+  // ======================================================================= consumers
   const int g = lane >> 2;  // fragment row group
-  const int t = lane & 3;   // thread in group: this lane's heads are 2t and 2t+1
-  const int hq0 = kvh * G;
-
-  // B operand of S^T = K . Q^T: Q^T[d][head], head = g (zero for padding heads)
-  uint32_t qb[KSTEPS][2];
-  {
-    const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
-        static_cast<const T *>(p.q) + ((size_t)b * p.num_q_heads + hq0 + (g < G ? g : 0)) * D);
-#pragma unroll
-    for (int kk = 0; kk < KSTEPS; ++kk) {
-      qb[kk][0] = g < G ? __ldg(qrow + (kk * 16 + 2 * t) / 2) : 0u;
-      qb[kk][1] = g < G ? __ldg(qrow + (kk * 16 + 8 + 2 * t) / 2) : 0u;
-    }
-  }
-
-  float o[KSTEPS][4];  // O^T fragments: rows d, columns heads 2t, 2t+1
-#pragma unroll
-  for (int mt = 0; mt < KSTEPS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max of heads 2t, 2t+1 (log2 units)
-  float l0 = 0.f, l1 = 0.f;              // this lane's share of the running sums
-
-  const int wrow = warp * 16;  // first token of this warp in a tile
-  // per-lane ldmatrix row / chunk offsets
-  const int ld_row_k = wrow + (lane & 7) + 8 * ((lane >> 3) & 1);  // QK: A = K rows
+  const int t = lane & 3;   // this lane's heads are 2t and 2t+1
+  const int wrow = warp * 16;
+  const int ld_row_k = wrow + (lane & 7) + 8 * ((lane >> 3) & 1);
   const int ld_chk_k = lane >> 4;
-  const int ld_row_v = wrow + (lane & 7) + 8 * (lane >> 4);        // PV: A = V^T
+  const int ld_row_v = wrow + (lane & 7) + 8 * (lane >> 4);
   const int ld_chk_v = (lane >> 3) & 1;
+
+  uint32_t qb[KSTEPS][2];
+  float o[KSTEPS][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % NS;
-    const bool landed = mbar_wait_bounded(&full_bar[s], (i / NS) & 1, abort_flag);
-    if (!__all_sync(0xffffffffu, landed)) break;
+    // after a give-up the loop runs on (on whatever the stage holds) so every
+    // consumer warp reaches every barrier below
+    mbar_wait_bounded(&full_bar[s], (i / NS) & 1, abort_flag);
+    __syncwarp();
+    const TileMeta mt = meta[s];
     const uint32_t kst = ring + s * C::kStageBytes;
     const uint32_t vst = kst + C::kPanels * kPanelBytes;
-    const int nvalid = min(kTile, t_end - (t_begin + i * kTile));
+    if (mt.flags & 1) {
+      // a new segment piece: reset the state and take its q rows (Q^T as the B operand)
+      const uint32_t *qs =
+          reinterpret_cast<const uint32_t *>(smem + C::kQOffset + s * C::kQBytes);
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+        qb[kk][0] = g < G ? qs[(g * D + kk * 16 + 2 * t) / 2] : 0u;
+        qb[kk][1] = g < G ? qs[(g * D + kk * 16 + 8 + 2 * t) / 2] : 0u;
+      }
+#pragma unroll
+      for (int x = 0; x < KSTEPS; ++x) o[x][0] = o[x][1] = o[x][2] = o[x][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+    }
+    const int nvalid = mt.nvalid;
     if (nvalid < wrow + 16) {
       // rows past the valid tokens may hold anything (0 * NaN would poison the
       // product): zero this warp's own V rows there before reading them
@@ -835,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kCtasPerSm)
       __syncwarp();
     }
 
-    // ---- scores: S^T[16 tokens][8 heads], two accumulators to shorten the chain
+    // ---- S^T[16 tokens][8 heads] = K . Q^T
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < KSTEPS; kk += 2) {
@@ -852,7 +979,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kCtasPerSm)
     const float s2 = vb ? (sa[2] + sb[2]) * p.scale_log2 : -INFINITY;
     const float s3 = vb ? (sa[3] + sb[3]) * p.scale_log2 : -INFINITY;
 
-    // ---- online softmax over this warp's 16 tokens (max shared by the 8 lanes of a column)
+    // ---- online softmax over the warp's 16 tokens (max shared by a column's 8 lanes)
     float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
     for (int off = 4; off <= 16; off <<= 1) {
@@ -865,113 +992,160 @@ __global__ void __launch_bounds__(kThreads, Cfg<D>::kCtasPerSm)
     m0 = mn0;
     m1 = mn1;
     float r0, r1, r2, r3;
-    const uint32_t x0 = Mma<T>::pack(s0 == -INFINITY ? 0.f : exp2f(s0 - mn0),
-                                     s1 == -INFINITY ? 0.f : exp2f(s1 - mn1), r0, r1);
-    const uint32_t x1 = Mma<T>::pack(s2 == -INFINITY ? 0.f : exp2f(s2 - mn0),
-                                     s3 == -INFINITY ? 0.f : exp2f(s3 - mn1), r2, r3);
+    const uint32_t x0w = Mma<T>::pack(s0 == -INFINITY ? 0.f : exp2f(s0 - mn0),
+                                      s1 == -INFINITY ? 0.f : exp2f(s1 - mn1), r0, r1);
+    const uint32_t x1w = Mma<T>::pack(s2 == -INFINITY ? 0.f : exp2f(s2 - mn0),
+                                      s3 == -INFINITY ? 0.f : exp2f(s3 - mn1), r2, r3);
     l0 = l0 * al0 + (r0 + r2);
     l1 = l1 * al1 + (r1 + r3);
     if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-      for (int mt = 0; mt < KSTEPS; ++mt) {
-        o[mt][0] *= al0;
-        o[mt][1] *= al1;
-        o[mt][2] *= al0;
-        o[mt][3] *= al1;
+      for (int x = 0; x < KSTEPS; ++x) {
+        o[x][0] *= al0;
+        o[x][1] *= al1;
+        o[x][2] *= al0;
+        o[x][3] *= al1;
       }
     }
-    // P^T fragments as the B operand: rows tokens, columns heads -> transposed in registers
-    const uint32_t pb0 = movmatrix_trans(x0);
-    const uint32_t pb1 = movmatrix_trans(x1);
+    const uint32_t pb0 = movmatrix_trans(x0w);
+    const uint32_t pb1 = movmatrix_trans(x1w);
 
     // ---- O^T[d][heads] += V^T[d][tokens] . P[tokens][heads]
 #pragma unroll
-    for (int mt = 0; mt < KSTEPS; ++mt) {
+    for (int x = 0; x < KSTEPS; ++x) {
       uint32_t a[4];
-      ldsm_x4_trans(swz(vst + (mt / 4) * kPanelBytes, ld_row_v, 2 * (mt % 4) + ld_chk_v), a);
-      Mma<T>::run(o[mt], a, pb0, pb1);
+      ldsm_x4_trans(swz(vst + (x / 4) * kPanelBytes, ld_row_v, 2 * (x % 4) + ld_chk_v), a);
+      Mma<T>::run(o[x], a, pb0, pb1);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty_bar[s]);
-  }
 
-  // ---- per warp: complete the sums over the 8 lanes that share a head column
+    if (!(mt.flags & 2)) continue;
+    // ================================= end of this CTA's piece of the segment: flush
+    float sl0 = l0, sl1 = l1;
 #pragma unroll
-  for (int off = 4; off <= 16; off <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-  }
-  if (g == 0) {
-    mlbuf[(warp * 8 + 2 * t) * 2] = m0;
-    mlbuf[(warp * 8 + 2 * t) * 2 + 1] = l0;
-    mlbuf[(warp * 8 + 2 * t + 1) * 2] = m1;
-    mlbuf[(warp * 8 + 2 * t + 1) * 2 + 1] = l1;
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
-  // ---- merge the warps in a fixed order
-  float *red = reinterpret_cast<float *>(smem);  // [warp][G][D]; the ring is idle now
-  {
-    const int h0 = 2 * t, h1 = 2 * t + 1;
-    float f0 = 0.f, f1 = 0.f;
-    if (h0 < G) {
-      float M = -INFINITY;
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h0) * 2]);
-      f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+    for (int off = 4; off <= 16; off <<= 1) {
+      sl0 += __shfl_xor_sync(0xffffffffu, sl0, off);
+      sl1 += __shfl_xor_sync(0xffffffffu, sl1, off);
     }
-    if (h1 < G) {
-      float M = -INFINITY;
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h1) * 2]);
-      f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+    if (g == 0) {
+      mlbuf[(warp * 8 + 2 * t) * 2] = m0;
+      mlbuf[(warp * 8 + 2 * t) * 2 + 1] = sl0;
+      mlbuf[(warp * 8 + 2 * t + 1) * 2] = m1;
+      mlbuf[(warp * 8 + 2 * t + 1) * 2 + 1] = sl1;
     }
-#pragma unroll
-    for (int mt = 0; mt < KSTEPS; ++mt) {
-      const int d = mt * 16 + g;
+    asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+    {
+      const int h0 = 2 * t, h1 = 2 * t + 1;
+      float f0 = 0.f, f1 = 0.f;
       if (h0 < G) {
-        red[((size_t)warp * G + h0) * D + d] = o[mt][0] * f0;
-        red[((size_t)warp * G + h0) * D + d + 8] = o[mt][2] * f0;
+        float M = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h0) * 2]);
+        f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
       }
       if (h1 < G) {
-        red[((size_t)warp * G + h1) * D + d] = o[mt][1] * f1;
-        red[((size_t)warp * G + h1) * D + d + 8] = o[mt][3] * f1;
+        float M = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h1) * 2]);
+        f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+      }
+#pragma unroll
+      for (int x = 0; x < KSTEPS; ++x) {
+        const int d = x * 16 + g;
+        if (h0 < G) {
+          red[(warp * G + h0) * D + d] = o[x][0] * f0;
+          red[(warp * G + h0) * D + d + 8] = o[x][2] * f0;
+        }
+        if (h1 < G) {
+          red[(warp * G + h1) * D + d] = o[x][1] * f1;
+          red[(warp * G + h1) * D + d + 8] = o[x][3] * f1;
+        }
       }
     }
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
-
-  const bool single = (nparts == 1);
-  for (int e0 = tid * 4; e0 < G * D; e0 += kWarps * 32 * 4) {
-    const int h = e0 / D, d = e0 % D;
-    float M = -INFINITY;
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h) * 2]);
-    float L = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      const float mw = mlbuf[(w * 8 + h) * 2];
-      if (mw != -INFINITY) L += exp2f(mw - M) * mlbuf[(w * 8 + h) * 2 + 1];
-    }
-    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int w = 0; w < kWarps; ++w) {
-      const float4 v = *reinterpret_cast<const float4 *>(red + ((size_t)w * G + h) * D + d);
-      sum.x += v.x;
-      sum.y += v.y;
-      sum.z += v.z;
-      sum.w += v.w;
-    }
-    const size_t hq = (size_t)b * p.num_q_heads + hq0 + h;
-    if (single) {
-      const float inv = L > 0.f ? 1.f / L : 0.f;
-      T *out = static_cast<T *>(p.out);
-      *reinterpret_cast<uint2 *>(out + hq * D + d) =
-          Elem<T>::from_f32x4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
-    } else {
-      *reinterpret_cast<float4 *>(p.ws_acc + (hq * p.max_parts + part) * D + d) = sum;
-      if (d == 0) {
-        p.ws_ml[(hq * p.max_parts + part) * 2] = M;
-        p.ws_ml[(hq * p.max_parts + part) * 2 + 1] = L;
+    asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+    const bool whole = mt.seg_first_x >= x0 && (long long)mt.seg_first_x + mt.seg_tiles <= x1;
+    const bool first_of_cta = mt.seg_first_x <= x0;
+    const int slot = first_of_cta ? 2 * cta : 2 * cta + 1;
+    const size_t hq_base = (size_t)mt.b * p.num_q_heads + (size_t)mt.kvh * G;
+    for (int e0 = tid * 4; e0 < G * D; e0 += kWarps * 32 * 4) {
+      const int h = e0 / D, d = e0 % D;
+      float M = -INFINITY;
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mlbuf[(w * 8 + h) * 2]);
+      float L = 0.f;
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = mlbuf[(w * 8 + h) * 2];
+        if (mw != -INFINITY) L += exp2f(mw - M) * mlbuf[(w * 8 + h) * 2 + 1];
+      }
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int w = 0; w < kWarps; ++w) {
+        const float4 v = *reinterpret_cast<const float4 *>(red + (w * G + h) * D + d);
+        sum.x += v.x;
+        sum.y += v.y;
+        sum.z += v.z;
+        sum.w += v.w;
+      }
+      if (whole) {
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        *reinterpret_cast<uint2 *>(static_cast<T *>(p.out) + (hq_base + h) * D + d) =
+            Elem<T>::from_f32x4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
+      } else {
+        float *pc = p.ws_pieces + ((size_t)slot * G + h) * kPieceStride;
+        *reinterpret_cast<float4 *>(pc + d) = sum;
+        if (d == 0) {
+          pc[D] = M;
+          pc[D + 1] = L;
+        }
       }
     }
+    if (!whole) {
+      // the piece is out; the CTA that completes the segment's last piece merges
+      __threadfence();
+      asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+      const long long sf = mt.seg_first_x;
+      const int ca = owner_cta(sf, W, nctas);
+      const int cb = owner_cta(sf + mt.seg_tiles - 1, W, nctas);
+      if (tid == 0) {
+        int pieces = 0;  // one per CTA in [ca, cb] that owns tiles
+        for (int cc = ca; cc <= cb; ++cc) pieces += cta_has_tiles(cc, W, nctas) ? 1 : 0;
+        *last_flag = atomicAdd(p.ws_counters + ca, 1) == pieces - 1;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+      if (*last_flag) {
+        __threadfence();
+        const long long x0a = (long long)ca * W / nctas;
+        for (int e0 = tid * 4; e0 < G * D; e0 += kWarps * 32 * 4) {
+          const int h = e0 / D, d = e0 % D;
+          float M = -INFINITY;
+          for (int cc = ca; cc <= cb; ++cc) {
+            if (!cta_has_tiles(cc, W, nctas)) continue;
+            const int sl = (cc == ca && sf > x0a) ? 2 * cc + 1 : 2 * cc;
+            M = fmaxf(M, __ldcg(p.ws_pieces + ((size_t)sl * G + h) * kPieceStride + D));
+          }
+          float L = 0.f;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int cc = ca; cc <= cb; ++cc) {
+            if (!cta_has_tiles(cc, W, nctas)) continue;
+            const int sl = (cc == ca && sf > x0a) ? 2 * cc + 1 : 2 * cc;
+            const float *pc = p.ws_pieces + ((size_t)sl * G + h) * kPieceStride;
+            const float mc = __ldcg(pc + D);
+            if (mc == -INFINITY) continue;
+            const float w = exp2f(mc - M);
+            L += w * __ldcg(pc + D + 1);
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(pc + d));
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
+          }
+          const float inv = L > 0.f ? 1.f / L : 0.f;
+          *reinterpret_cast<uint2 *>(static_cast<T *>(p.out) + (hq_base + h) * D + d) =
+              Elem<T>::from_f32x4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        }
+        if (tid == 0) p.ws_counters[ca] = 0;  // every piece has arrived: ready for the next call
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");  // red / mlbuf reused next
   }
 }
-
 }  // namespace tc
 
 // ------------------------------------------------------------------------------ merge kernel
@@ -1007,6 +1181,10 @@ __global__ void __launch_bounds__(D) pa_decode_merge_kernel(
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kPartitionQuantum = 64;   // partitions are whole tiles for every head_dim
+constexpr int kMaxPartitionTokens = 8192;
+constexpr int kSmCount = 148;
+constexpr int kCtasPerSm = 3;
 
 // ---- TMA tensor maps over a pool viewed as [num_blocks * num_kv_heads * block_size rows][D]
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -1086,32 +1264,104 @@ bool ensure_smem(Kernel kernel, size_t smem, size_t (&configured)[kMaxDevices]) 
   return true;
 }
 
+// Bytes at the start of every workspace that hold the even-split kernel's
+// counters; they must be zero before the first call and every call leaves them
+// zero. The split-partition scratch of the SIMT path starts after them.
+constexpr size_t kCounterRegion = 64 * 1024;
+constexpr int kMaxStreamCtas = (int)(kCounterRegion / sizeof(int));
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return kSmCount;
+  return n;
+}
+
+template <int D, int G>
+int stream_ctas_per_sm() {
+  static int per_sm[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
+  if (!per_sm[dev]) {
+    auto kernel = tc::pa_decode_stream_kernel<__nv_bfloat16, D, G>;
+    const size_t smem = tc::Cfg<D, G>::kBytes;
+    int n = 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, tc::kThreads, smem) !=
+            cudaSuccess ||
+        n <= 0)
+      n = 1;
+    per_sm[dev] = n;
+  }
+  return per_sm[dev];
+}
+
+template <int D>
+int stream_ctas_per_sm_g(int group) {
+  switch (group) {
+    case 2: return stream_ctas_per_sm<D, 2>();
+    case 4: return stream_ctas_per_sm<D, 4>();
+    default: return stream_ctas_per_sm<D, 8>();
+  }
+}
+
+// CTAs of the even-split kernel: one resident wave by default; with
+// partition_tokens > 0, about partition_tokens tokens of one kv head per CTA.
+int stream_grid(int num_seqs, int num_kv_heads, int group, int head_dim, int max_context_len,
+                int partition_tokens) {
+  long long n;
+  if (partition_tokens > 0) {
+    const long long tiles = (long long)num_seqs * num_kv_heads *
+                            std::max(1, (max_context_len + 63) / 64);
+    n = (tiles + partition_tokens / 64 - 1) / (partition_tokens / 64);
+  } else {
+    n = (long long)sm_count() *
+        (head_dim == 128 ? stream_ctas_per_sm_g<128>(group) : stream_ctas_per_sm_g<64>(group));
+  }
+  return (int)std::max(1LL, std::min<long long>(n, kMaxStreamCtas));
+}
+
+bool uses_stream_kernel(int group, int block_size, int num_blocks, int num_kv_heads) {
+  const long long rows = (long long)num_blocks * num_kv_heads * block_size;
+  // one q head per kv head leaves 7/8 of the MMA N dimension idle: the SIMT
+  // kernel measured faster there
+  return group > 1 && tensor_core_block_size(block_size) && rows <= INT32_MAX;
+}
+
+size_t stream_workspace(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                        int max_context_len, int partition_tokens) {
+  const int group = num_q_heads / num_kv_heads;
+  const int n = stream_grid(num_seqs, num_kv_heads, group, head_dim, max_context_len,
+                            partition_tokens);
+  return (size_t)2 * n * group * (head_dim + 4) * sizeof(float);
+}
+
 template <typename T, int D, int G>
 pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dtype dtype,
                         cudaStream_t stream) {
-  dim3 grid((unsigned)prm.max_parts, (unsigned)prm.num_kv_heads, (unsigned)num_seqs);
-  const long long pool_rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
-  // G = 1 (one q head per kv head) leaves 7/8 of the MMA N dimension idle; the
-  // SIMT kernel measured faster there.
-  if (G > 1 && tensor_core_block_size(prm.block_size) && pool_rows <= INT32_MAX) {
-    using C = tc::Cfg<D>;
+  if (uses_stream_kernel(G, prm.block_size, prm.num_blocks, prm.num_kv_heads)) {
+    using C = tc::Cfg<D, G>;
     static size_t configured[kMaxDevices] = {};
-    const size_t smem = C::bytes(prm.table_slice);
-    const long long rows = pool_rows;
+    const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
     const int box_rows = prm.block_size < tc::kTile ? prm.block_size : tc::kTile;
     CUtensorMap tk, tv;
     if (!pool_tensor_map(&tk, prm.k_cache, rows, D, box_rows, dtype) ||
         !pool_tensor_map(&tv, prm.v_cache, rows, D, box_rows, dtype))
       return PA_ERR_CUDA;
-    if (!ensure_smem(tc::pa_decode_tc_kernel<T, D, G>, smem, configured)) return PA_ERR_CUDA;
-    tc::pa_decode_tc_kernel<T, D, G><<<grid, tc::kThreads, smem, stream>>>(tk, tv, prm);
-  } else {
-    using L = Smem<T, D, G>;
-    static size_t configured[kMaxDevices] = {};
-    const size_t smem = L::bytes(prm.table_slice);
-    if (!ensure_smem(pa_decode_partition_kernel<T, D, G>, smem, configured)) return PA_ERR_CUDA;
-    pa_decode_partition_kernel<T, D, G><<<grid, kThreads, smem, stream>>>(prm);
+    if (!ensure_smem(tc::pa_decode_stream_kernel<T, D, G>, (size_t)C::kBytes, configured))
+      return PA_ERR_CUDA;
+    tc::pa_decode_stream_kernel<T, D, G>
+        <<<(unsigned)prm.grid_ctas, tc::kThreads, C::kBytes, stream>>>(tk, tv, prm);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
+  using L = Smem<T, D, G>;
+  static size_t configured[kMaxDevices] = {};
+  const size_t smem = L::bytes(prm.table_slice);
+  if (!ensure_smem(pa_decode_partition_kernel<T, D, G>, smem, configured)) return PA_ERR_CUDA;
+  dim3 grid((unsigned)prm.max_parts, (unsigned)prm.num_kv_heads, (unsigned)num_seqs);
+  pa_decode_partition_kernel<T, D, G><<<grid, kThreads, smem, stream>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   if (prm.max_parts > 1) {
     dim3 mgrid((unsigned)prm.num_q_heads, (unsigned)num_seqs);
@@ -1145,10 +1395,6 @@ pa_status dispatch_dim(int head_dim, int group, const DecodeParams &prm, int num
   }
 }
 
-constexpr int kPartitionQuantum = 64;   // partitions are whole tiles for every head_dim
-constexpr int kMaxPartitionTokens = 8192;
-constexpr int kSmCount = 148;
-constexpr int kCtasPerSm = 3;
 
 int resolve_partition(int num_seqs, int num_kv_heads, int max_context_len, int requested) {
   if (requested > 0) return requested;
@@ -1172,16 +1418,43 @@ extern "C" int pa_decode_default_partition(int num_seqs, int num_kv_heads, int m
   return pt < kPartitionQuantum ? kPartitionQuantum : pt;
 }
 
-extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
-                                           int head_dim, int max_context_len,
-                                           int partition_tokens) {
-  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
-      max_context_len <= 0 || partition_tokens < 0)
-    return 0;
+size_t simt_workspace(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                      int max_context_len, int partition_tokens) {
   const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
   const long long parts = (max_context_len + pt - 1) / pt;
   if (parts <= 1) return 0;
   return (size_t)num_seqs * num_q_heads * parts * (head_dim + 2) * sizeof(float);
+}
+
+extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                                           int head_dim, int max_context_len,
+                                           int partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      max_context_len <= 0 || partition_tokens < 0 || num_q_heads % num_kv_heads)
+    return 0;
+  // either kernel may run (it depends on the block size): size for the larger
+  const size_t simt = simt_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                     max_context_len, partition_tokens);
+  const int group = num_q_heads / num_kv_heads;
+  const size_t stream = (group == 2 || group == 4 || group == 8) &&
+                                (head_dim == 64 || head_dim == 128)
+                            ? stream_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                               max_context_len, partition_tokens)
+                            : 0;
+  const size_t body = simt > stream ? simt : stream;
+  return body ? kCounterRegion + body : 0;
+}
+
+extern "C" int pa_decode_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                  int block_size, int num_blocks, int max_context_len,
+                                  int partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+      block_size <= 0 || num_blocks <= 0 || head_dim <= 0)
+    return 0;
+  const int group = num_q_heads / num_kv_heads;
+  if (uses_stream_kernel(group, block_size, num_blocks, num_kv_heads)) return 1;
+  const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
+  return max_context_len > pt ? 2 : 1;
 }
 
 extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -1205,13 +1478,25 @@ extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, co
     return PA_ERR_INVALID;
   if ((long long)num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_INVALID;
 
+  const int group = num_q_heads / num_kv_heads;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_UNSUPPORTED;
   const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
   const int max_parts = max_context_len > 0 ? (max_context_len + pt - 1) / pt : 1;
-  const size_t need =
-      max_parts > 1 ? (size_t)num_seqs * num_q_heads * max_parts * (head_dim + 2) * sizeof(float)
-                    : 0;
+  const bool streamk = uses_stream_kernel(group, block_size, num_blocks, num_kv_heads);
+  const int nctas = streamk ? stream_grid(num_seqs, num_kv_heads, group, head_dim,
+                                          max_context_len, partition_tokens)
+                            : 0;
+  size_t need;
+  if (streamk)
+    need = kCounterRegion + (size_t)2 * nctas * group * (head_dim + 4) * sizeof(float);
+  else
+    need = max_parts > 1 ? kCounterRegion + (size_t)num_seqs * num_q_heads * max_parts *
+                                                (head_dim + 2) * sizeof(float)
+                         : 0;
   if (need > workspace_bytes || (need && (!workspace || !aligned(workspace, 16))))
     return PA_ERR_INVALID;
+  float *ws_body =
+      need ? reinterpret_cast<float *>(static_cast<char *>(workspace) + kCounterRegion) : nullptr;
 
   DecodeParams prm;
   prm.out = out;
@@ -1220,10 +1505,13 @@ extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, co
   prm.v_cache = v_cache;
   prm.block_tables = block_tables;
   prm.context_lens = context_lens;
-  prm.ws_acc = static_cast<float *>(workspace);
-  prm.ws_ml = need ? static_cast<float *>(workspace) +
-                         (size_t)num_seqs * num_q_heads * max_parts * head_dim
-                   : nullptr;
+  prm.ws_acc = streamk ? nullptr : ws_body;
+  prm.ws_ml = (!streamk && need) ? ws_body + (size_t)num_seqs * num_q_heads * max_parts * head_dim
+                                 : nullptr;
+  prm.num_seqs = num_seqs;
+  prm.grid_ctas = nctas;
+  prm.ws_counters = streamk ? static_cast<int *>(workspace) : nullptr;
+  prm.ws_pieces = streamk ? ws_body : nullptr;
   prm.max_blocks_per_seq = max_blocks_per_seq;
   prm.max_context_len = max_context_len;
   prm.num_q_heads = num_q_heads;
@@ -1236,7 +1524,6 @@ extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, co
   prm.scale_log2 = scale * 1.4426950408889634f;
   if ((size_t)prm.table_slice * 4 > 16384) return PA_ERR_UNSUPPORTED;
 
-  const int group = num_q_heads / num_kv_heads;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == PA_BF16)
     return dispatch_dim<__nv_bfloat16>(head_dim, group, prm, num_seqs, out, dtype, st);

@@ -36,15 +36,19 @@ class DecodeStep:
         hkv = k_cache.shape[1]
         nbytes = abi.pa_decode_workspace_size(B, hq, hkv, d, self.max_context_len,
                                               self.partition_tokens)
-        self.workspace = (torch.empty(max(nbytes, 16) // 4 + 4, dtype=torch.float32,
+        # zero-filled once: pa_decode keeps its counters zero between calls
+        self.workspace = (torch.zeros(max(nbytes, 16) // 4 + 4, dtype=torch.float32,
                                       device=q.device) if nbytes else None)
-        pt = self.partition_tokens or abi.pa_decode_default_partition(B, hkv, self.max_context_len)
-        self.partition = pt
-        self.max_parts = max(1, -(-self.max_context_len // pt))
+        nb, _, bs, _ = k_cache.shape
+        self.decode_launches = abi.pa_decode_launches(B, hq, hkv, d, bs, nb,
+                                                      self.max_context_len,
+                                                      self.partition_tokens)
+        self.partition = self.partition_tokens or abi.pa_decode_default_partition(
+            B, hkv, self.max_context_len)
 
     def launches(self) -> int:
         """Kernels one run() launches."""
-        n = 2 + (1 if self.max_parts > 1 else 0)
+        n = 1 + self.decode_launches
         if self.copy_pairs is not None and self.copy_pairs.numel():
             n += 1
         return n
@@ -72,37 +76,45 @@ class DecodeStep:
 class HostDecodeStep:
     """A DecodeStep whose per-step inputs and output live in pinned host memory.
 
-    The KV pools stay resident on the device (they are the cache); every run()
-    copies q, the new K/V, the slots, the block tables, the lengths and any
-    copy pairs host->device, runs the step and copies the output back."""
+    The KV pools stay resident on the device (they are the cache). The step's
+    inputs -- q, the new K/V, the slots, the block tables, the lengths and any
+    copy pairs -- are packed back to back (16-byte aligned) in one pinned host
+    buffer, so every run() is one host->device copy, the step's kernels, and one
+    device->host copy of the output."""
 
     def __init__(self, *, k_cache, v_cache, q, k_new, v_new, slot_mapping, block_tables,
                  context_lens, max_context_len: int, scale: float, partition_tokens: int = 0,
                  copy_pairs=None):
         dev = k_cache.device
-
-        def pin(t):
-            return t.detach().to("cpu").contiguous().pin_memory()
-
-        self.h_in = {"q": pin(q), "k_new": pin(k_new), "v_new": pin(v_new),
-                     "slot_mapping": pin(slot_mapping), "block_tables": pin(block_tables),
-                     "context_lens": pin(context_lens)}
+        parts = {"q": q, "k_new": k_new, "v_new": v_new, "slot_mapping": slot_mapping,
+                 "block_tables": block_tables, "context_lens": context_lens}
         if copy_pairs is not None and copy_pairs.numel():
-            self.h_in["copy_pairs"] = pin(copy_pairs)
-        self.d_in = {k: torch.empty_like(v, device=dev) for k, v in self.h_in.items()}
-        self.step = DecodeStep(k_cache=k_cache, v_cache=v_cache, q=self.d_in["q"],
-                               k_new=self.d_in["k_new"], v_new=self.d_in["v_new"],
-                               slot_mapping=self.d_in["slot_mapping"],
-                               block_tables=self.d_in["block_tables"],
-                               context_lens=self.d_in["context_lens"],
+            parts["copy_pairs"] = copy_pairs
+        offsets, total = {}, 0
+        for name, t in parts.items():
+            offsets[name] = total
+            total += -(-t.numel() * t.element_size() // 16) * 16
+        self.h_in = torch.empty(total, dtype=torch.uint8).pin_memory()
+        self.d_in = torch.empty(total, dtype=torch.uint8, device=dev)
+        views = {}
+        for name, t in parts.items():
+            n = t.numel() * t.element_size()
+            src = t.detach().contiguous().view(torch.uint8).reshape(-1).cpu()
+            self.h_in[offsets[name]:offsets[name] + n].copy_(src)
+            views[name] = self.d_in[offsets[name]:offsets[name] + n].view(t.dtype).view(t.shape)
+        self.step = DecodeStep(k_cache=k_cache, v_cache=v_cache, q=views["q"],
+                               k_new=views["k_new"], v_new=views["v_new"],
+                               slot_mapping=views["slot_mapping"],
+                               block_tables=views["block_tables"],
+                               context_lens=views["context_lens"],
                                max_context_len=max_context_len, scale=scale,
                                partition_tokens=partition_tokens,
-                               copy_pairs=self.d_in.get("copy_pairs"))
+                               copy_pairs=views.get("copy_pairs"))
         self.h_out = torch.empty(tuple(q.shape), dtype=q.dtype).pin_memory()
 
     @property
     def h2d_bytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in self.h_in.values())
+        return self.h_in.numel()
 
     @property
     def d2h_bytes(self) -> int:
@@ -111,9 +123,8 @@ class HostDecodeStep:
     def launches(self) -> int:
         return self.step.launches()
 
-    def run(self, stream=None):
-        for k, h in self.h_in.items():
-            self.d_in[k].copy_(h, non_blocking=True)
-        out = self.step.run(stream)
+    def run(self):
+        self.d_in.copy_(self.h_in, non_blocking=True)
+        out = self.step.run()
         self.h_out.copy_(out, non_blocking=True)
         return self.h_out

@@ -253,15 +253,19 @@ def test_decode_rejects_bad_arguments_before_launch():
 
 
 def test_workspace_size():
-    # one partition: no workspace
-    assert abi.pa_decode_workspace_size(4, 8, 2, 128, 300, 512) == 0
-    # three partitions of 512 for 1100 tokens: acc [D] + (max, sum) per (seq, head, partition)
-    assert abi.pa_decode_workspace_size(4, 8, 2, 128, 1100, 512) == 4 * 8 * 3 * (128 + 2) * 4
+    # a fixed 64 KiB counter region, then room for the larger of the two kernels' scratch
+    region = 64 * 1024
+    # fixed partitions (SIMT kernel): acc [D] + (max, sum) per (seq, q head, partition);
+    # even split with 512 tokens per CTA: 2 pieces per CTA of G heads x (D + 4)
+    simt = 4 * 8 * 3 * (128 + 2) * 4
+    ctas = -(-(4 * 2 * -(-1100 // 64)) // (512 // 64))
+    stream = 2 * ctas * 4 * (128 + 4) * 4
+    assert abi.pa_decode_workspace_size(4, 8, 2, 128, 1100, 512) == region + max(simt, stream)
+    assert abi.pa_decode_workspace_size(4, 8, 2, 128, 1100, 0) >= region
+    assert abi.pa_decode_workspace_size(4, 6, 4, 128, 1100, 0) == 0  # 6 / 4 heads: invalid
     pt = abi.pa_decode_default_partition(64, 8, 2048)
     assert pt % 64 == 0 and 64 <= pt <= 8192
-    parts = -(-2048 // pt)
-    assert abi.pa_decode_workspace_size(64, 32, 8, 128, 2048, 0) == (
-        0 if parts == 1 else 64 * 32 * parts * 130 * 4)
+
 
 
 # ------------------------------------------------------------------------------ byte accounting

@@ -207,7 +207,7 @@ def test_llama8b_full():
 
 def test_long_skew_full():
     g, out, s = _full_size(synth.long_skew())
-    assert g.step.max_parts > 1
+    assert g.step.workspace is not None  # sequences are split between CTAs and merged
 
 
 def test_mixed_sweep_full():
