@@ -69,6 +69,8 @@ def parse_args():
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--pool-blocks", type=int, default=65536,
                     help="llama8b pool size (smaller for profiler captures)")
+    ap.add_argument("--no-fuse", action="store_true",
+                    help="separate KV-write kernel instead of pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -239,7 +241,7 @@ def device_steps(args, batches, torch, device):
                           block_tables=torch.from_numpy(b.block_tables).to(device),
                           context_lens=torch.from_numpy(b.context_lens).to(device),
                           max_context_len=b.max_context_len, scale=float(b.scale),
-                          partition_tokens=args.partition_tokens)
+                          partition_tokens=args.partition_tokens, fused=not args.no_fuse)
         del k_all, v_all
         steps.append(step)
         infos.append(_byte_info(b.context_lens, b.num_q_heads, b.num_kv_heads, b.head_dim,
@@ -300,7 +302,8 @@ def shared_prompt_steps(args, torch, device):
                       context_lens=torch.from_numpy(lens).to(device),
                       max_context_len=int(lens.max()), scale=float(s.scale),
                       partition_tokens=args.partition_tokens,
-                      copy_pairs=torch.tensor(pairs, dtype=torch.int64, device=device))
+                      copy_pairs=torch.tensor(pairs, dtype=torch.int64, device=device),
+                      fused=not args.no_fuse)
     torch.cuda.synchronize()
     info = _byte_info(lens, 40, 40, 128, 16, step.partition, len(ids))
     info["copy"] = 2 * 2 * len(pairs) * 40 * 16 * 128 * 2
@@ -340,9 +343,20 @@ def run_ours(args, rank, world, local, dist):
     batches = make_batches(args, rank)
     steps, infos = device_steps(args, batches, torch, device)
     pt = steps[0].partition
-    # graphs: [copies + write] and [decode (+ merge)] per batch
-    g_write = [capture(lambda s=s: (s.copy(), s.write()), torch) for s in steps]
-    g_dec = [capture(lambda s=s: s.attend(), torch) for s in steps]
+    # graphs per batch: [copy-on-write copies (+ the KV write unless fused)] and
+    # [decode (with the fused KV write)]
+    fused = steps[0].fused
+
+    def pre(s):
+        s.copy()
+        if not s.fused:
+            s.write()
+
+    def has_pre(s):
+        return (not s.fused) or (s.copy_pairs is not None and s.copy_pairs.numel() > 0)
+
+    g_write = [capture(lambda s=s: pre(s), torch) if has_pre(s) else None for s in steps]
+    g_dec = [capture(lambda s=s: s.append() if s.fused else s.attend(), torch) for s in steps]
     V = len(steps)
 
     def barrier():
@@ -352,7 +366,8 @@ def run_ours(args, rank, world, local, dist):
 
     stream = torch.cuda.current_stream()
     for i in range(args.warmup):
-        g_write[i % V].replay()
+        if g_write[i % V] is not None:
+            g_write[i % V].replay()
         g_dec[i % V].replay()
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -370,7 +385,8 @@ def run_ours(args, rank, world, local, dist):
     for i in range(K):
         e = ev[i]
         e[0].record(stream)
-        g_write[i % V].replay()
+        if g_write[i % V] is not None:
+            g_write[i % V].replay()
         e[1].record(stream)
         g_dec[i % V].replay()
         e[2].record(stream)
@@ -389,7 +405,9 @@ def run_ours(args, rank, world, local, dist):
 
     peak, peak_kind = measured_peaks()
     dec_avg_ms = float(np.mean(dec_ms))
-    dec_bytes = float(np.mean(step_bytes))
+    # the fused kernel also reads each new token's K/V and stores it at its slot
+    dec_bytes = float(np.mean([infos[i % V]["decode"]["total"] +
+                               (infos[i % V]["write"] if fused else 0) for i in range(K)]))
     achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
     traffic = recorded_traffic() if args.workload == "llama8b" else None
     launches = sum(s.launches() for s in (steps[i % V] for i in range(K)))
@@ -411,13 +429,15 @@ def run_ours(args, rank, world, local, dist):
         "query_tokens_per_s": round(q_tok, 1),
         "pct_of_hbm_measured": round(100 * gbs / world / peak, 2),
         "pct_of_hbm_nominal_8tbs": round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
-        "roofline": {"bound": "hbm", "kernel": "pa_decode (partition kernel + LSE merge)",
+        "roofline": {"bound": "hbm",
+                     "kernel": ("pa_decode_append (KV write + decode, one kernel)" if fused
+                                else "pa_decode"),
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "traffic": traffic, "algorithmic_bytes_per_launch": int(dec_bytes),
                      "avg_launch_ms": round(dec_avg_ms, 5),
                      "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4)},
-        "kernel_ms": {"write(+copy)": round(float(np.mean(wr_ms)), 5),
+        "kernel_ms": {"before_decode": round(float(np.mean(wr_ms)), 5),
                       "decode": round(dec_avg_ms, 5)},
         "extra_bytes_per_step": {"split_scratch": int(np.mean([infos[i % V]["scratch"]
                                                                for i in range(K)])),
@@ -443,7 +463,7 @@ def run_e2e(args, steps, infos, torch, device, dist, world):
                                      block_tables=s.block_tables, context_lens=s.context_lens,
                                      max_context_len=s.max_context_len, scale=s.scale,
                                      partition_tokens=s.partition_tokens,
-                                     copy_pairs=s.copy_pairs))
+                                     copy_pairs=s.copy_pairs, fused=s.fused))
     graphs = [capture(h.run, torch) for h in hsteps]
     V = len(graphs)
     for i in range(args.warmup):

@@ -179,6 +179,37 @@ pa_status pa_decode_static_workspace(void *out, const void *q, const void *k_cac
                                      int num_blocks, float scale, pa_dtype dtype,
                                      int partition_tokens, void *stream);
 
+/* ------------------------------------------------------------------------------------------
+ * pa_decode_append -- one decode step: store every sequence's new K/V at its slot,
+ * then attend (pa_reshape_and_cache followed by pa_decode, in one call).
+ * [P3, section "为什么叫 PagedAttention" (the slot write) and the sources of
+ * pa_decode above; the order -- write, then attend over a history that includes
+ * the new token -- is this library's reading.]
+ *
+ *   k_new, v_new   device, [num_seqs][num_kv_heads][head_dim]: the new token of
+ *                  sequence b, which is its position context_lens[b] - 1
+ *   slot_mapping   device, int64 [num_seqs]: that token's slot; -1 stores nothing
+ *                  (pass -1 for sequences with context_lens[b] == 0)
+ *   k_cache, v_cache  updated in place; all other arguments as pa_decode
+ * Result: identical pools to pa_reshape_and_cache, outputs within the rounding
+ * of pa_decode. Where pa_decode runs its even-split kernel (2-8 q heads per kv
+ * head, power-of-two block_size >= 8) the write happens inside that kernel: the
+ * CTA that reads a sequence's last tile stores the new rows and uses them
+ * directly (one launch per step). Otherwise the write kernel runs first.
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                           const int64_t *slot_mapping, void *k_cache, void *v_cache,
+                           const int32_t *block_tables, int max_blocks_per_seq,
+                           const int32_t *context_lens, int max_context_len, int num_seqs,
+                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, float scale, pa_dtype dtype, void *workspace,
+                           size_t workspace_bytes, int partition_tokens, void *stream);
+
+/* Kernels one pa_decode_append call with these arguments launches (0 if none). */
+int pa_decode_append_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                              int block_size, int num_blocks, int max_context_len,
+                              int partition_tokens);
+
 /* Kernels one pa_decode call with these arguments launches (0 if none). */
 int pa_decode_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                        int block_size, int num_blocks, int max_context_len, int partition_tokens);

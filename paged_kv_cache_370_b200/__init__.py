@@ -9,7 +9,8 @@ Names are resolved from ``abi`` on first use, so that ``build`` can run
 before the library exists; using any of them without the library raises.
 """
 _EXPORTS = (
-    "BlockManager", "OutOfBlocks", "PAError", "pa_copy_blocks", "pa_decode",
+    "BlockManager", "OutOfBlocks", "PAError", "pa_copy_blocks", "pa_decode", "pa_decode_append",
+    "pa_decode_append_launches",
     "pa_decode_default_partition", "pa_decode_launches", "pa_decode_static_workspace",
     "pa_decode_workspace_size", "pa_device_status", "pa_reshape_and_cache", "pa_slot_mapping",
 )

@@ -58,6 +58,9 @@ def _load() -> ctypes.CDLL:
         "pa_decode": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, P, sz, i, P]),
         "pa_decode_default_partition": (i, [i, i, i]),
         "pa_decode_launches": (i, [i, i, i, i, i, i, i, i]),
+        "pa_decode_append": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, P, sz,
+                                 i, P]),
+        "pa_decode_append_launches": (i, [i, i, i, i, i, i, i, i]),
         "pa_decode_static_workspace": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P]),
         "pa_device_status": (i, [P, P]),
         "pa_status_string": (ctypes.c_char_p, [i]),
@@ -184,6 +187,31 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
                         _dtype_code(q), _dev_ptr(workspace, "workspace"), ws_bytes,
                         int(partition_tokens), _stream(stream))
     _check(st, "pa_decode")
+
+
+def pa_decode_append(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,
+                     context_lens, max_context_len, scale, workspace=None, partition_tokens=0,
+                     stream=None):
+    """One decode step: store k_new/v_new [B, Hkv, D] at slot_mapping[B] (the token at
+    position context_lens[b] - 1), then attend, as pa_reshape_and_cache + pa_decode."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.pa_decode_append(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_new, "k_new"), _dev_ptr(v_new, "v_new"),
+        _dev_ptr(slot_mapping, "slot_mapping"), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+        int(block_tables.shape[1]), _dev_ptr(context_lens, "context_lens"), int(max_context_len),
+        B, hq, hkv, d, bs, nb, float(scale), _dtype_code(q), _dev_ptr(workspace, "workspace"),
+        ws_bytes, int(partition_tokens), _stream(stream))
+    _check(st, "pa_decode_append")
+
+
+def pa_decode_append_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                              num_blocks, max_context_len, partition_tokens=0) -> int:
+    return int(_lib.pa_decode_append_launches(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                              block_size, num_blocks, max_context_len,
+                                              partition_tokens))
 
 
 def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_lens,

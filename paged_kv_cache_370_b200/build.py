@@ -60,7 +60,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
     objs = []
     for src in cu:
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        cmd = [nvcc, *ARCH_FLAGS, *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", "-c", src, "-o", obj]
+        extra = os.environ.get("PA370_NVCC_FLAGS", "").split()  # e.g. -DPA_STREAM_STAGES_D128=4
+        cmd = [nvcc, *ARCH_FLAGS, *NVCC_FLAGS, *extra, f"-I{INCLUDE}", f"-I{CSRC}", "-c", src, "-o",
+               obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.run(cmd, check=True)

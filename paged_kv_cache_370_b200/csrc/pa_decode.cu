@@ -221,6 +221,13 @@ struct DecodeParams {
   int grid_ctas;       // CTAs sharing the tiles
   int *ws_counters;    // [grid_ctas] pieces finished per split segment; zero between calls
   float *ws_pieces;    // [2 * grid_ctas][G][D + 4] partial (acc[D], max, sum, pad) per piece
+  // fused KV write (pa_decode_append): the new token of sequence b is position
+  // context_lens[b] - 1, with rows k_new[b], v_new[b] and slot new_slots[b]
+  const void *k_new;
+  const void *v_new;
+  const int64_t *new_slots;  // nullptr: no fused write
+  void *k_cache_w;
+  void *v_cache_w;
 };
 
 template <int D>
@@ -605,12 +612,25 @@ __global__ void __launch_bounds__(kThreads, 3)
 //    another.
 // Requires a power-of-two block size >= 8 (every TMA box then starts on a
 // 1024-byte boundary and blocks align with 64-token tiles).
+// Pipeline depth of the even-split kernel (stages of 64 tokens of K and V).
+#ifndef PA_STREAM_STAGES_D128
+#define PA_STREAM_STAGES_D128 3
+#endif
+#ifndef PA_STREAM_STAGES_D64
+#define PA_STREAM_STAGES_D64 4
+#endif
+
 namespace tc {
 
 constexpr int kTile = 64;            // tokens per stage
 constexpr int kWarps = 4;            // consumer warps, 16 tokens each
-constexpr int kThreads = (kWarps + 1) * 32;
+// two producer warps: warp kWarps stages K (plus per-tile metadata, q rows and
+// the new token), warp kWarps + 1 stages V. Issuing tensor copies takes the
+// issuing warp time in proportion to the bytes, so one issuer per CTA would cap
+// the CTA below its share of HBM bandwidth.
+constexpr int kThreads = (kWarps + 2) * 32;
 constexpr int kPanelBytes = kTile * 128;  // 64 columns of 2 bytes x 64 rows
+constexpr int kIdWindow = 8;             // tiles of block ids fetched ahead of their copies
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar) {
@@ -619,6 +639,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// 4-byte global -> shared copy that does not block the issuing thread
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -690,25 +722,32 @@ struct TileMeta {
   int seg_tiles;      // tiles of the segment
   int nvalid;         // valid tokens in this tile (0..64)
   int seg_first_x;    // global index of the segment's first tile
-  int flags;          // 1: first tile of this CTA's piece, 2: last tile of it
+  int flags;          // 1: first tile of this CTA's piece, 2: last tile of it,
+                      // 4: holds the sequence's new token (fused write)
   int pad;
+  long long new_slot;  // slot of the new token (flags & 4)
 };
 
 template <int D, int G>
 struct Cfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kStageBytes = 2 * kPanels * kPanelBytes;  // K panels then V panels
-  static constexpr int kStages = D == 128 ? 3 : 4;
+  static constexpr int kStages = D == 128 ? PA_STREAM_STAGES_D128 : PA_STREAM_STAGES_D64;
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kQBytes = G * D * 2;  // the q rows of one GQA group
   static constexpr int kQOffset = kRingBytes;
-  static constexpr int kRedOffset = kQOffset + kStages * kQBytes;
+  static constexpr int kNewBytes = 2 * D * 2;  // the new token's K and V rows
+  static constexpr int kNewOffset = kQOffset + kStages * kQBytes;
+  static constexpr int kRedOffset = kNewOffset + kStages * kNewBytes;
   static constexpr int kRedBytes = kWarps * G * D * 4;
   static constexpr int kMetaOffset = kRedOffset + kRedBytes;
   static constexpr int kBarOffset = kMetaOffset + kStages * (int)sizeof(TileMeta);
   static constexpr int kMlOffset = kBarOffset + 2 * kStages * 8;
-  static constexpr int kCtrlOffset = kMlOffset + kWarps * 8 * 2 * 4;
+  static constexpr int kIdsOffset = kMlOffset + kWarps * 8 * 2 * 4;
+  static constexpr int kCtrlOffset = kIdsOffset + 2 * kIdWindow * 8 * 4;  // one window per producer
   static constexpr int kBytes = 1024 + kCtrlOffset + 64;  // + slack to align the ring to 1 KB
+  // CTAs per SM the register budget is sized for
+  static constexpr int kMinCtas = D == 64 ? 3 : (G <= 4 ? 2 : 1);
 };
 
 // The CTA owning global tile x when W tiles are split evenly over n CTAs
@@ -735,12 +774,12 @@ __device__ __forceinline__ int clamp_len(int len, int cap, int max_len, bool &ba
 // floats per stored piece of one head: acc[D], max, sum and padding that keeps
 // every piece 16-byte aligned for vector access
 template <int D>
-constexpr int piece_stride() { return D + 4; }
+__host__ __device__ constexpr int piece_stride() { return D + 4; }
 
 __device__ __forceinline__ int seg_tiles(int len) { return len > 0 ? (len + kTile - 1) / kTile : 1; }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     pa_decode_stream_kernel(const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using C = Cfg<D, G>;
@@ -799,8 +838,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (x0 >= x1) return;  // nothing for this CTA (uniform)
   const int ntiles = (int)(x1 - x0);
 
-  if (warp == kWarps) {
-    // ===================================================================== producer
+  if (warp >= kWarps) {
+    // ==================================================================== producers
+    const bool v_producer = warp == kWarps + 1;
     // find the segment holding tile x0: sequences in order, kv heads inner
     long long pre = 0;
     int b = 0;
@@ -827,12 +867,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       pre += total;
     }
     int len_b = clamp_len(__ldg(p.context_lens + b), cap, p.max_context_len, bad);
+    // the next sequence's length, loaded ahead of need
+    int len_next = b + 1 < B ? __ldg(p.context_lens + b + 1) : 0;
+    const bool fused = p.new_slots != nullptr;
+    long long slot_b = fused ? __ldg(p.new_slots + b) : -1;
+    long long slot_next = fused && b + 1 < B ? __ldg(p.new_slots + b + 1) : -1;
     int tb = seg_tiles(len_b);
     int kvh = (int)((x0 - pre) / tb);
     int j = (int)((x0 - pre) % tb);
     const int box_rows = bs < kTile ? bs : kTile;
     const uint32_t box_bytes = 2u * C::kPanels * box_rows * 128u;
     const int32_t *tables = p.block_tables;
+    // boxes of the tile at (b, j) and this lane's block id for it (issued one tile
+    // ahead so the load overlaps the wait for a free stage)
+    auto tile_boxes = [&](int jj, int len) {
+      const int t0 = jj * kTile;
+      const int nv = max(0, min(kTile, len - t0));
+      return nv > 0 ? (bs <= kTile ? (t0 + nv - 1) / bs - t0 / bs + 1 : 1) : 0;
+    };
+    // Block ids travel through a window of kIdWindow tiles in shared memory, filled
+    // by non-blocking copies kIdWindow tiles ahead of use: the tables are mostly
+    // out of L2 (the K/V stream evicts them), so each id load costs a full HBM
+    // round trip that must overlap the copies of the tiles before it.
+    const uint32_t ids = smem_u32(smem + C::kIdsOffset) + (v_producer ? kIdWindow * 8 * 4 : 0);
+    int ab = b, akvh = kvh, aj = j, alen = len_b, atb = tb;  // cursor of the tile being fetched
+    auto fetch_ids = [&](int slot) {
+      if (lane < tile_boxes(aj, alen))
+        cp_async_4(ids + (slot * 8 + lane) * 4,
+                   tables + (size_t)ab * p.max_blocks_per_seq + (aj * kTile) / bs + lane);
+      cp_async_commit();
+    };
+    auto advance_ahead = [&]() {
+      if (++aj == atb) {
+        aj = 0;
+        if (++akvh == Hkv) {
+          akvh = 0;
+          if (++ab < B) {
+            alen = clamp_len(__ldg(p.context_lens + ab), cap, p.max_context_len, bad);
+            atb = seg_tiles(alen);
+          }
+        }
+      }
+    };
+    for (int k = 0; k < kIdWindow; ++k) {
+      if (k < ntiles) {
+        fetch_ids(k);
+        if (k + 1 < ntiles) advance_ahead();
+      } else {
+        cp_async_commit();  // keep one group per tile
+      }
+    }
+    int phys = -1;
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
@@ -842,20 +927,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // stage free? (after a give-up the loop runs on without waiting: no early exits)
       if (i >= NS) mbar_wait_bounded(&empty_bar[s], ((i / NS) & 1) ^ 1, abort_flag);
       __syncwarp();
+      // this tile's ids have landed once at most kIdWindow - 1 newer groups are pending
+      cp_async_wait<kIdWindow - 1>();
+      __syncwarp();
+      phys = lane < tile_boxes(j, len_b)
+                 ? reinterpret_cast<const int *>(smem + C::kIdsOffset +
+                                                 (v_producer ? kIdWindow * 8 * 4 : 0))[(i % kIdWindow) * 8 + lane]
+                 : -1;
       const int t0 = j * kTile;
       const int nvalid = max(0, min(kTile, len_b - t0));
       const bool seg_begin = (j == 0) || (i == 0);
       const bool seg_end = (j == tb - 1) || (i == ntiles - 1);
-      const int nbox = nvalid > 0 ? (bs <= kTile ? (t0 + nvalid - 1) / bs - t0 / bs + 1 : 1) : 0;
-      int phys = -1;
-      bool ok = false;
-      if (lane < nbox) {
-        phys = __ldg(tables + (size_t)b * p.max_blocks_per_seq + t0 / bs + lane);
-        ok = phys >= 0 && phys < p.num_blocks;
-        if (!ok) atomicOr(&g_decode_error, PA_DEVERR_BLOCK_ID);
-      }
+      const bool new_tok = fused && j == tb - 1 && len_b > 0;  // tile of position len - 1
+      const bool ok = lane < tile_boxes(j, len_b) && phys >= 0 && phys < p.num_blocks;
+      if (lane < tile_boxes(j, len_b) && !ok && !v_producer)
+        atomicOr(&g_decode_error, PA_DEVERR_BLOCK_ID);
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
-      if (lane == 0) {
+      if (lane == 0 && !v_producer) {
         TileMeta &m = meta[s];
         m.b = b;
         m.kvh = kvh;
@@ -863,38 +951,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         m.seg_tiles = tb;
         m.nvalid = nvalid;
         m.seg_first_x = (int)(x0 + i - j);
-        m.flags = (seg_begin ? 1 : 0) | (seg_end ? 2 : 0);
+        m.flags = (seg_begin ? 1 : 0) | (seg_end ? 2 : 0) | (new_tok ? 4 : 0);
+        m.new_slot = slot_b;
         mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes +
-                                                (seg_begin ? (uint32_t)C::kQBytes : 0u));
+                                                (seg_begin ? (uint32_t)C::kQBytes : 0u) +
+                                                (new_tok ? (uint32_t)C::kNewBytes : 0u));
       }
       __syncwarp();
       const uint32_t stage = ring + s * C::kStageBytes;
-      if (ok) {
-        // box of block t0/bs + lane: whole block (bs <= 64) or a 64-row slice (bs > 64)
-        const int r0 = bs > kTile ? t0 % bs : 0;
-        const int row = bs > kTile ? 0 : lane * bs;
-        const int y = (phys * Hkv + kvh) * bs + r0;
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_2d(stage + pn * kPanelBytes + row * 128, &tmap_k, pn * 64, y, &full_bar[s]);
-          tma_load_2d(stage + (C::kPanels + pn) * kPanelBytes + row * 128, &tmap_v, pn * 64, y,
-                      &full_bar[s]);
+      {
+        // one copy per lane: (box, panel) of this producer's operand (K or V)
+        const int box = lane / C::kPanels;
+        const int which = v_producer ? 1 : 0;
+        const int pn = lane % C::kPanels;
+        const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
+        const bool box_ok = box < 32 && ((okmask >> (box & 31)) & 1u);
+        if (box_ok) {
+          // box of block t0/bs + box: whole block (bs <= 64) or a 64-row slice (bs > 64)
+          const int r0 = bs > kTile ? t0 % bs : 0;
+          const int row = bs > kTile ? 0 : box * bs;
+          const int y = (box_phys * Hkv + kvh) * bs + r0;
+          tma_load_2d(stage + (which * C::kPanels + pn) * kPanelBytes + row * 128,
+                      which ? &tmap_v : &tmap_k, pn * 64, y, &full_bar[s]);
         }
       }
-      if (lane == 0 && seg_begin)
+      if (lane == 0 && seg_begin && !v_producer)
         bulk_g2s(smem + C::kQOffset + s * C::kQBytes,
                  static_cast<const T *>(p.q) + ((size_t)b * p.num_q_heads + (size_t)kvh * G) * D,
                  C::kQBytes, &full_bar[s]);
+      if (lane == 0 && new_tok && !v_producer) {
+        const size_t row = ((size_t)b * Hkv + kvh) * D;
+        unsigned char *dst = smem + C::kNewOffset + s * C::kNewBytes;
+        bulk_g2s(dst, static_cast<const T *>(p.k_new) + row, D * 2, &full_bar[s]);
+        bulk_g2s(dst + D * 2, static_cast<const T *>(p.v_new) + row, D * 2, &full_bar[s]);
+      }
       // next tile: kv heads inner, then sequences
-      if (++j == tb) {
-        j = 0;
-        if (++kvh == Hkv) {
-          kvh = 0;
-          if (++b < B) {
-            len_b = clamp_len(__ldg(p.context_lens + b), cap, p.max_context_len, bad);
+      if (i + 1 < ntiles) {
+        if (++j == tb) {
+          j = 0;
+          if (++kvh == Hkv) {
+            kvh = 0;
+            ++b;
+            len_b = clamp_len(len_next, cap, p.max_context_len, bad);
             tb = seg_tiles(len_b);
+            len_next = b + 1 < B ? __ldg(p.context_lens + b + 1) : 0;
+            slot_b = slot_next;
+            slot_next = fused && b + 1 < B ? __ldg(p.new_slots + b + 1) : -1;
           }
         }
+      }
+      // refill the window slot just used with the ids of tile i + kIdWindow
+      if (i + kIdWindow < ntiles) {
+        fetch_ids(i % kIdWindow);
+        if (i + kIdWindow + 1 < ntiles) advance_ahead();
+      } else {
+        cp_async_commit();
       }
     }
     // do not leave while copies may still land in this CTA's shared memory
@@ -950,6 +1061,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       l0 = l1 = 0.f;
     }
     const int nvalid = mt.nvalid;
+    if ((mt.flags & 4) && (nvalid - 1) / 16 == warp) {
+      // fused write: the new token (last valid row) replaces what the cache held
+      // in this tile, and is stored at its slot for later steps
+      constexpr int kChunks = D / 8;  // 16-byte chunks per row
+      const int r = nvalid - 1;
+      if (lane < 2 * kChunks) {
+        const int which = lane / kChunks, c = lane % kChunks;  // which: 0 = K, 1 = V
+        const uint4 v = *reinterpret_cast<const uint4 *>(smem + C::kNewOffset +
+                                                         s * C::kNewBytes + which * D * 2 + c * 16);
+        unsigned char *panel = smem + s * C::kStageBytes + (which * C::kPanels + c / 8) * kPanelBytes;
+        *reinterpret_cast<uint4 *>(panel + r * 128 + (((c % 8) ^ (r & 7)) << 4)) = v;
+        const long long slot = mt.new_slot;
+        if (slot >= 0 && slot < (long long)p.num_blocks * bs) {
+          const long long blk = slot / bs, off = slot - blk * bs;
+          unsigned char *cache = static_cast<unsigned char *>(which ? p.v_cache_w : p.k_cache_w);
+          *reinterpret_cast<uint4 *>(cache + (((size_t)blk * Hkv + mt.kvh) * bs + off) * D * 2 +
+                                     c * 16) = v;
+        } else if (slot >= 0 && lane == 0) {
+          atomicOr(&g_decode_error, PA_DEVERR_SLOT);
+        }
+      }
+      __syncwarp();
+    }
     if (nvalid < wrow + 16) {
       // rows past the valid tokens may hold anything (0 * NaN would poison the
       // product): zero this warp's own V rows there before reading them
@@ -1457,12 +1591,24 @@ extern "C" int pa_decode_launches(int num_seqs, int num_q_heads, int num_kv_head
   return max_context_len > pt ? 2 : 1;
 }
 
-extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
-                               const int32_t *block_tables, int max_blocks_per_seq,
-                               const int32_t *context_lens, int max_context_len, int num_seqs,
-                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                               int num_blocks, float scale, pa_dtype dtype, void *workspace,
-                               size_t workspace_bytes, int partition_tokens, void *stream) {
+namespace {
+
+// The new token of every sequence, written by the decode kernel itself.
+struct FusedWrite {
+  const void *k_new;
+  const void *v_new;
+  const int64_t *slots;
+  void *k_cache;
+  void *v_cache;
+};
+
+pa_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, int max_blocks_per_seq,
+                      const int32_t *context_lens, int max_context_len, int num_seqs,
+                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, float scale, pa_dtype dtype, void *workspace,
+                      size_t workspace_bytes, int partition_tokens, void *stream,
+                      const FusedWrite *fw) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
       block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
       (dtype != PA_F16 && dtype != PA_BF16))
@@ -1512,6 +1658,12 @@ extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, co
   prm.grid_ctas = nctas;
   prm.ws_counters = streamk ? static_cast<int *>(workspace) : nullptr;
   prm.ws_pieces = streamk ? ws_body : nullptr;
+  prm.k_new = fw ? fw->k_new : nullptr;
+  prm.v_new = fw ? fw->v_new : nullptr;
+  prm.new_slots = fw ? fw->slots : nullptr;
+  prm.k_cache_w = fw ? fw->k_cache : nullptr;
+  prm.v_cache_w = fw ? fw->v_cache : nullptr;
+  if (fw && !streamk) return PA_ERR_INVALID;  // only the even-split kernel writes
   prm.max_blocks_per_seq = max_blocks_per_seq;
   prm.max_context_len = max_context_len;
   prm.num_q_heads = num_q_heads;
@@ -1528,6 +1680,66 @@ extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, co
   if (dtype == PA_BF16)
     return dispatch_dim<__nv_bfloat16>(head_dim, group, prm, num_seqs, out, dtype, st);
   return dispatch_dim<__half>(head_dim, group, prm, num_seqs, out, dtype, st);
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                               const int32_t *block_tables, int max_blocks_per_seq,
+                               const int32_t *context_lens, int max_context_len, int num_seqs,
+                               int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int num_blocks, float scale, pa_dtype dtype, void *workspace,
+                               size_t workspace_bytes, int partition_tokens, void *stream) {
+  return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, partition_tokens,
+                     stream, nullptr);
+}
+
+extern "C" int pa_decode_append_launches(int num_seqs, int num_q_heads, int num_kv_heads,
+                                         int head_dim, int block_size, int num_blocks,
+                                         int max_context_len, int partition_tokens) {
+  const int decode = pa_decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                        block_size, num_blocks, max_context_len,
+                                        partition_tokens);
+  if (decode == 0) return 0;
+  const int group = num_q_heads / num_kv_heads;
+  return uses_stream_kernel(group, block_size, num_blocks, num_kv_heads) ? 1 : 1 + decode;
+}
+
+extern "C" pa_status pa_decode_append(void *out, const void *q, const void *k_new,
+                                      const void *v_new, const int64_t *slot_mapping,
+                                      void *k_cache, void *v_cache, const int32_t *block_tables,
+                                      int max_blocks_per_seq, const int32_t *context_lens,
+                                      int max_context_len, int num_seqs, int num_q_heads,
+                                      int num_kv_heads, int head_dim, int block_size,
+                                      int num_blocks, float scale, pa_dtype dtype,
+                                      void *workspace, size_t workspace_bytes,
+                                      int partition_tokens, void *stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+      block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!k_new || !v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+      !aligned(slot_mapping, 8))
+    return PA_ERR_INVALID;
+  const int group = num_q_heads / num_kv_heads;
+  if (uses_stream_kernel(group, block_size, num_blocks, num_kv_heads)) {
+    const FusedWrite fw{k_new, v_new, slot_mapping, k_cache, v_cache};
+    return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                       max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       block_size, num_blocks, scale, dtype, workspace, workspace_bytes,
+                       partition_tokens, stream, &fw);
+  }
+  // other shapes: the write kernel, then the decode
+  const pa_status st = pa_reshape_and_cache(k_new, v_new, slot_mapping, num_seqs, k_cache,
+                                            v_cache, num_blocks, num_kv_heads, block_size,
+                                            head_dim, dtype, stream);
+  if (st != PA_OK) return st;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, partition_tokens,
+                     stream, nullptr);
 }
 
 pa_status pa_internal_decode_status(cudaStream_t stream, int32_t *code) {

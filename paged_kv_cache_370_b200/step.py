@@ -22,7 +22,10 @@ from . import abi
 class DecodeStep:
     def __init__(self, *, k_cache, v_cache, q, k_new, v_new, slot_mapping, block_tables,
                  context_lens, max_context_len: int, scale: float, partition_tokens: int = 0,
-                 copy_pairs=None, out=None):
+                 copy_pairs=None, out=None, fused: bool = False):
+        """``fused``: write the new tokens inside the decode (pa_decode_append);
+        k_new/v_new then hold one token per sequence, at position len - 1."""
+        self.fused = fused
         self.k_cache, self.v_cache = k_cache, v_cache
         self.q, self.k_new, self.v_new = q, k_new, v_new
         self.slot_mapping = slot_mapping
@@ -43,12 +46,15 @@ class DecodeStep:
         self.decode_launches = abi.pa_decode_launches(B, hq, hkv, d, bs, nb,
                                                       self.max_context_len,
                                                       self.partition_tokens)
+        self.append_launches = abi.pa_decode_append_launches(B, hq, hkv, d, bs, nb,
+                                                             self.max_context_len,
+                                                             self.partition_tokens)
         self.partition = self.partition_tokens or abi.pa_decode_default_partition(
             B, hkv, self.max_context_len)
 
     def launches(self) -> int:
         """Kernels one run() launches."""
-        n = 1 + self.decode_launches
+        n = self.append_launches if self.fused else 1 + self.decode_launches
         if self.copy_pairs is not None and self.copy_pairs.numel():
             n += 1
         return n
@@ -66,10 +72,19 @@ class DecodeStep:
                       self.context_lens, self.max_context_len, self.scale, self.workspace,
                       self.partition_tokens, stream)
 
+    def append(self, stream=None):
+        abi.pa_decode_append(self.out, self.q, self.k_new, self.v_new, self.slot_mapping,
+                             self.k_cache, self.v_cache, self.block_tables, self.context_lens,
+                             self.max_context_len, self.scale, self.workspace,
+                             self.partition_tokens, stream)
+
     def run(self, stream=None):
         self.copy(stream)
-        self.write(stream)
-        self.attend(stream)
+        if self.fused:
+            self.append(stream)
+        else:
+            self.write(stream)
+            self.attend(stream)
         return self.out
 
 
@@ -84,7 +99,7 @@ class HostDecodeStep:
 
     def __init__(self, *, k_cache, v_cache, q, k_new, v_new, slot_mapping, block_tables,
                  context_lens, max_context_len: int, scale: float, partition_tokens: int = 0,
-                 copy_pairs=None):
+                 copy_pairs=None, fused: bool = False):
         dev = k_cache.device
         parts = {"q": q, "k_new": k_new, "v_new": v_new, "slot_mapping": slot_mapping,
                  "block_tables": block_tables, "context_lens": context_lens}
@@ -109,7 +124,7 @@ class HostDecodeStep:
                                context_lens=views["context_lens"],
                                max_context_len=max_context_len, scale=scale,
                                partition_tokens=partition_tokens,
-                               copy_pairs=views.get("copy_pairs"))
+                               copy_pairs=views.get("copy_pairs"), fused=fused)
         self.h_out = torch.empty(tuple(q.shape), dtype=q.dtype).pin_memory()
 
     @property

@@ -40,7 +40,8 @@ class GpuBatch:
     at slots from pa_slot_mapping, and a DecodeStep that writes each sequence's
     last token and decodes."""
 
-    def __init__(self, batch, partition_tokens: int = 0, device="cuda", tables=None):
+    def __init__(self, batch, partition_tokens: int = 0, device="cuda", tables=None,
+                 fused: bool = False):
         self.batch = batch
         bs, dt = batch.block_size, batch.dtype
         shape = (batch.num_blocks, batch.num_kv_heads, bs, batch.head_dim)
@@ -77,7 +78,7 @@ class GpuBatch:
             block_tables=torch.from_numpy(np.ascontiguousarray(self.tables_np)).to(device),
             context_lens=torch.from_numpy(batch.context_lens).to(device),
             max_context_len=max(batch.max_context_len, 1), scale=float(batch.scale),
-            partition_tokens=partition_tokens)
+            partition_tokens=partition_tokens, fused=fused)
 
     def run(self):
         out = self.step.run()
@@ -177,7 +178,7 @@ def _step_appends(script, append):
 SHARED_TABLE_WIDTH = 48
 
 
-def shared_prompt_gpu(script, device="cuda"):
+def shared_prompt_gpu(script, device="cuda", fused=False):
     bs, H, D = script.block_size, script.num_heads, script.head_dim
     mgr = abi.BlockManager(script.num_blocks, bs)
     shape = (script.num_blocks, H, bs, D)
@@ -195,7 +196,7 @@ def shared_prompt_gpu(script, device="cuda"):
                       block_tables=torch.from_numpy(tables).to(device),
                       context_lens=torch.from_numpy(lens).to(device),
                       max_context_len=int(lens.max()), scale=float(script.scale),
-                      copy_pairs=torch.from_numpy(pairs).to(device))
+                      copy_pairs=torch.from_numpy(pairs).to(device), fused=fused)
     return mgr, step, tables, lens, pairs
 
 

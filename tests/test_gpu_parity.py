@@ -29,8 +29,8 @@ def _status_clean():
     assert code == 0, f"device error word {code:#x}"
 
 
-def _run_and_compare(batch, partition_tokens=0, full_pool=True):
-    g = GpuBatch(batch, partition_tokens=partition_tokens)
+def _run_and_compare(batch, partition_tokens=0, full_pool=True, fused=False):
+    g = GpuBatch(batch, partition_tokens=partition_tokens, fused=fused)
     out = widen_out(g.run())
     kp, vp = oracle_pools(batch, full=full_pool)
     if full_pool:
@@ -67,14 +67,15 @@ SHAPES = [
 ]
 
 
-@pytest.mark.parametrize("pt", [0, 64, 192])
+@pytest.mark.parametrize("mode", ["pt0", "pt64", "pt192", "fused", "fused_pt64"])
 @pytest.mark.parametrize("shape", range(len(SHAPES)))
-def test_shapes(shape, pt):
+def test_shapes(shape, mode):
     hq, hkv, d, dt, bs, lens = SHAPES[shape]
     width = max(1, -(-max(lens) // bs))
     nb = len(lens) * width + 3
     batch = synth.small_random(100 + shape, len(lens), lens, hq, hkv, d, bs, nb, dt, width)
-    _run_and_compare(batch, partition_tokens=pt)
+    pt = int(mode.split("pt")[1]) if "pt" in mode else 0
+    _run_and_compare(batch, partition_tokens=pt, fused=mode.startswith("fused"))
 
 
 def test_partitions_agree():
@@ -189,8 +190,8 @@ def _sampled_pool_check(g, batch):
     assert np.array_equal(k_rows, batch.k[pick]) and np.array_equal(v_rows, batch.v[pick])
 
 
-def _full_size(batch, partition_tokens=0):
-    g = GpuBatch(batch, partition_tokens=partition_tokens)
+def _full_size(batch, partition_tokens=0, fused=False):
+    g = GpuBatch(batch, partition_tokens=partition_tokens, fused=fused)
     out = widen_out(g.run())
     _status_clean()
     _sampled_pool_check(g, batch)
@@ -203,6 +204,28 @@ def _full_size(batch, partition_tokens=0):
 
 def test_llama8b_full():
     _full_size(synth.llama8b())
+
+
+@pytest.mark.parametrize("make", [synth.llama8b, synth.long_skew], ids=["llama8b", "long_skew"])
+def test_fused_write_full(make):
+    batch = make()
+    g, out, s = _full_size(batch, fused=True)
+    assert g.step.launches() == 1  # write and decode in one kernel
+    # the fused write leaves exactly the pool the separate write kernel leaves
+    ref = GpuBatch(batch)
+    ref.run()
+    assert torch.equal(ref.k_cache.view(torch.int16), g.k_cache.view(torch.int16))
+    assert torch.equal(ref.v_cache.view(torch.int16), g.v_cache.view(torch.int16))
+
+
+def test_fused_write_reports_bad_slots():
+    batch = synth.small_random(16, 3, [40, 70, 9], 8, 2, 128, 16, 20, "bf16")
+    g = GpuBatch(batch, fused=True)
+    g.run()
+    _status_clean()
+    g.step.slot_mapping[1] = batch.num_blocks * batch.block_size + 7
+    g.run()
+    assert abi.pa_device_status() & abi.PA_DEVERR_SLOT
 
 
 def test_long_skew_full():
@@ -223,9 +246,10 @@ def test_mixed_sweep_full():
         assert np.array_equal(o, outs[0]), "block size changed the output bits"
 
 
-def test_shared_prompt_copy_on_write():
+@pytest.mark.parametrize("fused", [False, True])
+def test_shared_prompt_copy_on_write(fused):
     script = synth.shared_prompt()
-    mgr, step, tables, lens, pairs = shared_prompt_gpu(script)
+    mgr, step, tables, lens, pairs = shared_prompt_gpu(script, fused=fused)
     assert len(pairs) == script.num_prompts  # one copy-on-write per prompt
     out = widen_out(step.run())
     torch.cuda.synchronize()
