@@ -67,6 +67,10 @@ def _load(path: str):
     L.oracle_decode_partitioned.argtypes = [P, P, P, P, P, i, P, i, i, i, i, i, i, f, i,
                                             i, i, P, P, P, i]
     L.oracle_max_threads.restype = i
+    L.oracle_decode_window.restype = i
+    L.oracle_decode_window.argtypes = [P, P, P, P, P, i, P, i, i, i, i, i, i, f, i, i, i]
+    L.oracle_swap_blocks.restype = i
+    L.oracle_swap_blocks.argtypes = [P, P, i, P, P, i, P, i, i, i, i]
     L.oracle_max_threads.argtypes = []
     return L
 
@@ -170,6 +174,18 @@ def copy_blocks(k_cache, v_cache, block_pairs):
     _check(rc, "oracle_copy_blocks")
 
 
+def swap_blocks(dst_k, dst_v, src_k, src_v, block_pairs):
+    """dst pools [block] = src pools [block] for each (src, dst) pair (K and V)."""
+    nd, hkv, bs, d = dst_k.shape
+    ns = src_k.shape[0]
+    assert src_k.shape[1:] == dst_k.shape[1:]
+    pairs = _need(np.ascontiguousarray(block_pairs, dtype=np.int64).reshape(-1, 2), np.int64)
+    rc = lib().oracle_swap_blocks(_ptr(_need(dst_k, np.uint16)), _ptr(_need(dst_v, np.uint16)), nd,
+                                  _ptr(_need(src_k, np.uint16)), _ptr(_need(src_v, np.uint16)), ns,
+                                  _ptr(pairs), len(pairs), hkv, bs, d)
+    _check(rc, "oracle_swap_blocks")
+
+
 def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype, num_threads=0):
     """fp64 outputs [B, Hq, D] of paged decode attention (unrounded)."""
     B, hq, d = q.shape
@@ -182,6 +198,25 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype, num_th
                              _ptr(_need(v_cache, np.uint16)), _ptr(bt), bt.shape[1], _ptr(cl), B,
                              hq, hkv, d, bs, nb, float(scale), DTYPE_CODE[dtype], num_threads)
     _check(rc, "oracle_decode")
+    return out
+
+
+def decode_window(q, k_cache, v_cache, block_tables, context_lens, scale, dtype, window,
+                  num_threads=0):
+    """fp64 outputs [B, Hq, D] of sliding-window decode: each sequence attends to
+    its last ``window`` positions (``window`` <= 0: all of them)."""
+    B, hq, d = q.shape
+    nb, hkv, bs, d2 = k_cache.shape
+    assert d == d2
+    out = np.zeros((B, hq, d), dtype=np.float64)
+    bt = _need(np.ascontiguousarray(block_tables, dtype=np.int32), np.int32)
+    cl = _need(np.ascontiguousarray(context_lens, dtype=np.int32), np.int32)
+    rc = lib().oracle_decode_window(_ptr(out), _ptr(_need(q, np.uint16)),
+                                    _ptr(_need(k_cache, np.uint16)),
+                                    _ptr(_need(v_cache, np.uint16)), _ptr(bt), bt.shape[1],
+                                    _ptr(cl), B, hq, hkv, d, bs, nb, float(scale),
+                                    DTYPE_CODE[dtype], int(window), num_threads)
+    _check(rc, "oracle_decode_window")
     return out
 
 

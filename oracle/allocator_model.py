@@ -22,13 +22,28 @@ It restates, one step at a time, what the pages say a block manager does:
   count is above one, a new block is allocated, the old block's contents
   are copied into it, the table entry is pointed at the new block and the
   old block's count drops by one (second page, section 2.3). A sole owner
-  writes in place.
+  writes in place;
+* sliding window: blocks that fall wholly out of the attention window are
+  given back (second page, section 5.2). Here a block is out of the window
+  of length W when all its positions precede len - W; the sequence drops its
+  reference and its table entry becomes -1;
+* swapping: a preempted request's blocks move to CPU memory and come back
+  later (third page, section "分页还顺带解决了什么"; second page, section 3.1,
+  swap_out of a victim). Here a group of sequences moves together: each
+  distinct block the group uses is copied once into a free host block (its
+  host count = the group's references), the device block loses those
+  references, and the tables then name host blocks; swapping in is the
+  mirror image. A block also used outside the group stays where it is for
+  the others, so the group gets its own copy.
 
 Which physical id the free list hands out is not fixed by the pages; this
 model pops the most recently freed block (a LIFO stack). Tests compare the
 product allocator with this model only up to a relabelling of ids.
 """
 from __future__ import annotations
+
+
+RELEASED = -1  # table entry of a block given back by the sliding window
 
 
 class OutOfBlocks(RuntimeError):
@@ -49,6 +64,9 @@ class BlockManagerModel:
         self.ref = [0] * num_blocks
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
+        self.swapped: set[int] = set()
+        self.host_free: list[int] = []
+        self.host_ref: list[int] = []
 
     # -- allocation ---------------------------------------------------------------------------
     def _blocks_for(self, num_tokens: int) -> int:
@@ -77,20 +95,21 @@ class BlockManagerModel:
 
     def fork(self, parent: int, child: int):
         """The child shares every block of the parent; each gains a reference."""
-        if parent not in self.tables or child in self.tables:
+        if parent not in self.tables or child in self.tables or parent in self.swapped:
             raise BadState("bad fork")
         self.tables[child] = list(self.tables[parent])
         self.lens[child] = self.lens[parent]
         for blk in self.tables[child]:
-            self.ref[blk] += 1
+            if blk != RELEASED:
+                self.ref[blk] += 1
 
     def append_slot(self, seq: int):
         """Reserve the slot of the sequence's next token.
 
         Returns (slot, cow_src, cow_dst); cow_* are -1 unless the write had
         to copy a shared block first. Nothing changes if no block is free."""
-        if seq not in self.tables:
-            raise BadState(f"no sequence {seq}")
+        if seq not in self.tables or seq in self.swapped:
+            raise BadState(f"no resident sequence {seq}")
         table = self.tables[seq]
         pos = self.lens[seq]
         logical = pos // self.block_size
@@ -113,18 +132,99 @@ class BlockManagerModel:
         go back on the free list."""
         if seq not in self.tables:
             raise BadState(f"no sequence {seq}")
+        ref, free = (self.host_ref, self.host_free) if seq in self.swapped else (self.ref, self.free)
         for blk in reversed(self.tables.pop(seq)):
-            if self.ref[blk] <= 0:
+            if blk == RELEASED:
+                continue
+            if ref[blk] <= 0:
                 raise BadState("reference count underflow")
+            ref[blk] -= 1
+            if ref[blk] == 0:
+                free.append(blk)
+        del self.lens[seq]
+        self.swapped.discard(seq)
+
+    def slide_window(self, seq: int, window: int) -> int:
+        """Give back every block whose positions all precede len - window.
+        Returns how many blocks went back on the free list."""
+        if seq not in self.tables or seq in self.swapped:
+            raise BadState(f"no resident sequence {seq}")
+        if window <= 0:
+            raise ValueError("window must be positive")
+        start = max(0, self.lens[seq] - window)      # first position inside the window
+        table = self.tables[seq]
+        freed = 0
+        for i in range(start // self.block_size):     # blocks ending at or before start
+            blk = table[i]
+            if blk == RELEASED:
+                continue
+            table[i] = RELEASED
             self.ref[blk] -= 1
             if self.ref[blk] == 0:
                 self.free.append(blk)
-        del self.lens[seq]
+                freed += 1
+        return freed
+
+    # -- swapping -----------------------------------------------------------------------------
+    def set_host_blocks(self, num_host_blocks: int):
+        if self.host_ref:
+            raise BadState("swap space already set")
+        self.host_ref = [0] * num_host_blocks
+        self.host_free = list(range(num_host_blocks - 1, -1, -1))
+
+    def _swap(self, seqs, out: bool):
+        if not self.host_ref:
+            raise BadState("no swap space")
+        if len(set(seqs)) != len(seqs):
+            raise ValueError("sequence listed twice")
+        for s in seqs:
+            if s not in self.tables or (s in self.swapped) == out:
+                raise BadState(f"sequence {s} is not on the side it leaves")
+        order, refs = [], {}
+        for s in seqs:
+            for blk in self.tables[s]:
+                if blk == RELEASED:
+                    continue
+                if blk not in refs:
+                    refs[blk] = 0
+                    order.append(blk)
+                refs[blk] += 1
+        src_ref, src_free = (self.ref, self.free) if out else (self.host_ref, self.host_free)
+        dst_ref, dst_free = (self.host_ref, self.host_free) if out else (self.ref, self.free)
+        if len(order) > len(dst_free):
+            raise OutOfBlocks(f"need {len(order)} blocks on the other side, {len(dst_free)} free")
+        moved, pairs = {}, []
+        for blk in order:
+            new = dst_free.pop()
+            dst_ref[new] = refs[blk]
+            src_ref[blk] -= refs[blk]
+            if src_ref[blk] == 0:
+                src_free.append(blk)
+            moved[blk] = new
+            pairs.append((blk, new))
+        for s in seqs:
+            self.tables[s] = [moved[b] if b != RELEASED else RELEASED for b in self.tables[s]]
+            if out:
+                self.swapped.add(s)
+            else:
+                self.swapped.discard(s)
+        return pairs
+
+    def swap_out(self, seqs):
+        """Move a group to the host swap space; returns (device block, host block) pairs."""
+        return self._swap(list(seqs), True)
+
+    def swap_in(self, seqs):
+        """Bring a swapped group back; returns (host block, device block) pairs."""
+        return self._swap(list(seqs), False)
 
     # -- queries ------------------------------------------------------------------------------
     def slot(self, seq: int, pos: int) -> int:
         table = self.tables[seq]
-        return table[pos // self.block_size] * self.block_size + pos % self.block_size
+        blk = table[pos // self.block_size]
+        if blk == RELEASED:
+            raise BadState("position released by the sliding window")
+        return blk * self.block_size + pos % self.block_size
 
     def seq_slots(self, seq: int, start: int, count: int) -> list[int]:
         return [self.slot(seq, p) for p in range(start, start + count)]
@@ -142,8 +242,12 @@ class BlockManagerModel:
         sequence referencing it has stored in it."""
         filled: dict[int, int] = {}
         for seq, table in self.tables.items():
+            if seq in self.swapped:
+                continue
             n = self.lens[seq]
             for i, blk in enumerate(table):
+                if blk == RELEASED:
+                    continue
                 f = min(self.block_size, n - i * self.block_size)
                 filled[blk] = max(filled.get(blk, 0), max(f, 0))
         used_blocks = self.num_blocks - len(self.free)

@@ -452,6 +452,108 @@ int oracle_decode_partitioned(double *out, const uint16_t *q, const uint16_t *k_
 }
 
 /* Threads the OpenMP runtime would use for num_threads = 0. */
+/* Swap: copy whole blocks (every KV head, every slot, K and V) between two
+ * pools of the same block shape -- device blocks out to a host swap space, or
+ * back ("08. PagedAttention：把 KV Cache 分页管理", section "分页还顺带解决了什么":
+ * a preempted request's blocks move to CPU memory and return later; blocks of
+ * one size make the move simple). For each (src, dst) of `block_pairs`
+ * ([num_pairs][2]): dst_pool[dst] = src_pool[src], in pair order. */
+int oracle_swap_blocks(uint16_t *dst_k, uint16_t *dst_v, int dst_blocks, const uint16_t *src_k,
+                       const uint16_t *src_v, int src_blocks, const int64_t *block_pairs,
+                       int num_pairs, int num_kv_heads, int block_size, int head_dim)
+{
+    size_t block_elems = (size_t)num_kv_heads * block_size * head_dim;
+    for (int p = 0; p < num_pairs; ++p) {
+        int64_t src = block_pairs[2 * p], dst = block_pairs[2 * p + 1];
+        if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks)
+            return ORC_BAD_BLOCK;
+        for (size_t i = 0; i < block_elems; ++i) {
+            dst_k[(size_t)dst * block_elems + i] = src_k[(size_t)src * block_elems + i];
+            dst_v[(size_t)dst * block_elems + i] = src_v[(size_t)src * block_elems + i];
+        }
+    }
+    return ORC_OK;
+}
+
+/* Sliding-window decode ("PagedAttention 核心思想解析", section 5.2: blocks
+ * that fall out of the window are reclaimed). Each sequence attends only to
+ * its last `window` positions, [lo, n) with lo = max(0, n - window); window
+ * <= 0 means no window (all n positions). Only the positions in [lo, n) are
+ * looked up, so table entries of blocks wholly before lo may hold anything
+ * (a freed block's entry). Same arguments and output as oracle_decode. */
+static int gather_span(double *dst, const uint16_t *pool, const int32_t *table_row, int lo,
+                       int n, int kv_head, int num_blocks, int num_kv_heads, int block_size,
+                       int head_dim, int dtype)
+{
+    for (int t = lo; t < n; ++t) {
+        int64_t slot = oracle_slot(table_row, t, block_size);
+        int64_t block = slot / block_size;
+        int offset = (int)(slot % block_size);
+        if (block < 0 || block >= num_blocks)
+            return ORC_BAD_BLOCK;
+        for (int d = 0; d < head_dim; ++d)
+            dst[(size_t)(t - lo) * head_dim + d] =
+                widen(pool[pool_index(block, kv_head, offset, d, num_kv_heads, block_size,
+                                      head_dim)], dtype);
+    }
+    return ORC_OK;
+}
+
+int oracle_decode_window(double *out, const uint16_t *q, const uint16_t *k_cache,
+                         const uint16_t *v_cache, const int32_t *block_tables,
+                         int max_blocks_per_seq, const int32_t *context_lens, int num_seqs,
+                         int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                         int num_blocks, float scale, int dtype, int window, int num_threads)
+{
+    int rc = check_shapes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                          num_blocks, max_blocks_per_seq);
+    if (rc)
+        return rc;
+    for (int b = 0; b < num_seqs; ++b)
+        if (context_lens[b] < 0 || context_lens[b] > max_blocks_per_seq * block_size)
+            return ORC_BAD_ARG;
+    int group = num_q_heads / num_kv_heads;
+    int nthreads = set_threads(num_threads);
+    int status = ORC_OK;
+    long long units = (long long)num_seqs * num_q_heads;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (long long u = 0; u < units; ++u) {
+        int b = (int)(u / num_q_heads), h = (int)(u % num_q_heads);
+        int n = context_lens[b];
+        int lo = (window > 0 && n > window) ? n - window : 0;
+        int m = n - lo;
+        int g = h / group;
+        double *K = malloc(sizeof(double) * ((size_t)m * head_dim + 1));
+        double *V = malloc(sizeof(double) * ((size_t)m * head_dim + 1));
+        double *s = malloc(sizeof(double) * ((size_t)m + 1));
+        double *qd = malloc(sizeof(double) * (size_t)head_dim);
+        const int32_t *row = block_tables + (size_t)b * max_blocks_per_seq;
+        int r1 = gather_span(K, k_cache, row, lo, n, g, num_blocks, num_kv_heads, block_size,
+                             head_dim, dtype);
+        int r2 = gather_span(V, v_cache, row, lo, n, g, num_blocks, num_kv_heads, block_size,
+                             head_dim, dtype);
+        if (r1 || r2) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+            status = ORC_BAD_BLOCK;
+        } else {
+            for (int d = 0; d < head_dim; ++d)
+                qd[d] = widen(q[((size_t)b * num_q_heads + h) * head_dim + d], dtype);
+            attend_rows(out + ((size_t)b * num_q_heads + h) * head_dim, qd, K, V, m, head_dim,
+                        (double)scale, s);
+        }
+        free(K);
+        free(V);
+        free(s);
+        free(qd);
+    }
+    (void)nthreads;
+    return status;
+}
+
 int oracle_max_threads(void)
 {
     return set_threads(0);

@@ -253,6 +253,110 @@ def _dense_scores(batch):
     return res
 
 
+# --------------------------------------------------------------------------- sliding window
+WINDOWS = (1, 2, 3, 4, 15, 16, 17, 33, 1000)
+
+
+def _window_lo(n, window):
+    return n - window if 0 < window < n else 0
+
+
+def dense_window_reference(batch, window):
+    """Unpaged attention over the logical rows [n - window, n) of each sequence,
+    numpy fp64 (the window's definition applied to the dense arrays)."""
+    G = batch.num_q_heads // batch.num_kv_heads
+    out = np.zeros((batch.num_seqs, batch.num_q_heads, batch.head_dim))
+    q = lib_f64(batch.q, batch.dtype)
+    for b in range(batch.num_seqs):
+        n = int(batch.context_lens[b])
+        if n == 0:
+            continue
+        rows = np.arange(batch.rows(b).start, batch.rows(b).stop)[_window_lo(n, window):n]
+        K = lib_f64(batch.k[rows], batch.dtype)
+        V = lib_f64(batch.v[rows], batch.dtype)
+        for h in range(batch.num_q_heads):
+            s = (K[:, h // G, :] @ q[b, h]) * float(batch.scale)
+            w = np.exp(s - s.max())
+            out[b, h] = (w @ V[:, h // G, :]) / w.sum()
+    return out
+
+
+def forget_before_window(batch, kp, vp, window):
+    """What a moved window leaves behind: pool rows before each sequence's window
+    poisoned, and the table entries of blocks wholly before it set to -1."""
+    bs = batch.block_size
+    tables = np.array(batch.block_tables, dtype=np.int32, copy=True)
+    kp, vp = kp.copy(), vp.copy()
+    for b in range(batch.num_seqs):
+        lo = _window_lo(int(batch.context_lens[b]), window)
+        for t in range(lo):
+            kp[tables[b, t // bs], :, t % bs, :] = NAN_BITS[batch.dtype]
+            vp[tables[b, t // bs], :, t % bs, :] = NAN_BITS[batch.dtype]
+        tables[b, :lo // bs] = -1
+    return kp, vp, tables
+
+
+def pin_window_dense():
+    for batch in small_batches():
+        kp, vp = place_numpy(batch)
+        for w in WINDOWS:
+            got = oracle.decode_window(batch.q, kp, vp, batch.block_tables, batch.context_lens,
+                                       batch.scale, batch.dtype, w)
+            ref = dense_window_reference(batch, w)
+            err = np.max(np.abs(got - ref)) if got.size else 0.0
+            assert err <= 1e-12, f"{batch.name} window {w}: off by {err}"
+
+
+def pin_window_one_returns_last_v():
+    batch = synth.small_random(26, 4, [1, 9, 16, 40], 8, 2, 16, 8, 24, "f16")
+    kp, vp = place_numpy(batch)
+    got = oracle.decode_window(batch.q, kp, vp, batch.block_tables, batch.context_lens,
+                               batch.scale, batch.dtype, 1)
+    G = batch.num_q_heads // batch.num_kv_heads
+    for b in range(batch.num_seqs):
+        v = lib_f64(batch.v[batch.rows(b).stop - 1], batch.dtype)
+        for h in range(batch.num_q_heads):
+            assert np.array_equal(got[b, h], v[h // G]), "window 1 must return the last V"
+
+
+def pin_window_ignores_what_it_left():
+    batch = synth.small_random(27, 5, [2, 16, 31, 47, 64], 4, 2, 16, 4, 90, "bf16")
+    kp, vp = place_numpy(batch)
+    for w in (3, 8, 17):
+        base = oracle.decode_window(batch.q, kp, vp, batch.block_tables, batch.context_lens,
+                                    batch.scale, batch.dtype, w)
+        kf, vf, tf = forget_before_window(batch, kp, vp, w)
+        got = oracle.decode_window(batch.q, kf, vf, tf, batch.context_lens, batch.scale,
+                                   batch.dtype, w)
+        assert np.all(np.isfinite(got)), "rows before the window reached the output"
+        assert np.array_equal(got, base), "rows or ids before the window changed the output"
+
+
+def pin_window_bruteforce_fsum():
+    batch = synth.small_random(28, 3, [5, 9, 14], 4, 2, 8, 4, 12, "f16")
+    kp, vp = place_numpy(batch)
+    window = 6
+    got = oracle.decode_window(batch.q, kp, vp, batch.block_tables, batch.context_lens,
+                               batch.scale, batch.dtype, window)
+    G = batch.num_q_heads // batch.num_kv_heads
+    q = lib_f64(batch.q, batch.dtype).tolist()
+    for b in range(batch.num_seqs):
+        rows = np.arange(batch.rows(b).start, batch.rows(b).stop)[-window:]
+        K = lib_f64(batch.k[rows], batch.dtype).tolist()
+        V = lib_f64(batch.v[rows], batch.dtype).tolist()
+        for h in range(batch.num_q_heads):
+            g = h // G
+            s = [float(batch.scale) * math.fsum(q[b][h][d] * K[t][g][d]
+                                                for d in range(batch.head_dim))
+                 for t in range(len(K))]
+            m = max(s)
+            wts = [math.exp(x - m) for x in s]
+            den = math.fsum(wts)
+            for d in range(batch.head_dim):
+                ref = math.fsum(wts[t] * V[t][g][d] for t in range(len(K))) / den
+                assert abs(got[b, h, d] - ref) <= 1e-13, "window brute force disagrees"
+
+
 # --------------------------------------------------------------------------- write / copy
 def pin_reshape_layout():
     """Write the worked example's 10 tokens (block size 4, blocks 8, 3, 15) at the
@@ -296,6 +400,32 @@ def pin_copy_blocks():
         exp_k[d] = k0[s]
         exp_v[d] = v0[s]
     assert np.array_equal(kc, exp_k) and np.array_equal(vc, exp_v), "copy_blocks"
+
+
+def pin_swap_blocks():
+    """Swap out then in: the host pool gets exactly the named device blocks
+    (numpy indexing as the reference), untouched host blocks keep their bits,
+    and bringing the blocks back into other device blocks restores every row."""
+    rng = np.random.default_rng(2)
+    dev_shape, host_shape = (10, 2, 4, 8), (6, 2, 4, 8)
+    dk = rng.integers(0, 1 << 16, size=dev_shape, dtype=np.uint64).astype(np.uint16)
+    dv = rng.integers(0, 1 << 16, size=dev_shape, dtype=np.uint64).astype(np.uint16)
+    hk = rng.integers(0, 1 << 16, size=host_shape, dtype=np.uint64).astype(np.uint16)
+    hv = rng.integers(0, 1 << 16, size=host_shape, dtype=np.uint64).astype(np.uint16)
+    hk0, hv0 = hk.copy(), hv.copy()
+    out_pairs = np.array([[7, 0], [2, 5], [9, 3]], dtype=np.int64)
+    oracle.swap_blocks(hk, hv, dk, dv, out_pairs)
+    exp_k, exp_v = hk0.copy(), hv0.copy()
+    exp_k[out_pairs[:, 1]] = dk[out_pairs[:, 0]]
+    exp_v[out_pairs[:, 1]] = dv[out_pairs[:, 0]]
+    assert np.array_equal(hk, exp_k) and np.array_equal(hv, exp_v), "swap out"
+    in_pairs = np.array([[0, 1], [5, 4], [3, 8]], dtype=np.int64)  # host -> other device blocks
+    dk2, dv2 = dk.copy(), dv.copy()
+    oracle.swap_blocks(dk2, dv2, hk, hv, in_pairs)
+    for (d_src, _), (_, d_dst) in zip(out_pairs, in_pairs):
+        assert np.array_equal(dk2[d_dst], dk[d_src]) and np.array_equal(dv2[d_dst], dv[d_src])
+    untouched = [b for b in range(dev_shape[0]) if b not in in_pairs[:, 1]]
+    assert np.array_equal(dk2[untouched], dk[untouched]), "swap in wrote outside its pairs"
 
 
 # --------------------------------------------------------------------------- block manager
@@ -369,9 +499,62 @@ def pin_allocator_cow():
     assert m.num_free() == 16 and all(r == 0 for r in m.ref)
 
 
+def pin_allocator_sliding_window():
+    """Sliding-window release worked by hand (second page, section 5.2: blocks
+    leave as the window moves; growth is block by block): block size 16,
+    window 32. A 40-token prompt takes 3 blocks; nothing precedes position
+    40 - 32 = 8 by a whole block. After 24 more tokens (length 64, 4 blocks) the
+    window starts at 32, so blocks 0 and 1 (positions 0-31) go back; the free
+    count returns to 8 - 4 + 2 = 6 and the table reads [-1, -1, c, d]."""
+    m = BlockManagerModel(8, 16)
+    t = m.add_seq(0, 40)
+    assert len(t) == 3 and m.num_free() == 5
+    assert m.slide_window(0, 32) == 0 and m.block_table(0) == t
+    for _ in range(24):
+        m.append_slot(0)
+    t4 = m.block_table(0)
+    assert len(t4) == 4 and m.num_free() == 4
+    assert m.slide_window(0, 32) == 2
+    assert m.block_table(0) == [-1, -1, t4[2], t4[3]] and m.num_free() == 6
+    # the released blocks are the next ones handed out (free list is a stack)
+    assert sorted(m.free[-2:]) == sorted(t4[:2])
+    m.free_seq(0)
+    assert m.num_free() == 8
+
+
+def pin_allocator_swap():
+    """Swapping worked by hand (third page, section "分页还顺带解决了什么": a
+    request's blocks go to CPU memory and come back; second page, section 3.1).
+    Block size 4, 8 device blocks, 4 host blocks. A 6-token prompt (2 blocks)
+    forked once is one group sharing 2 blocks: swapping it out moves 2 blocks
+    (not 4), each host block then counted twice, and all 8 device blocks are
+    free; swapping back takes 2 device blocks, counted twice each, and frees
+    the host space again."""
+    m = BlockManagerModel(8, 4)
+    m.set_host_blocks(4)
+    t = m.add_seq(0, 6)
+    m.fork(0, 1)
+    out = m.swap_out([0, 1])
+    assert len(out) == 2 and sorted(d for d, _ in out) == sorted(t)
+    assert m.num_free() == 8 and len(m.host_free) == 2
+    assert [m.host_ref[h] for _, h in out] == [2, 2]
+    assert m.block_table(0) == m.block_table(1) == [h for _, h in out]
+    back = m.swap_in([0, 1])
+    assert [h for h, _ in back] == [h for _, h in out]
+    assert m.num_free() == 6 and len(m.host_free) == 4
+    assert [m.ref[d] for _, d in back] == [2, 2]
+    assert m.block_table(0) == [d for _, d in back]
+    m.free_seq(0)
+    m.free_seq(1)
+    assert m.num_free() == 8
+
+
 ALL_ORACLE_PINS = [
     pin_f16_decoder, pin_bf16_decoder, pin_worked_example_slots, pin_bs16_tables, pin_dense,
     pin_len1_returns_v, pin_identical_keys_mean_v, pin_bruteforce_fsum, pin_relabel, pin_poison,
-    pin_partition_merge, pin_reshape_layout, pin_copy_blocks,
+    pin_partition_merge, pin_reshape_layout, pin_copy_blocks, pin_window_dense,
+    pin_window_one_returns_last_v, pin_window_ignores_what_it_left, pin_window_bruteforce_fsum,
+    pin_swap_blocks,
 ]
-ALL_MODEL_PINS = [pin_allocator_worked_example, pin_allocator_capacity, pin_allocator_cow]
+ALL_MODEL_PINS = [pin_allocator_worked_example, pin_allocator_capacity, pin_allocator_cow,
+                  pin_allocator_sliding_window, pin_allocator_swap]

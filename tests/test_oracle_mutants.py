@@ -31,6 +31,14 @@ MUTANTS = {
     "f16_bias": ("mag = ldexp((double)(1024 + f), e - 25);", "mag = ldexp((double)(1024 + f), e - 24);"),
     "bf16_bias": ("mag = ldexp((double)(128 + f), e - 134);", "mag = ldexp((double)(128 + f), e - 133);"),
     "write_skips_slot0": ("if (slot < 0)\n            continue;", "if (slot <= 0)\n            continue;"),
+    "window_one_short": ("int lo = (window > 0 && n > window) ? n - window : 0;",
+                         "int lo = (window > 0 && n > window) ? n - window + 1 : 0;"),
+    "window_ignored": ("int lo = (window > 0 && n > window) ? n - window : 0;",
+                       "int lo = 0;"),
+    "window_rows_shifted": ("dst[(size_t)(t - lo) * head_dim + d] =\n                widen(pool[pool_index(block, kv_head, offset, d,",
+                            "dst[(size_t)(t - lo) * head_dim + d] =\n                widen(pool[pool_index(block, kv_head, offset > 0 ? offset - 1 : 0, d,"),
+    "swap_v_from_k": ("dst_v[(size_t)dst * block_elems + i] = src_v[(size_t)src * block_elems + i];",
+                      "dst_v[(size_t)dst * block_elems + i] = src_k[(size_t)src * block_elems + i];"),
     "copy_k_only": ("v_cache[(size_t)dst * block_elems + i] = v_cache[(size_t)src * block_elems + i];",
                     ";"),
 }
