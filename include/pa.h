@@ -97,6 +97,42 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_pair
                          pa_dtype dtype, void *stream);
 
 /* ------------------------------------------------------------------------------------------
+ * Host swap space -- blocks moved out of the device pool and back.
+ * [P3, section "分页还顺带解决了什么": under memory pressure a request's blocks
+ * may be moved to CPU memory and brought back later, which same-size blocks
+ * make easy. P2, section 3.1: swap_out of a preempted victim; section 6.1: a
+ * CPU swap space of configurable size.]
+ *
+ * pa_swap_space_create allocates pinned host memory for num_host_blocks
+ * blocks of K and of V, laid out like the device pools ([num_host_blocks]
+ * [num_kv_heads][block_size][head_dim], the given dtype), and maps it into
+ * the current device's address space. This is the library's only
+ * allocation, made once, off the hot path; pa_swap_space_destroy frees it.
+ * pa_swap_space_pools returns the host addresses of the two pools (for
+ * inspection or checkpointing). PA_ERR_CUDA if the pinned allocation fails.
+ *
+ * pa_swap_out copies, for each pair (device block, host block) of
+ * block_pairs, the whole device block (every KV head and slot, K and V) into
+ * the host block; pa_swap_in copies pairs (host block, device block) back.
+ * One launch moves all pairs; stream-ordered like every device op, so a
+ * device block freed by pa_alloc_swap_out may be reused by later work on the
+ * same stream. block_pairs: device-accessible int64 [num_pairs][2]. An id
+ * outside its pool skips that pair and sets PA_DEVERR_COPY_PAIR. Destinations
+ * must be distinct (undefined otherwise). The device pools must have the
+ * swap space's block shape.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct pa_swap_space pa_swap_space;
+
+pa_status pa_swap_space_create(int num_host_blocks, int num_kv_heads, int block_size, int head_dim,
+                               pa_dtype dtype, pa_swap_space **out);
+void pa_swap_space_destroy(pa_swap_space *space);
+pa_status pa_swap_space_pools(const pa_swap_space *space, void **k_host, void **v_host);
+pa_status pa_swap_out(const pa_swap_space *space, const void *k_cache, const void *v_cache,
+                      int num_blocks, const int64_t *block_pairs, int num_pairs, void *stream);
+pa_status pa_swap_in(const pa_swap_space *space, void *k_cache, void *v_cache, int num_blocks,
+                     const int64_t *block_pairs, int num_pairs, void *stream);
+
+/* ------------------------------------------------------------------------------------------
  * pa_decode -- paged attention for one query token per sequence.
  * [P1, section 5: out = softmax(Q K^T / sqrt(d)) V, where the kernel finds
  * each token's logical block and maps it through the block table to the
@@ -246,7 +282,7 @@ pa_status pa_slot_mapping(const int32_t *block_tables, int max_blocks_per_seq,
  * immediate reuse. P3, section "借用操作系统的办法：分页": same; section
  * "分页还顺带解决了什么": blocks shared by several tables carry a reference
  * count. P2, section 2.3: copy-on-write. P2, section 5.1: forking sampled
- * sequences from a shared prompt.]
+ * sequences from a shared prompt. P2, section 5.2: sliding-window release.]
  * Which free block is handed out is not part of the contract.
  * ========================================================================================== */
 typedef struct pa_alloc pa_alloc;
@@ -277,6 +313,42 @@ pa_status pa_alloc_seq_slots(const pa_alloc *a, int64_t seq_id, int start, int c
 /* Drop the sequence: each block loses a reference; blocks reaching zero go
  * back on the free list. */
 pa_status pa_alloc_free_seq(pa_alloc *a, int64_t seq_id);
+
+/* Sliding-window release [P2, section 5.2: blocks that fall out of the window
+ * are reclaimed automatically]. Every block wholly before the window
+ * [len - window, len) of the sequence's current length loses this sequence's
+ * reference (blocks reaching zero go back on the free list) and its table
+ * entry becomes -1. Decode with the same or a smaller window never reads those
+ * entries (pa_decode_window). *freed (may be NULL) = blocks returned to the
+ * free list. window <= 0: PA_ERR_INVALID. Entries already released are skipped,
+ * so the call may be repeated every step. Slots of released positions are no
+ * longer available (pa_alloc_seq_slots answers PA_ERR_STATE). */
+pa_status pa_alloc_slide_window(pa_alloc *a, int64_t seq_id, int window, int *freed);
+
+/* Swapping a group of sequences (the blocks of a preempted request and of the
+ * samples forked from it) [P3, section "分页还顺带解决了什么"; P2, section 3.1].
+ * pa_alloc_set_host_blocks gives the manager a host swap space of
+ * num_host_blocks blocks (once; PA_ERR_STATE if already given).
+ * pa_alloc_swap_out moves the n sequences seq_ids (all resident) to the host:
+ * each distinct block they use gets one free host block, whose count is the
+ * group's references; the device block loses those references (returning to
+ * the free list at zero) and the tables then name host blocks. pairs[0 ..
+ * *num_pairs) receives (device block, host block) -- the copies pa_swap_out
+ * must make. pa_alloc_swap_in is the mirror image for a swapped group:
+ * pairs are (host block, device block) for pa_swap_in. A block also used by
+ * a sequence outside the group stays in place for it, and the group gets its
+ * own copy. All or nothing: PA_ERR_OUT_OF_BLOCKS if the other side lacks free
+ * blocks, PA_ERR_STATE if a sequence is unknown or already on the other side,
+ * PA_ERR_INVALID if one is listed twice or cap is short. While swapped a
+ * sequence can only be swapped in, freed or queried (pa_alloc_block_table
+ * then lists host blocks); other calls answer PA_ERR_STATE. */
+pa_status pa_alloc_set_host_blocks(pa_alloc *a, int num_host_blocks);
+pa_status pa_alloc_swap_out(pa_alloc *a, const int64_t *seq_ids, int n, int64_t *pairs, int cap,
+                            int *num_pairs);
+pa_status pa_alloc_swap_in(pa_alloc *a, const int64_t *seq_ids, int n, int64_t *pairs, int cap,
+                           int *num_pairs);
+pa_status pa_alloc_is_swapped(const pa_alloc *a, int64_t seq_id, int *swapped);
+pa_status pa_alloc_host_free(const pa_alloc *a, int *free_host_blocks);
 
 /* Copy the sequence's block table into out[0 .. cap); report its block and
  * token counts (either pointer may be NULL). PA_ERR_INVALID if cap is short. */

@@ -13,6 +13,7 @@ _EXPORTS = (
     "pa_decode_append_launches",
     "pa_decode_default_partition", "pa_decode_launches", "pa_decode_static_workspace",
     "pa_decode_workspace_size", "pa_device_status", "pa_reshape_and_cache", "pa_slot_mapping",
+    "SwapSpace", "pa_swap_out", "pa_swap_in",
 )
 
 __all__ = list(_EXPORTS)

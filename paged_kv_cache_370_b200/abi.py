@@ -72,6 +72,17 @@ def _load() -> ctypes.CDLL:
         "pa_alloc_append_slot": (i, [P, i64, P, P, P]),
         "pa_alloc_seq_slots": (i, [P, i64, i, i, P]),
         "pa_alloc_free_seq": (i, [P, i64]),
+        "pa_alloc_slide_window": (i, [P, i64, i, P]),
+        "pa_alloc_set_host_blocks": (i, [P, i]),
+        "pa_swap_space_create": (i, [i, i, i, i, i, P]),
+        "pa_swap_space_destroy": (None, [P]),
+        "pa_swap_space_pools": (i, [P, P, P]),
+        "pa_swap_out": (i, [P, P, P, i, P, i, P]),
+        "pa_swap_in": (i, [P, P, P, i, P, i, P]),
+        "pa_alloc_swap_out": (i, [P, P, i, P, i, P]),
+        "pa_alloc_swap_in": (i, [P, P, i, P, i, P]),
+        "pa_alloc_is_swapped": (i, [P, i64, P]),
+        "pa_alloc_host_free": (i, [P, P]),
         "pa_alloc_block_table": (i, [P, i64, P, i, P, P]),
         "pa_alloc_fill_tables": (i, [P, P, i, P, i, ctypes.c_int32, P]),
         "pa_alloc_ref_count": (i, [P, ctypes.c_int32, P]),
@@ -154,6 +165,56 @@ def pa_copy_blocks(k_cache, v_cache, block_pairs, stream=None):
                              _dev_ptr(block_pairs, "block_pairs"), n, nb, hkv, bs, d,
                              _dtype_code(k_cache), _stream(stream))
     _check(st, "pa_copy_blocks")
+
+
+class SwapSpace:
+    """Pinned, device-mapped host memory for ``num_host_blocks`` KV blocks
+    (pa_swap_space_*). ``k_host`` / ``v_host`` are numpy views of the two host
+    pools, [num_host_blocks, num_kv_heads, block_size, head_dim] of 16-bit words."""
+
+    def __init__(self, num_host_blocks: int, num_kv_heads: int, block_size: int, head_dim: int,
+                 dtype: str):
+        code = {"f16": PA_F16, "bf16": PA_BF16}[dtype]
+        h = ctypes.c_void_p()
+        _check(_lib.pa_swap_space_create(num_host_blocks, num_kv_heads, block_size, head_dim, code,
+                                         ctypes.byref(h)), "pa_swap_space_create")
+        self._h = h
+        self.shape = (num_host_blocks, num_kv_heads, block_size, head_dim)
+        kp, vp = ctypes.c_void_p(), ctypes.c_void_p()
+        _check(_lib.pa_swap_space_pools(h, ctypes.byref(kp), ctypes.byref(vp)), "pa_swap_space_pools")
+        n = int(np.prod(self.shape))
+        self.k_host = np.ctypeslib.as_array((ctypes.c_uint16 * n).from_address(kp.value)).reshape(self.shape)
+        self.v_host = np.ctypeslib.as_array((ctypes.c_uint16 * n).from_address(vp.value)).reshape(self.shape)
+
+    def close(self):
+        if self._h:
+            self.k_host = self.v_host = None
+            _lib.pa_swap_space_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:  # noqa: BLE001 -- interpreter shutdown
+            pass
+
+
+def pa_swap_out(space: SwapSpace, k_cache, v_cache, block_pairs, stream=None):
+    """Copy device blocks to host blocks for every (device, host) row of block_pairs."""
+    n = int(block_pairs.shape[0]) if block_pairs.numel() else 0
+    st = _lib.pa_swap_out(space._h, _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+                          int(k_cache.shape[0]), _dev_ptr(block_pairs, "block_pairs"), n,
+                          _stream(stream))
+    _check(st, "pa_swap_out")
+
+
+def pa_swap_in(space: SwapSpace, k_cache, v_cache, block_pairs, stream=None):
+    """Copy host blocks to device blocks for every (host, device) row of block_pairs."""
+    n = int(block_pairs.shape[0]) if block_pairs.numel() else 0
+    st = _lib.pa_swap_in(space._h, _dev_ptr(k_cache, "k_cache"), _dev_ptr(v_cache, "v_cache"),
+                         int(k_cache.shape[0]), _dev_ptr(block_pairs, "block_pairs"), n,
+                         _stream(stream))
+    _check(st, "pa_swap_in")
 
 
 def pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
@@ -293,6 +354,48 @@ class BlockManager:
 
     def free_seq(self, seq_id: int):
         _check(_lib.pa_alloc_free_seq(self._h, seq_id), "pa_alloc_free_seq")
+
+    def slide_window(self, seq_id: int, window: int) -> int:
+        """Release the blocks wholly before the last ``window`` positions; returns
+        how many went back on the free list."""
+        freed = ctypes.c_int(0)
+        _check(_lib.pa_alloc_slide_window(self._h, seq_id, window, ctypes.byref(freed)),
+               "pa_alloc_slide_window")
+        return freed.value
+
+    def set_host_blocks(self, num_host_blocks: int):
+        """Give the manager a host swap space of ``num_host_blocks`` blocks."""
+        _check(_lib.pa_alloc_set_host_blocks(self._h, num_host_blocks), "pa_alloc_set_host_blocks")
+
+    def _swap(self, fn, name, seq_ids):
+        ids = np.ascontiguousarray(np.asarray(list(seq_ids), dtype=np.int64))
+        cap = 0
+        for s in ids.tolist():
+            cap += len(self.block_table(int(s)))
+        pairs = np.zeros((max(cap, 1), 2), dtype=np.int64)
+        n = ctypes.c_int(0)
+        _check(fn(self._h, _np_ptr(ids), len(ids), _np_ptr(pairs), cap, ctypes.byref(n)), name)
+        return pairs[: n.value].copy()
+
+    def swap_out(self, seq_ids) -> np.ndarray:
+        """Move a group of sequences to the host swap space; returns the
+        (device block, host block) pairs to copy (pa_swap_out)."""
+        return self._swap(_lib.pa_alloc_swap_out, "pa_alloc_swap_out", seq_ids)
+
+    def swap_in(self, seq_ids) -> np.ndarray:
+        """Bring a swapped group back; returns (host block, device block) pairs
+        to copy (pa_swap_in)."""
+        return self._swap(_lib.pa_alloc_swap_in, "pa_alloc_swap_in", seq_ids)
+
+    def is_swapped(self, seq_id: int) -> bool:
+        v = ctypes.c_int(0)
+        _check(_lib.pa_alloc_is_swapped(self._h, seq_id, ctypes.byref(v)), "pa_alloc_is_swapped")
+        return bool(v.value)
+
+    def host_free(self) -> int:
+        v = ctypes.c_int(0)
+        _check(_lib.pa_alloc_host_free(self._h, ctypes.byref(v)), "pa_alloc_host_free")
+        return v.value
 
     def block_table(self, seq_id: int) -> list[int]:
         nb, nt = ctypes.c_int(), ctypes.c_int()

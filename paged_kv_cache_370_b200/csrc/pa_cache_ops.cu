@@ -7,6 +7,13 @@
 //  * pa_copy_blocks: whole-block copies for copy-on-write (page
 //    "PagedAttention 核心思想解析", section 2.3: allocate a new block, copy
 //    the original block's contents, update the table).
+//  * pa_swap_out / pa_swap_in: whole-block copies between the device pools and
+//    a host swap space (page "08. PagedAttention：把 KV Cache 分页管理",
+//    section "分页还顺带解决了什么": a preempted request's blocks go to CPU
+//    memory and come back later; same-size blocks make this easy). The swap
+//    space is pinned host memory mapped into the device's address space, so
+//    one kernel moves every block of a swap over PCIe / C2C, instead of one
+//    copy call per block.
 //
 // Both move 16-byte vectors (every row is head_dim * 2 bytes, a multiple of
 // 16), index in 64 bits, and check the ids they are given: a slot or block
@@ -16,6 +23,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <new>
 
 #include "pa.h"
 #include "pa_internal.h"
@@ -83,6 +91,38 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
   }
 }
 
+constexpr int kSwapUnroll = 8;  // 16-byte loads in flight per thread (host memory is far)
+
+// grid = (chunks of a block / (threads * unroll), pairs, 2: K then V). Pair i
+// copies source block pairs[i][0] to destination block pairs[i][1].
+__global__ void __launch_bounds__(kCopyThreads) swap_blocks_kernel(
+    uint4 *__restrict__ dst_k, uint4 *__restrict__ dst_v, int64_t dst_blocks,
+    const uint4 *__restrict__ src_k, const uint4 *__restrict__ src_v, int64_t src_blocks,
+    const int64_t *__restrict__ block_pairs, int64_t chunks_per_block) {
+  const int pair = blockIdx.y;
+  const int64_t src = block_pairs[2 * pair];
+  const int64_t dst = block_pairs[2 * pair + 1];
+  if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.z == 0)
+      atomicOr(&g_cache_ops_error, PA_DEVERR_COPY_PAIR);
+    return;
+  }
+  const uint4 *s = (blockIdx.z == 0 ? src_k : src_v) + src * chunks_per_block;
+  uint4 *d = (blockIdx.z == 0 ? dst_k : dst_v) + dst * chunks_per_block;
+  const int64_t base = (int64_t)blockIdx.x * kCopyThreads * kSwapUnroll + threadIdx.x;
+  uint4 buf[kSwapUnroll];
+#pragma unroll
+  for (int u = 0; u < kSwapUnroll; ++u) {
+    const int64_t j = base + (int64_t)u * kCopyThreads;
+    if (j < chunks_per_block) buf[u] = s[j];
+  }
+#pragma unroll
+  for (int u = 0; u < kSwapUnroll; ++u) {
+    const int64_t j = base + (int64_t)u * kCopyThreads;
+    if (j < chunks_per_block) d[j] = buf[u];
+  }
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool valid_pool_args(int num_blocks, int num_kv_heads, int block_size, int head_dim,
@@ -134,6 +174,113 @@ extern "C" pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t 
       num_blocks);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
+
+struct pa_swap_space {
+  void *k_host = nullptr;  // pinned, mapped: [num_blocks][num_kv_heads][block_size][head_dim]
+  void *v_host = nullptr;
+  uint4 *k_dev = nullptr;  // the same memory as the device sees it
+  uint4 *v_dev = nullptr;
+  int num_blocks = 0, num_kv_heads = 0, block_size = 0, head_dim = 0;
+  pa_dtype dtype = PA_F16;
+};
+
+extern "C" {
+
+pa_status pa_swap_space_create(int num_host_blocks, int num_kv_heads, int block_size, int head_dim,
+                               pa_dtype dtype, pa_swap_space **out) {
+  if (!out || !valid_pool_args(num_host_blocks, num_kv_heads, block_size, head_dim, dtype))
+    return PA_ERR_INVALID;
+  const size_t bytes = (size_t)num_host_blocks * num_kv_heads * block_size * head_dim * 2;
+  pa_swap_space *sp = new (std::nothrow) pa_swap_space();
+  if (!sp) return PA_ERR_INVALID;
+  const unsigned flags = cudaHostAllocMapped | cudaHostAllocPortable;
+  void *dk = nullptr, *dv = nullptr;
+  if (cudaHostAlloc(&sp->k_host, bytes, flags) != cudaSuccess ||
+      cudaHostAlloc(&sp->v_host, bytes, flags) != cudaSuccess ||
+      cudaHostGetDevicePointer(&dk, sp->k_host, 0) != cudaSuccess ||
+      cudaHostGetDevicePointer(&dv, sp->v_host, 0) != cudaSuccess) {
+    if (sp->k_host) cudaFreeHost(sp->k_host);
+    if (sp->v_host) cudaFreeHost(sp->v_host);
+    delete sp;
+    return PA_ERR_CUDA;
+  }
+  sp->k_dev = static_cast<uint4 *>(dk);
+  sp->v_dev = static_cast<uint4 *>(dv);
+  sp->num_blocks = num_host_blocks;
+  sp->num_kv_heads = num_kv_heads;
+  sp->block_size = block_size;
+  sp->head_dim = head_dim;
+  sp->dtype = dtype;
+  *out = sp;
+  return PA_OK;
+}
+
+void pa_swap_space_destroy(pa_swap_space *sp) {
+  if (!sp) return;
+  cudaFreeHost(sp->k_host);
+  cudaFreeHost(sp->v_host);
+  delete sp;
+}
+
+pa_status pa_swap_space_pools(const pa_swap_space *sp, void **k_host, void **v_host) {
+  if (!sp || !k_host || !v_host) return PA_ERR_INVALID;
+  *k_host = sp->k_host;
+  *v_host = sp->v_host;
+  return PA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+pa_status launch_swap(uint4 *dst_k, uint4 *dst_v, int64_t dst_blocks, const uint4 *src_k,
+                      const uint4 *src_v, int64_t src_blocks, const int64_t *block_pairs,
+                      int num_pairs, int64_t chunks, cudaStream_t stream) {
+  const int64_t per_cta = (int64_t)kCopyThreads * kSwapUnroll;
+  for (int first = 0; first < num_pairs; first += 65535) {
+    const int n = num_pairs - first < 65535 ? num_pairs - first : 65535;
+    dim3 grid((unsigned)((chunks + per_cta - 1) / per_cta), (unsigned)n, 2);
+    swap_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(dst_k, dst_v, dst_blocks, src_k, src_v,
+                                                          src_blocks, block_pairs + 2 * (size_t)first,
+                                                          chunks);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+  }
+  return PA_OK;
+}
+
+bool swap_args_ok(const pa_swap_space *sp, const void *k_cache, const void *v_cache,
+                  int num_blocks, const int64_t *block_pairs, int num_pairs) {
+  return sp && num_pairs >= 0 && num_blocks > 0 &&
+         (num_pairs == 0 || (k_cache && v_cache && block_pairs && aligned16(k_cache) &&
+                             aligned16(v_cache) &&
+                             (reinterpret_cast<uintptr_t>(block_pairs) & 7u) == 0));
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_swap_out(const pa_swap_space *sp, const void *k_cache, const void *v_cache,
+                      int num_blocks, const int64_t *block_pairs, int num_pairs, void *stream) {
+  if (!swap_args_ok(sp, k_cache, v_cache, num_blocks, block_pairs, num_pairs)) return PA_ERR_INVALID;
+  if (num_pairs == 0) return PA_OK;
+  const int64_t chunks = (int64_t)sp->num_kv_heads * sp->block_size * sp->head_dim * 2 / 16;
+  return launch_swap(sp->k_dev, sp->v_dev, sp->num_blocks, static_cast<const uint4 *>(k_cache),
+                     static_cast<const uint4 *>(v_cache), num_blocks, block_pairs, num_pairs, chunks,
+                     (cudaStream_t)stream);
+}
+
+pa_status pa_swap_in(const pa_swap_space *sp, void *k_cache, void *v_cache, int num_blocks,
+                     const int64_t *block_pairs, int num_pairs, void *stream) {
+  if (!swap_args_ok(sp, k_cache, v_cache, num_blocks, block_pairs, num_pairs)) return PA_ERR_INVALID;
+  if (num_pairs == 0) return PA_OK;
+  const int64_t chunks = (int64_t)sp->num_kv_heads * sp->block_size * sp->head_dim * 2 / 16;
+  return launch_swap(static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), num_blocks,
+                     sp->k_dev, sp->v_dev, sp->num_blocks, block_pairs, num_pairs, chunks,
+                     (cudaStream_t)stream);
+}
+
+}  // extern "C"
 
 // Read and clear this file's error word (stream-ordered; synchronises the stream).
 pa_status pa_internal_cache_ops_status(cudaStream_t stream, int32_t *code) {

@@ -8,7 +8,8 @@
 // "借用操作系统的办法：分页"), block tables shared between sequences with a
 // reference count per block (same page, section "分页还顺带解决了什么"), and
 // copy-on-write when a sequence writes into a shared block ("PagedAttention
-// 核心思想解析", section 2.3). Slots are block_table[logical block] *
+// 核心思想解析", section 2.3), and the release of blocks a sliding window has
+// moved past (same page, section 5.2). Slots are block_table[logical block] *
 // block_size + offset (third page, section "为什么叫 PagedAttention").
 //
 // The free list is a LIFO stack of block ids: a freed block is the next one
@@ -23,9 +24,13 @@
 
 namespace {
 
+// Table entry of a block released because a sliding window moved past it.
+constexpr int32_t kReleased = -1;
+
 struct Sequence {
-  std::vector<int32_t> blocks;  // logical block i -> physical block
+  std::vector<int32_t> blocks;  // logical block i -> physical block (or kReleased)
   int64_t len = 0;              // tokens stored
+  bool swapped = false;         // blocks name host swap-space blocks
 };
 
 }  // namespace
@@ -36,6 +41,8 @@ struct pa_alloc {
   std::vector<int32_t> free_stack;  // back() is handed out next
   std::vector<int32_t> ref_count;   // per physical block
   std::unordered_map<int64_t, Sequence> seqs;
+  std::vector<int32_t> host_free;   // host swap-space blocks, back() handed out next
+  std::vector<int32_t> host_ref;    // per host block
 
   int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
 
@@ -80,9 +87,10 @@ pa_status pa_alloc_add_seq(pa_alloc *a, int64_t seq_id, int num_tokens) {
 pa_status pa_alloc_fork(pa_alloc *a, int64_t parent, int64_t child) {
   if (!a) return PA_ERR_INVALID;
   auto it = a->seqs.find(parent);
-  if (it == a->seqs.end() || a->seqs.count(child)) return PA_ERR_STATE;
+  if (it == a->seqs.end() || a->seqs.count(child) || it->second.swapped) return PA_ERR_STATE;
   Sequence c = it->second;
-  for (int32_t b : c.blocks) a->ref_count[b] += 1;
+  for (int32_t b : c.blocks)
+    if (b != kReleased) a->ref_count[b] += 1;
   a->seqs.emplace(child, std::move(c));
   return PA_OK;
 }
@@ -91,7 +99,7 @@ pa_status pa_alloc_append_slot(pa_alloc *a, int64_t seq_id, int64_t *slot, int64
                                int64_t *cow_dst) {
   if (!a || !slot) return PA_ERR_INVALID;
   auto it = a->seqs.find(seq_id);
-  if (it == a->seqs.end()) return PA_ERR_STATE;
+  if (it == a->seqs.end() || it->second.swapped) return PA_ERR_STATE;
   Sequence &s = it->second;
   const int64_t pos = s.len;
   const int64_t logical = pos / a->block_size;
@@ -124,9 +132,11 @@ pa_status pa_alloc_seq_slots(const pa_alloc *a, int64_t seq_id, int start, int c
                              int64_t *slots) {
   if (!a || start < 0 || count < 0 || (count && !slots)) return PA_ERR_INVALID;
   auto it = a->seqs.find(seq_id);
-  if (it == a->seqs.end()) return PA_ERR_STATE;
+  if (it == a->seqs.end() || it->second.swapped) return PA_ERR_STATE;
   const Sequence &s = it->second;
   if ((int64_t)start + count > s.len) return PA_ERR_INVALID;
+  for (int i = 0; i < count; ++i)
+    if (s.blocks[((int64_t)start + i) / a->block_size] == kReleased) return PA_ERR_STATE;
   for (int i = 0; i < count; ++i) {
     int64_t pos = (int64_t)start + i;
     slots[i] = (int64_t)s.blocks[pos / a->block_size] * a->block_size + pos % a->block_size;
@@ -139,12 +149,37 @@ pa_status pa_alloc_free_seq(pa_alloc *a, int64_t seq_id) {
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PA_ERR_STATE;
   const std::vector<int32_t> &blocks = it->second.blocks;
+  std::vector<int32_t> &ref = it->second.swapped ? a->host_ref : a->ref_count;
+  std::vector<int32_t> &free_list = it->second.swapped ? a->host_free : a->free_stack;
   for (int32_t b : blocks)
-    if (a->ref_count[b] <= 0) return PA_ERR_STATE;  // would underflow: refuse, change nothing
+    if (b != kReleased && ref[b] <= 0) return PA_ERR_STATE;  // would underflow: refuse, change nothing
   for (auto r = blocks.rbegin(); r != blocks.rend(); ++r) {
-    if (--a->ref_count[*r] == 0) a->free_stack.push_back(*r);
+    if (*r != kReleased && --ref[*r] == 0) free_list.push_back(*r);
   }
   a->seqs.erase(it);
+  return PA_OK;
+}
+
+pa_status pa_alloc_slide_window(pa_alloc *a, int64_t seq_id, int window, int *freed) {
+  if (!a || window <= 0) return PA_ERR_INVALID;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end() || it->second.swapped) return PA_ERR_STATE;
+  Sequence &s = it->second;
+  // blocks wholly before the window [len - window, len) of the current length
+  const int64_t lo = s.len > window ? s.len - window : 0;
+  const int64_t gone = lo / a->block_size;
+  int n = 0;
+  for (int64_t i = 0; i < gone; ++i) {
+    int32_t b = s.blocks[i];
+    if (b == kReleased) continue;
+    if (a->ref_count[b] <= 0) return PA_ERR_STATE;
+    s.blocks[i] = kReleased;
+    if (--a->ref_count[b] == 0) {
+      a->free_stack.push_back(b);
+      ++n;
+    }
+  }
+  if (freed) *freed = n;
   return PA_OK;
 }
 
@@ -170,7 +205,7 @@ pa_status pa_alloc_fill_tables(const pa_alloc *a, const int64_t *seq_ids, int n,
     return PA_ERR_INVALID;
   for (int i = 0; i < n; ++i) {
     auto it = a->seqs.find(seq_ids[i]);
-    if (it == a->seqs.end()) return PA_ERR_STATE;
+    if (it == a->seqs.end() || it->second.swapped) return PA_ERR_STATE;
     const Sequence &s = it->second;
     if ((int)s.blocks.size() > max_blocks_per_seq) return PA_ERR_INVALID;
     int32_t *row = block_tables + (size_t)i * max_blocks_per_seq;
@@ -194,7 +229,9 @@ pa_status pa_alloc_stats(const pa_alloc *a, int *free_blocks, int64_t *used_toke
   std::unordered_map<int32_t, int> fill;
   for (const auto &kv : a->seqs) {
     const Sequence &s = kv.second;
+    if (s.swapped) continue;  // its blocks are in the host swap space
     for (size_t i = 0; i < s.blocks.size(); ++i) {
+      if (s.blocks[i] == kReleased) continue;
       int64_t f = std::min<int64_t>(a->block_size, s.len - (int64_t)i * a->block_size);
       int &cur = fill[s.blocks[i]];
       cur = std::max<int>(cur, (int)std::max<int64_t>(f, 0));
@@ -206,6 +243,91 @@ pa_status pa_alloc_stats(const pa_alloc *a, int *free_blocks, int64_t *used_toke
   if (free_blocks) *free_blocks = (int)a->free_stack.size();
   if (used_tokens) *used_tokens = used;
   if (wasted_tokens) *wasted_tokens = used_blocks * a->block_size - used;
+  return PA_OK;
+}
+
+pa_status pa_alloc_set_host_blocks(pa_alloc *a, int num_host_blocks) {
+  if (!a || num_host_blocks <= 0) return PA_ERR_INVALID;
+  if (!a->host_ref.empty()) return PA_ERR_STATE;
+  a->host_ref.assign(num_host_blocks, 0);
+  a->host_free.resize(num_host_blocks);
+  for (int i = 0; i < num_host_blocks; ++i) a->host_free[i] = num_host_blocks - 1 - i;
+  return PA_OK;
+}
+
+// Move a group of sequences between the device pool and the host swap space.
+// Blocks the group shares move once; a block also held outside the group is
+// copied and stays on its side for the others. All or nothing.
+static pa_status swap_group(pa_alloc *a, const int64_t *seq_ids, int n, int64_t *pairs, int cap,
+                            int *num_pairs, bool out) {
+  if (!a || n < 0 || (n && !seq_ids) || !num_pairs || cap < 0 || (cap && !pairs))
+    return PA_ERR_INVALID;
+  if (a->host_ref.empty()) return PA_ERR_STATE;  // no swap space
+  std::vector<Sequence *> group;
+  for (int i = 0; i < n; ++i) {
+    auto it = a->seqs.find(seq_ids[i]);
+    if (it == a->seqs.end() || it->second.swapped == out) return PA_ERR_STATE;
+    for (Sequence *g : group)
+      if (g == &it->second) return PA_ERR_INVALID;  // listed twice
+    group.push_back(&it->second);
+  }
+  // distinct blocks in order of first use, with the group's references to each
+  std::vector<int32_t> order;
+  std::unordered_map<int32_t, int> refs;
+  for (Sequence *g : group)
+    for (int32_t b : g->blocks) {
+      if (b == kReleased) continue;
+      if (refs[b]++ == 0) order.push_back(b);
+    }
+  std::vector<int32_t> &src_ref = out ? a->ref_count : a->host_ref;
+  std::vector<int32_t> &src_free = out ? a->free_stack : a->host_free;
+  std::vector<int32_t> &dst_ref = out ? a->host_ref : a->ref_count;
+  std::vector<int32_t> &dst_free = out ? a->host_free : a->free_stack;
+  for (int32_t b : order)
+    if (src_ref[b] < refs[b]) return PA_ERR_STATE;
+  if (order.size() > dst_free.size()) return PA_ERR_OUT_OF_BLOCKS;
+  if ((int)order.size() > cap) return PA_ERR_INVALID;
+  std::unordered_map<int32_t, int32_t> moved;
+  for (size_t i = 0; i < order.size(); ++i) {
+    const int32_t b = order[i];
+    const int32_t d = dst_free.back();
+    dst_free.pop_back();
+    dst_ref[d] = refs[b];
+    if ((src_ref[b] -= refs[b]) == 0) src_free.push_back(b);
+    moved[b] = d;
+    pairs[2 * i] = b;
+    pairs[2 * i + 1] = d;
+  }
+  for (Sequence *g : group) {
+    for (int32_t &b : g->blocks)
+      if (b != kReleased) b = moved[b];
+    g->swapped = out;
+  }
+  *num_pairs = (int)order.size();
+  return PA_OK;
+}
+
+pa_status pa_alloc_swap_out(pa_alloc *a, const int64_t *seq_ids, int n, int64_t *pairs, int cap,
+                            int *num_pairs) {
+  return swap_group(a, seq_ids, n, pairs, cap, num_pairs, true);
+}
+
+pa_status pa_alloc_swap_in(pa_alloc *a, const int64_t *seq_ids, int n, int64_t *pairs, int cap,
+                           int *num_pairs) {
+  return swap_group(a, seq_ids, n, pairs, cap, num_pairs, false);
+}
+
+pa_status pa_alloc_is_swapped(const pa_alloc *a, int64_t seq_id, int *swapped) {
+  if (!a || !swapped) return PA_ERR_INVALID;
+  auto it = a->seqs.find(seq_id);
+  if (it == a->seqs.end()) return PA_ERR_STATE;
+  *swapped = it->second.swapped ? 1 : 0;
+  return PA_OK;
+}
+
+pa_status pa_alloc_host_free(const pa_alloc *a, int *free_host_blocks) {
+  if (!a || !free_host_blocks) return PA_ERR_INVALID;
+  *free_host_blocks = (int)a->host_free.size();
   return PA_OK;
 }
 

@@ -151,30 +151,41 @@ def test_state_errors():
         m.append_slot(0)
 
 
-def _relabel_consistent(model, prod, seqs):
-    """True if one bijection of block ids maps every model table onto the product's."""
+def _relabel_consistent(model, prod, seqs, host=False):
+    """True if one bijection of block ids maps every model table onto the product's
+    (device ids, or with ``host`` the host swap-space ids of swapped sequences)."""
     fwd, bwd = {}, {}
+    mref = model.host_ref if host else model.ref
     for s in seqs:
         a, b = model.block_table(s), prod.block_table(s)
         if len(a) != len(b):
             return False
         for x, y in zip(a, b):
+            if x == -1 or y == -1:  # released by a sliding window: on both sides
+                if x != y:
+                    return False
+                continue
             if fwd.setdefault(x, y) != y or bwd.setdefault(y, x) != x:
                 return False
-            if model.ref[x] != prod.ref_count(y):
+            if not host and mref[x] != prod.ref_count(y):
                 return False
     return True
 
 
-@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
 def test_random_trace_matches_model_up_to_relabelling(seed):
     rng = np.random.default_rng(seed)
-    bs, nb = 8, 96
+    bs, nb, nh = 8, 96, 40
     model, prod = BlockManagerModel(nb, bs), BlockManager(nb, bs)
+    model.set_host_blocks(nh)
+    prod.set_host_blocks(nh)
     live, next_id = [], 0
-    for _ in range(1500):
-        op = rng.choice(["add", "fork", "append", "append", "append", "free"])
-        if op == "add" or not live:
+    ops = ["add", "fork", "append", "append", "append", "free", "window", "swap_out", "swap_in"]
+    for _ in range(2000):
+        op = rng.choice(ops)
+        resident = [s for s in live if s not in model.swapped]
+        swapped = [s for s in live if s in model.swapped]
+        if op == "add" or not resident:
             n = int(rng.integers(0, 40))
             try:
                 model.add_seq(next_id, n)
@@ -189,13 +200,13 @@ def test_random_trace_matches_model_up_to_relabelling(seed):
                     prod.add_seq(next_id, n)
             next_id += 1
         elif op == "fork":
-            p = int(rng.choice(live))
+            p = int(rng.choice(resident))
             model.fork(p, next_id)
             prod.fork(p, next_id)
             live.append(next_id)
             next_id += 1
         elif op == "append":
-            s = int(rng.choice(live))
+            s = int(rng.choice(resident))
             try:
                 ms, msrc, mdst = model.append_slot(s)
                 ok = True
@@ -208,14 +219,69 @@ def test_random_trace_matches_model_up_to_relabelling(seed):
             else:
                 with pytest.raises(OutOfBlocks):
                     prod.append_slot(s)
+        elif op == "window":
+            s = int(rng.choice(resident))
+            w = int(rng.integers(1, 30))
+            assert model.slide_window(s, w) == prod.slide_window(s, w)
+        elif op in ("swap_out", "swap_in"):
+            pool = resident if op == "swap_out" else swapped
+            if not pool:
+                continue
+            k = int(rng.integers(1, min(3, len(pool)) + 1))
+            group = [int(x) for x in rng.choice(pool, size=k, replace=False)]
+            try:
+                mp = getattr(model, op)(group)
+                ok = True
+            except ModelOOM:
+                ok = False
+            if ok:
+                pp = getattr(prod, op)(group)
+                assert len(mp) == len(pp)
+                for g in group:
+                    assert prod.is_swapped(g) == (op == "swap_out")
+            else:
+                with pytest.raises(OutOfBlocks):
+                    getattr(prod, op)(group)
         else:
             s = int(rng.choice(live))
             model.free_seq(s)
             prod.free_seq(s)
             live.remove(s)
         assert model.num_free() == prod.num_free()
-        assert _relabel_consistent(model, prod, live)
+        assert len(model.host_free) == prod.host_free()
+        assert _relabel_consistent(model, prod, [s for s in live if s not in model.swapped])
+        assert _relabel_consistent(model, prod, [s for s in live if s in model.swapped], host=True)
         assert model.stats() == prod.stats()
+
+
+def test_swap_group_shares_blocks_once():
+    m = BlockManager(16, 4)
+    m.set_host_blocks(8)
+    m.add_seq(0, 6)                  # 2 blocks
+    m.fork(0, 1)                     # both shared (ref 2)
+    m.add_seq(2, 3)                  # 1 private block
+    t0 = m.block_table(0)
+    free0 = m.num_free()
+    pairs = m.swap_out([0, 1])       # the shared blocks move once
+    assert sorted(pairs[:, 0].tolist()) == sorted(t0)
+    assert m.num_free() == free0 + 2 and m.host_free() == 6
+    assert m.block_table(0) == m.block_table(1) == pairs[:, 1].tolist()
+    with pytest.raises(PAError):
+        m.append_slot(0)             # swapped: no slots
+    with pytest.raises(PAError):
+        m.swap_out([0])              # already out
+    back = m.swap_in([1, 0])
+    assert back[:, 0].tolist() == pairs[:, 1].tolist()
+    assert m.block_table(0) == m.block_table(1) == back[:, 1].tolist()
+    assert [m.ref_count(b) for b in m.block_table(0)] == [2, 2] and m.host_free() == 8
+    # a block also held outside the group is copied and stays for the other sequence
+    m.fork(2, 3)
+    p2 = m.swap_out([3])
+    assert p2.shape == (1, 2) and m.ref_count(m.block_table(2)[0]) == 1
+    m.free_seq(3)                    # a swapped sequence frees its host blocks
+    assert m.host_free() == 8
+    with pytest.raises(PAError):
+        m.swap_in([2])               # not swapped
 
 
 def test_fill_tables():
@@ -291,3 +357,28 @@ def test_decode_step_bytes():
     assert b["kv"] == 2 * 50 * 8 * 128 * 2
     assert b["block_tables"] == (1 + 2 + 2) * 4
     assert b["total"] == b["kv"] + 2 * 3 * 32 * 128 * 2 + 20 + 12
+
+
+def test_slide_window_releases_only_blocks_before_the_window():
+    m = BlockManager(16, 4)
+    m.add_seq(0, 10)                       # blocks for positions 0-3, 4-7, 8-9
+    t0 = m.block_table(0)
+    assert m.slide_window(0, 5) == 1       # window [5, 10): only block 0 is wholly before it
+    assert m.block_table(0) == [-1] + t0[1:]
+    assert m.slide_window(0, 5) == 0       # repeating it changes nothing
+    with pytest.raises(PAError):
+        m.seq_slots(0, 3, 2)               # position 3 was released
+    assert m.seq_slots(0, 4, 6).tolist() == [t0[1] * 4 + i for i in range(4)] + [t0[2] * 4, t0[2] * 4 + 1]
+    m.fork(0, 1)                            # a fork shares what is left
+    assert m.block_table(1) == [-1] + t0[1:]
+    assert m.slide_window(1, 2) == 0       # block 1 is still held by sequence 0
+    assert m.ref_count(t0[1]) == 1
+    assert m.slide_window(0, 2) == 1       # now nobody holds it
+    m.free_seq(0)
+    m.free_seq(1)
+    assert m.stats()[0] == 16
+    with pytest.raises(PAError):
+        m.slide_window(7, 3)
+    m.add_seq(2, 3)
+    with pytest.raises(PAError):
+        m.slide_window(2, 0)
