@@ -71,6 +71,8 @@ def _load(path: str):
     L.oracle_decode_window.argtypes = [P, P, P, P, P, i, P, i, i, i, i, i, i, f, i, i, i]
     L.oracle_swap_blocks.restype = i
     L.oracle_swap_blocks.argtypes = [P, P, i, P, P, i, P, i, i, i, i]
+    L.oracle_prefill.restype = i
+    L.oracle_prefill.argtypes = [P, P, P, P, P, i, P, P, i, i, i, i, i, i, f, i, i, i]
     L.oracle_max_threads.argtypes = []
     return L
 
@@ -217,6 +219,27 @@ def decode_window(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
                                     _ptr(cl), B, hq, hkv, d, bs, nb, float(scale),
                                     DTYPE_CODE[dtype], int(window), num_threads)
     _check(rc, "oracle_decode_window")
+    return out
+
+
+def prefill(q, k_cache, v_cache, block_tables, context_lens, q_start, scale, dtype, window=0,
+            num_threads=0):
+    """fp64 outputs [T, Hq, D] of paged prefill attention: the query rows of
+    sequence b are q[q_start[b]:q_start[b+1]], its last positions; each attends
+    causally (and within ``window`` if > 0)."""
+    T, hq, d = q.shape
+    nb, hkv, bs, d2 = k_cache.shape
+    assert d == d2
+    out = np.zeros((T, hq, d), dtype=np.float64)
+    bt = _need(np.ascontiguousarray(block_tables, dtype=np.int32), np.int32)
+    cl = _need(np.ascontiguousarray(context_lens, dtype=np.int32), np.int32)
+    qs = _need(np.ascontiguousarray(q_start, dtype=np.int32), np.int32)
+    assert len(qs) == len(cl) + 1 and qs[-1] == T
+    rc = lib().oracle_prefill(_ptr(out), _ptr(_need(q, np.uint16)), _ptr(_need(k_cache, np.uint16)),
+                              _ptr(_need(v_cache, np.uint16)), _ptr(bt), bt.shape[1], _ptr(cl),
+                              _ptr(qs), len(cl), hq, hkv, d, bs, nb, float(scale),
+                              DTYPE_CODE[dtype], int(window), num_threads)
+    _check(rc, "oracle_prefill")
     return out
 
 

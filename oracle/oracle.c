@@ -554,6 +554,80 @@ int oracle_decode_window(double *out, const uint16_t *q, const uint16_t *k_cache
     return status;
 }
 
+/* Paged attention for several query tokens per sequence (prefill, or a chunk
+ * of one): "PagedAttention 核心思想解析", section 2.2 -- the rows of Q are cut
+ * into blocks, each scored against the sequence's K/V blocks found through the
+ * block table, the partial results merged by position. Sequence b holds
+ * n = context_lens[b] positions; its query tokens are rows q_start[b] ..
+ * q_start[b+1]-1 of q and are its last m = q_start[b+1] - q_start[b]
+ * positions, n-m .. n-1 (their K/V already in the pool). The token at position
+ * p attends to positions [lo, p] with lo = max(0, p + 1 - window) when
+ * window > 0, else lo = 0: a token sees itself and earlier positions only.
+ * out: double [T][num_q_heads][head_dim], T = q_start[num_seqs]. */
+int oracle_prefill(double *out, const uint16_t *q, const uint16_t *k_cache,
+                   const uint16_t *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                   const int32_t *context_lens, const int32_t *q_start, int num_seqs,
+                   int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                   int num_blocks, float scale, int dtype, int window, int num_threads)
+{
+    int rc = check_shapes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                          num_blocks, max_blocks_per_seq);
+    if (rc)
+        return rc;
+    if (q_start[0] != 0)
+        return ORC_BAD_ARG;
+    for (int b = 0; b < num_seqs; ++b) {
+        int m = q_start[b + 1] - q_start[b];
+        if (m < 0 || m > context_lens[b] || context_lens[b] > max_blocks_per_seq * block_size)
+            return ORC_BAD_ARG;
+    }
+    int group = num_q_heads / num_kv_heads;
+    int nthreads = set_threads(num_threads);
+    int status = ORC_OK;
+    long long units = (long long)q_start[num_seqs] * num_q_heads;
+#ifdef _OPENMP
+#pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
+#endif
+    for (long long u = 0; u < units; ++u) {
+        int tok = (int)(u / num_q_heads), h = (int)(u % num_q_heads);
+        int b = 0;
+        while (q_start[b + 1] <= tok)
+            ++b;
+        int n = context_lens[b];
+        int m = q_start[b + 1] - q_start[b];
+        int p = n - m + (tok - q_start[b]);           /* this token's position */
+        int lo = (window > 0 && p + 1 > window) ? p + 1 - window : 0;
+        int cnt = p + 1 - lo;
+        int g = h / group;
+        double *K = malloc(sizeof(double) * ((size_t)cnt * head_dim + 1));
+        double *V = malloc(sizeof(double) * ((size_t)cnt * head_dim + 1));
+        double *sc = malloc(sizeof(double) * ((size_t)cnt + 1));
+        double *qd = malloc(sizeof(double) * (size_t)head_dim);
+        const int32_t *row = block_tables + (size_t)b * max_blocks_per_seq;
+        int r1 = gather_span(K, k_cache, row, lo, p + 1, g, num_blocks, num_kv_heads, block_size,
+                             head_dim, dtype);
+        int r2 = gather_span(V, v_cache, row, lo, p + 1, g, num_blocks, num_kv_heads, block_size,
+                             head_dim, dtype);
+        if (r1 || r2) {
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+            status = ORC_BAD_BLOCK;
+        } else {
+            for (int d = 0; d < head_dim; ++d)
+                qd[d] = widen(q[((size_t)tok * num_q_heads + h) * head_dim + d], dtype);
+            attend_rows(out + ((size_t)tok * num_q_heads + h) * head_dim, qd, K, V, cnt,
+                        head_dim, (double)scale, sc);
+        }
+        free(K);
+        free(V);
+        free(sc);
+        free(qd);
+    }
+    (void)nthreads;
+    return status;
+}
+
 int oracle_max_threads(void)
 {
     return set_threads(0);

@@ -328,3 +328,40 @@ def small_random(seed: int, num_seqs: int, lens, num_q_heads: int, num_kv_heads:
     ids = rng.permutation(num_blocks)[: num_seqs * width]
     return _assemble("small", rng, dtype, lens, num_q_heads, num_kv_heads, head_dim, block_size,
                      num_blocks, ids, width)
+
+
+# ------------------------------------------------------------------------------------ prefill
+def prefill_random(seed: int, lens, q_lens, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                   block_size: int, num_blocks: int, dtype: str, width: int | None = None,
+                   name: str = "prefill") -> DecodeBatch:
+    """A prefill (or chunked-prefill) batch: sequence b holds lens[b] positions of
+    which the last q_lens[b] are this step's query tokens. ``q`` is [T, Hq, D]
+    with T = sum(q_lens), rows in sequence order; ``meta['q_start']`` (int32
+    [B + 1]) delimits each sequence's rows. K/V rows cover every position (the
+    new tokens' included: they are written to the pool before attending)."""
+    rng = np.random.default_rng(seed)
+    lens = np.asarray(lens, dtype=np.int32)
+    q_lens = np.asarray(q_lens, dtype=np.int32)
+    assert len(lens) == len(q_lens) and np.all(q_lens <= lens) and np.all(q_lens >= 0)
+    if width is None:
+        width = _table_width(int(lens.max()) if len(lens) else 1, block_size)
+    if len(lens) * width > num_blocks:
+        raise ValueError("pool too small for full-width tables")
+    ids = rng.permutation(num_blocks)[: len(lens) * width]
+    q_start = np.zeros(len(lens) + 1, dtype=np.int32)
+    np.cumsum(q_lens, out=q_start[1:])
+    q = _normal_bits(rng, (int(q_start[-1]), num_q_heads, head_dim), dtype)
+    return _assemble(name, rng, dtype, lens, num_q_heads, num_kv_heads, head_dim, block_size,
+                     num_blocks, ids, width, meta={"q_start": q_start, "q_lens": q_lens}, q=q)
+
+
+def llama8b_prefill(seed: int = SEED_BASE + 7, num_blocks: int = 65536) -> DecodeBatch:
+    """Chunked prefill on the Llama-3.1-8B shapes (32 q / 8 KV heads, head_dim
+    128, bf16, 16-token blocks): 16 sequences, each with a history uniform in
+    [0, 1536] positions and a chunk of 512 new query tokens."""
+    rng = np.random.default_rng(seed)
+    hist = rng.integers(0, 1537, size=16)
+    q_lens = np.full(16, 512, dtype=np.int32)
+    lens = (hist + q_lens).astype(np.int32)
+    return prefill_random(seed + 1, lens, q_lens, 32, 8, 128, 16, num_blocks, BF16,
+                          width=_table_width(2048, 16), name="llama8b_prefill")

@@ -357,6 +357,112 @@ def pin_window_bruteforce_fsum():
                 assert abs(got[b, h, d] - ref) <= 1e-13, "window brute force disagrees"
 
 
+# --------------------------------------------------------------------------- prefill
+def prefill_batches():
+    """Small prefill batches: GQA and MHA, both dtypes, chunks with and without
+    history, a whole prompt, single-token chunks, ragged block tails."""
+    return [
+        synth.prefill_random(61, [5, 20, 33, 7], [3, 20, 16, 1], 4, 2, 16, 4, 60, "f16", width=10),
+        synth.prefill_random(62, [64, 17, 40], [64, 9, 40], 8, 2, 32, 16, 30, "bf16", width=6),
+        synth.prefill_random(63, [1, 12, 30], [1, 12, 5], 6, 6, 8, 8, 40, "f16", width=6),
+    ]
+
+
+def dense_prefill_reference(batch, window=0):
+    """Causal attention of each sequence's query rows over its logical rows,
+    numpy fp64: query i of sequence b sits at position n - m + i and its
+    scores against later positions (or, with a window, positions before
+    p + 1 - window) are masked out before the softmax."""
+    G = batch.num_q_heads // batch.num_kv_heads
+    qs = batch.meta["q_start"]
+    q = lib_f64(batch.q, batch.dtype)
+    out = np.zeros(q.shape)
+    for b in range(batch.num_seqs):
+        n, m = int(batch.context_lens[b]), int(qs[b + 1] - qs[b])
+        if m == 0:
+            continue
+        K = lib_f64(batch.k[batch.rows(b)], batch.dtype)
+        V = lib_f64(batch.v[batch.rows(b)], batch.dtype)
+        pos = n - m + np.arange(m)
+        keys = np.arange(n)
+        mask = keys[None, :] > pos[:, None]
+        if window > 0:
+            mask |= keys[None, :] < (pos[:, None] + 1 - window)
+        for h in range(batch.num_q_heads):
+            S = (q[qs[b]:qs[b + 1], h, :] @ K[:, h // G, :].T) * float(batch.scale)
+            S[mask] = -np.inf
+            W = np.exp(S - S.max(axis=1, keepdims=True))
+            out[qs[b]:qs[b + 1], h, :] = (W @ V[:, h // G, :]) / W.sum(axis=1, keepdims=True)
+    return out
+
+
+def _oracle_prefill(batch, kp=None, vp=None, window=0, tables=None):
+    if kp is None:
+        kp, vp = place_numpy(batch)
+    return oracle.prefill(batch.q, kp, vp, batch.block_tables if tables is None else tables,
+                          batch.context_lens, batch.meta["q_start"], batch.scale, batch.dtype,
+                          window)
+
+
+def pin_prefill_dense():
+    for batch in prefill_batches():
+        kp, vp = place_numpy(batch)
+        for w in (0, 1, 3, 17):
+            got = _oracle_prefill(batch, kp, vp, w)
+            err = np.max(np.abs(got - dense_prefill_reference(batch, w)))
+            assert err <= 1e-12, f"{batch.name} window {w}: prefill off by {err}"
+
+
+def pin_prefill_first_token_of_a_prompt():
+    """A whole prompt as the chunk: its first token sees only itself, so its
+    output is its own V row exactly."""
+    batch = synth.prefill_random(64, [9, 30], [9, 30], 8, 4, 16, 4, 30, "bf16", width=9)
+    got = _oracle_prefill(batch)
+    G = batch.num_q_heads // batch.num_kv_heads
+    qs = batch.meta["q_start"]
+    for b in range(batch.num_seqs):
+        v0 = lib_f64(batch.v[batch.rows(b).start], batch.dtype)
+        for h in range(batch.num_q_heads):
+            assert np.array_equal(got[qs[b], h], v0[h // G]), "first prompt token must return its V"
+
+
+def pin_prefill_bruteforce_fsum():
+    batch = synth.prefill_random(65, [6, 4], [4, 2], 4, 2, 8, 4, 12, "f16", width=3)
+    got = _oracle_prefill(batch)
+    G = batch.num_q_heads // batch.num_kv_heads
+    qs = batch.meta["q_start"]
+    q = lib_f64(batch.q, batch.dtype).tolist()
+    for b in range(batch.num_seqs):
+        K = lib_f64(batch.k[batch.rows(b)], batch.dtype).tolist()
+        V = lib_f64(batch.v[batch.rows(b)], batch.dtype).tolist()
+        n, m = len(K), int(qs[b + 1] - qs[b])
+        for i in range(m):
+            p = n - m + i
+            for h in range(batch.num_q_heads):
+                g = h // G
+                s = [float(batch.scale) * math.fsum(q[qs[b] + i][h][d] * K[t][g][d]
+                                                    for d in range(batch.head_dim))
+                     for t in range(p + 1)]
+                mx = max(s)
+                w = [math.exp(x - mx) for x in s]
+                den = math.fsum(w)
+                for d in range(batch.head_dim):
+                    ref = math.fsum(w[t] * V[t][g][d] for t in range(p + 1)) / den
+                    assert abs(got[qs[b] + i, h, d] - ref) <= 1e-13, "prefill brute force"
+
+
+def pin_prefill_relabel():
+    batch = prefill_batches()[1]
+    kp, vp = place_numpy(batch)
+    base = _oracle_prefill(batch, kp, vp)
+    perm = np.random.default_rng(6).permutation(batch.num_blocks)
+    kp2, vp2 = np.empty_like(kp), np.empty_like(vp)
+    kp2[perm] = kp
+    vp2[perm] = vp
+    got = _oracle_prefill(batch, kp2, vp2, tables=perm[batch.block_tables].astype(np.int32))
+    assert np.array_equal(got, base), "relabelling physical blocks changed the prefill output"
+
+
 # --------------------------------------------------------------------------- write / copy
 def pin_reshape_layout():
     """Write the worked example's 10 tokens (block size 4, blocks 8, 3, 15) at the
@@ -554,7 +660,8 @@ ALL_ORACLE_PINS = [
     pin_len1_returns_v, pin_identical_keys_mean_v, pin_bruteforce_fsum, pin_relabel, pin_poison,
     pin_partition_merge, pin_reshape_layout, pin_copy_blocks, pin_window_dense,
     pin_window_one_returns_last_v, pin_window_ignores_what_it_left, pin_window_bruteforce_fsum,
-    pin_swap_blocks,
+    pin_swap_blocks, pin_prefill_dense, pin_prefill_first_token_of_a_prompt,
+    pin_prefill_bruteforce_fsum, pin_prefill_relabel,
 ]
 ALL_MODEL_PINS = [pin_allocator_worked_example, pin_allocator_capacity, pin_allocator_cow,
                   pin_allocator_sliding_window, pin_allocator_swap]

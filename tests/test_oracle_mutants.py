@@ -39,6 +39,9 @@ MUTANTS = {
                             "dst[(size_t)(t - lo) * head_dim + d] =\n                widen(pool[pool_index(block, kv_head, offset > 0 ? offset - 1 : 0, d,"),
     "swap_v_from_k": ("dst_v[(size_t)dst * block_elems + i] = src_v[(size_t)src * block_elems + i];",
                       "dst_v[(size_t)dst * block_elems + i] = src_k[(size_t)src * block_elems + i];"),
+    "prefill_not_causal": ("int p = n - m + (tok - q_start[b]);", "int p = n - 1;"),
+    "prefill_position_shifted": ("int p = n - m + (tok - q_start[b]);",
+                                 "int p = n - m + (tok - q_start[b]) - (tok > q_start[b]);"),
     "copy_k_only": ("v_cache[(size_t)dst * block_elems + i] = v_cache[(size_t)src * block_elems + i];",
                     ";"),
 }
