@@ -63,12 +63,14 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama8b",
-                    choices=["llama8b", "long_skew", "mixed", "shared_prompt"])
+                    choices=["llama8b", "long_skew", "mixed", "shared_prompt", "swap"])
     ap.add_argument("--block-size", type=int, default=16, help="block size of the mixed workload")
     ap.add_argument("--variants", type=int, default=4, help="batches rotated (llama8b)")
     ap.add_argument("--partition-tokens", type=int, default=0)
     ap.add_argument("--pool-blocks", type=int, default=65536,
                     help="llama8b pool size (smaller for profiler captures)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding window: attend to each sequence's last W positions (0: all)")
     ap.add_argument("--no-fuse", action="store_true",
                     help="separate KV-write kernel instead of pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
@@ -183,6 +185,13 @@ def make_batches(args, rank):
 
 
 def workload_config(args, batches, pt):
+    cfg = _workload_config(args, batches, pt)
+    if getattr(args, "window", 0) > 0:
+        cfg["window"] = args.window
+    return cfg
+
+
+def _workload_config(args, batches, pt):
     if args.workload == "llama8b":
         b = batches[0]
         return {"workload": "Llama-3.1-8B-shaped single-layer paged decode",
@@ -241,16 +250,20 @@ def device_steps(args, batches, torch, device):
                           block_tables=torch.from_numpy(b.block_tables).to(device),
                           context_lens=torch.from_numpy(b.context_lens).to(device),
                           max_context_len=b.max_context_len, scale=float(b.scale),
-                          partition_tokens=args.partition_tokens, fused=not args.no_fuse)
+                          partition_tokens=args.partition_tokens, fused=not args.no_fuse,
+                          window=args.window)
         del k_all, v_all
         steps.append(step)
         infos.append(_byte_info(b.context_lens, b.num_q_heads, b.num_kv_heads, b.head_dim,
-                                b.block_size, step.partition, b.num_seqs))
+                                b.block_size, step.partition, b.num_seqs, args.window))
     torch.cuda.synchronize()
     return steps, infos
 
 
-def _byte_info(lens, hq, hkv, d, bs, pt, ntok):
+def _byte_info(lens, hq, hkv, d, bs, pt, ntok, window=0):
+    if window > 0:
+        # the positions a window reads: the last `window` of each sequence
+        lens = np.minimum(np.asarray(lens), window)
     return {"decode": decode_step_bytes(lens, hq, hkv, d, bs),
             "scratch": split_scratch_bytes(lens, hq, d, pt),
             "write": new_token_bytes(ntok, hkv, d), "lens": np.asarray(lens)}
@@ -609,6 +622,49 @@ def run_reference(args, rank, world):
             "query_tokens_per_s": round(total_q / total_t, 2)}
 
 
+# ------------------------------------------------------------------------------------- swap
+def run_swap(args):
+    """Block swap between the device pool and the pinned host swap space
+    (pa_swap_out / pa_swap_in): Llama-3.1-8B-shaped blocks (8 kv heads x 16
+    slots x 128 bf16, K and V = 64 KiB per block), 2048 random blocks per call
+    (128 MiB each way), CUDA events on the stream, one call per direction per step."""
+    import torch
+    from paged_kv_cache_370_b200 import abi
+    dev = torch.device("cuda", 0)
+    nb, nh, hkv, bs, d, n = 65536, 4096, 8, 16, 128, 2048
+    kc = torch.zeros((nb, hkv, bs, d), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    space = abi.SwapSpace(nh, hkv, bs, d, "bf16")
+    rng = np.random.default_rng(9)
+    out_pairs = torch.from_numpy(np.stack([rng.permutation(nb)[:n], rng.permutation(nh)[:n]], 1)
+                                 .astype(np.int64)).to(dev)
+    in_pairs = torch.from_numpy(np.stack([out_pairs[:, 1].cpu().numpy(), rng.permutation(nb)[:n]], 1)
+                                .astype(np.int64)).to(dev)
+    nbytes = n * 2 * hkv * bs * d * 2
+    res = {}
+    for name, fn, pairs in (("out", abi.pa_swap_out, out_pairs), ("in", abi.pa_swap_in, in_pairs)):
+        for _ in range(args.warmup):
+            fn(space, kc, vc, pairs)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn(space, kc, vc, pairs)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        res[name] = {"ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 2)}
+    code = abi.pa_device_status()
+    space.close()
+    return {"metric": "KV block swap GB/s (device pool <-> pinned host swap space)",
+            "value": round((res["out"]["GB/s"] + res["in"]["GB/s"]) / 2, 2), "unit": "GB/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "swap 2048 random 64 KiB blocks each way", "bytes_per_call": nbytes},
+            "out": res["out"], "in": res["in"], "device_error_word": code,
+            "gpu_launches": 2 * args.steps}
+
+
 # ------------------------------------------------------------------------------------- main
 def main():
     args = parse_args()
@@ -617,6 +673,10 @@ def main():
         if rank != 0:
             return 0
         print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+    if args.workload == "swap":
+        if rank == 0:
+            print(json.dumps(run_swap(args)), flush=True)
         return 0
     dist = None
     if world > 1:

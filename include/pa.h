@@ -241,6 +241,71 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
                            int num_blocks, float scale, pa_dtype dtype, void *workspace,
                            size_t workspace_bytes, int partition_tokens, void *stream);
 
+/* ------------------------------------------------------------------------------------------
+ * pa_decode_window / pa_decode_append_window -- decode over a sliding window.
+ * [P2, section 5.2: a sliding window reclaims the blocks that fall out of it.]
+ * Each sequence of length len attends only to its last `window` positions,
+ * [max(0, len - window), len): softmax over those scores, the same arithmetic
+ * as pa_decode otherwise. Block-table entries of blocks wholly before that
+ * range are never read, so they may hold anything -- e.g. the -1 that
+ * pa_alloc_slide_window leaves. Arguments as pa_decode / pa_decode_append plus
+ * `window` (> 0; PA_ERR_INVALID otherwise); pa_decode_workspace_size covers it.
+ * A window runs in the partition kernel (partitions of the window's positions,
+ * then the merge kernel when the longest context has more than one);
+ * pa_decode_append_window writes the new tokens with pa_reshape_and_cache
+ * first. pa_decode_window_launches gives the kernels pa_decode_window launches
+ * (pa_decode_append_window: one more).
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_decode_window(void *out, const void *q, const void *k_cache, const void *v_cache,
+                           const int32_t *block_tables, int max_blocks_per_seq,
+                           const int32_t *context_lens, int max_context_len, int num_seqs,
+                           int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                           int num_blocks, float scale, int window, pa_dtype dtype,
+                           void *workspace, size_t workspace_bytes, int partition_tokens,
+                           void *stream);
+int pa_decode_window_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                              int max_context_len, int window, int partition_tokens);
+pa_status pa_decode_append_window(void *out, const void *q, const void *k_new, const void *v_new,
+                                  const int64_t *slot_mapping, void *k_cache, void *v_cache,
+                                  const int32_t *block_tables, int max_blocks_per_seq,
+                                  const int32_t *context_lens, int max_context_len, int num_seqs,
+                                  int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                  int num_blocks, float scale, int window, pa_dtype dtype,
+                                  void *workspace, size_t workspace_bytes, int partition_tokens,
+                                  void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * pa_prefill -- paged attention for several query tokens per sequence (a prompt, or one
+ * chunk of a chunked prefill).
+ * [P2, section 2.2: the rows of Q are cut into blocks, each block is scored against the
+ * sequence's K/V blocks found through the block table, and the partial results are merged
+ * by position. P3, section "借用操作系统的办法：分页": a request's prefill takes the blocks
+ * it needs.]
+ *
+ *   q             device, [num_tokens][num_q_heads][head_dim]: the query tokens of every
+ *                 sequence back to back, sequence b's rows q_start[b] .. q_start[b+1]-1
+ *   q_start       device, int32 [num_seqs + 1], q_start[0] = 0, non-decreasing,
+ *                 q_start[num_seqs] = num_tokens
+ *   context_lens  device, int32 [num_seqs]: positions of each sequence, the query tokens
+ *                 included -- they are its last q_start[b+1]-q_start[b] positions, and
+ *                 their K/V must already be in the pool (pa_reshape_and_cache)
+ *   max_q_len     host: the largest q_start[b+1]-q_start[b] (sizes the grid)
+ *   window        0, or > 0: each token attends to its last `window` positions only
+ *   out           device, [num_tokens][num_q_heads][head_dim], same dtype as q
+ * The token at position p of its sequence attends to positions [lo, p], lo = 0 or
+ * p + 1 - window: softmax(scale * q . K^T) V over those positions, fp32 arithmetic.
+ * head_dim 64 or 128; block_size a power of two >= 8 (PA_ERR_UNSUPPORTED otherwise).
+ * Allocates nothing. Lengths or q_start entries out of range are clamped and reported
+ * (PA_DEVERR_CONTEXT_LEN); bad block ids are skipped and reported (PA_DEVERR_BLOCK_ID).
+ * One kernel launch.
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *block_tables, int max_blocks_per_seq,
+                     const int32_t *context_lens, const int32_t *q_start, int num_seqs,
+                     int num_tokens, int max_q_len, int max_context_len, int num_q_heads,
+                     int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
+                     int window, pa_dtype dtype, void *stream);
+
 /* Kernels one pa_decode_append call with these arguments launches (0 if none). */
 int pa_decode_append_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                               int block_size, int num_blocks, int max_context_len,

@@ -61,6 +61,11 @@ def _load() -> ctypes.CDLL:
         "pa_decode_append": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, P, sz,
                                  i, P]),
         "pa_decode_append_launches": (i, [i, i, i, i, i, i, i, i]),
+        "pa_decode_window": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P, sz, i, P]),
+        "pa_decode_window_launches": (i, [i, i, i, i, i, i, i]),
+        "pa_prefill": (i, [P, P, P, P, P, i, P, P, i, i, i, i, i, i, i, i, i, f, i, i, P]),
+        "pa_decode_append_window": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i,
+                                        P, sz, i, P]),
         "pa_decode_static_workspace": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P]),
         "pa_device_status": (i, [P, P]),
         "pa_status_string": (ctypes.c_char_p, [i]),
@@ -248,6 +253,60 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
                         _dtype_code(q), _dev_ptr(workspace, "workspace"), ws_bytes,
                         int(partition_tokens), _stream(stream))
     _check(st, "pa_decode")
+
+
+def pa_decode_window(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len, scale,
+                     window, workspace=None, partition_tokens=0, stream=None):
+    """pa_decode over each sequence's last ``window`` positions only."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.pa_decode_window(_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+                               _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+                               int(block_tables.shape[1]), _dev_ptr(context_lens, "context_lens"),
+                               int(max_context_len), B, hq, hkv, d, bs, nb, float(scale),
+                               int(window), _dtype_code(q), _dev_ptr(workspace, "workspace"),
+                               ws_bytes, int(partition_tokens), _stream(stream))
+    _check(st, "pa_decode_window")
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, q_start, max_q_len,
+               max_context_len, scale, window=0, stream=None):
+    """Paged prefill attention: out[T, Hq, D] for the query tokens q[T, Hq, D] of every
+    sequence (rows q_start[b]:q_start[b+1], the sequence's last positions), causal."""
+    T, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    st = _lib.pa_prefill(_dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_cache, "k_cache"),
+                         _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+                         int(block_tables.shape[1]), _dev_ptr(context_lens, "context_lens"),
+                         _dev_ptr(q_start, "q_start"), int(context_lens.shape[0]), T,
+                         int(max_q_len), int(max_context_len), hq, hkv, d, bs, nb, float(scale),
+                         int(window), _dtype_code(q), _stream(stream))
+    _check(st, "pa_prefill")
+
+
+def pa_decode_window_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                              window, partition_tokens=0) -> int:
+    """Kernels one pa_decode_window call with these arguments launches."""
+    return int(_lib.pa_decode_window_launches(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                              max_context_len, window, partition_tokens))
+
+
+def pa_decode_append_window(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,
+                            context_lens, max_context_len, scale, window, workspace=None,
+                            partition_tokens=0, stream=None):
+    """pa_decode_append over each sequence's last ``window`` positions only."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.pa_decode_append_window(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_new, "k_new"), _dev_ptr(v_new, "v_new"),
+        _dev_ptr(slot_mapping, "slot_mapping"), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+        int(block_tables.shape[1]), _dev_ptr(context_lens, "context_lens"), int(max_context_len),
+        B, hq, hkv, d, bs, nb, float(scale), int(window), _dtype_code(q),
+        _dev_ptr(workspace, "workspace"), ws_bytes, int(partition_tokens), _stream(stream))
+    _check(st, "pa_decode_append_window")
 
 
 def pa_decode_append(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,

@@ -45,6 +45,7 @@
 
 #include "pa.h"
 #include "pa_internal.h"
+#include "pa_ptx.cuh"
 
 namespace {
 
@@ -55,45 +56,6 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kStages = 4;
 constexpr int kTileBytes = 8192;                 // bytes of K (and of V) per stage
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
-
-// ------------------------------------------------------------------------------------ PTX wraps
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_expect_tx_arrive(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
-                   smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
 
 // Wait for phase `parity` of `bar` to complete, at most kWaitLimitNs; also give
 // up when another thread of the CTA has raised *abort. Returns false on give-up.
@@ -111,60 +73,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
   }
 }
-
-// 1-D TMA bulk copy global -> shared, completion counted on `bar` in bytes.
-__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes,
-                                         uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst_smem)),
-      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// ------------------------------------------------------------------------ element conversions
-template <typename T>
-struct Elem;
-
-template <>
-struct Elem<__nv_bfloat16> {
-  // 8 packed bf16 -> 8 floats (a bf16 is the upper half of a float)
-  static __device__ __forceinline__ void to_f32(const uint4 &r, float (&f)[8]) {
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      f[2 * i] = __uint_as_float(w[i] << 16);
-      f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-  }
-  static __device__ __forceinline__ __nv_bfloat16 from_f32(float a) {
-    return __float2bfloat16_rn(a);
-  }
-  static __device__ __forceinline__ uint2 from_f32x4(float a, float b, float c, float d) {
-    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(c, d);
-    return make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-  }
-};
-
-template <>
-struct Elem<__half> {
-  static __device__ __forceinline__ void to_f32(const uint4 &r, float (&f)[8]) {
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 v = __half22float2(*reinterpret_cast<const __half2 *>(&w[i]));
-      f[2 * i] = v.x;
-      f[2 * i + 1] = v.y;
-    }
-  }
-  static __device__ __forceinline__ __half from_f32(float a) { return __float2half_rn(a); }
-  static __device__ __forceinline__ uint2 from_f32x4(float a, float b, float c, float d) {
-    __half2 lo = __floats2half2_rn(a, b);
-    __half2 hi = __floats2half2_rn(c, d);
-    return make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-  }
-};
 
 // ------------------------------------------------------------------- reduce-scatter over lanes
 // N values per lane, over the lanes of one token group (offsets O, O/2, ...):
@@ -228,7 +136,14 @@ struct DecodeParams {
   const int64_t *new_slots;  // nullptr: no fused write
   void *k_cache_w;
   void *v_cache_w;
+  // sliding window (partition kernel only): a sequence of length len attends
+  // to positions [len - window, len) (0: every position)
+  int window;
 };
+
+// First position attended by a sequence of length len under a window of w
+// positions (w <= 0: no window).
+__device__ __forceinline__ int window_lo(int len, int w) { return w > 0 && len > w ? len - w : 0; }
 
 template <int D>
 struct Shape {
@@ -291,9 +206,11 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (tid == 0 && part == 0 && kvh == 0) atomicOr(&g_decode_error, PA_DEVERR_CONTEXT_LEN);
     len = len < 0 ? 0 : min(min(len, cap), p.max_context_len);
   }
-  const int nparts = len > 0 ? (len + p.partition_tokens - 1) / p.partition_tokens : 1;
+  // partitions cover [lo, len): blocks before a sliding window are never read
+  const int lo = window_lo(len, p.window);
+  const int nparts = len > lo ? (len - lo + p.partition_tokens - 1) / p.partition_tokens : 1;
   if (part >= nparts) return;
-  const int t_begin = part * p.partition_tokens;
+  const int t_begin = lo + part * p.partition_tokens;
   const int t_end = min(len, t_begin + p.partition_tokens);
   const int ntok = t_end - t_begin;  // may be 0 only for an empty sequence
   const int ntiles = (ntok + TILE - 1) / TILE;
@@ -631,90 +548,6 @@ constexpr int kWarps = 4;            // consumer warps, 16 tokens each
 constexpr int kThreads = (kWarps + 2) * 32;
 constexpr int kPanelBytes = kTile * 128;  // 64 columns of 2 bytes x 64 rows
 constexpr int kIdWindow = 8;             // tiles of block ids fetched ahead of their copies
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// 4-byte global -> shared copy that does not block the issuing thread
-__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
-  uint32_t d;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
-  return d;
-}
-
-template <typename T>
-struct Mma;
-
-template <>
-struct Mma<__nv_bfloat16> {
-  static __device__ __forceinline__ void run(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                             uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
-        " {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
-  // two floats -> packed pair (lo in the low half) and the rounded values back
-  static __device__ __forceinline__ uint32_t pack(float lo, float hi, float &rlo, float &rhi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    rlo = __low2float(v);
-    rhi = __high2float(v);
-    return *reinterpret_cast<uint32_t *>(&v);
-  }
-};
-
-template <>
-struct Mma<__half> {
-  static __device__ __forceinline__ void run(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                             uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7},"
-        " {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
-  static __device__ __forceinline__ uint32_t pack(float lo, float hi, float &rlo, float &rhi) {
-    __half2 v = __floats2half2_rn(lo, hi);
-    rlo = __low2float(v);
-    rhi = __high2float(v);
-    return *reinterpret_cast<uint32_t *>(&v);
-  }
-};
-
-// byte address of 16-byte chunk `chunk` of row `row` in a 128-byte-swizzled panel
-__device__ __forceinline__ uint32_t swz(uint32_t panel, int row, int chunk) {
-  return panel + row * 128 + ((chunk ^ (row & 7)) << 4);
-}
 
 // Per-tile schedule handed from the producer warp to the consumers with the tile.
 struct TileMeta {
@@ -1289,11 +1122,11 @@ template <typename T, int D>
 __global__ void __launch_bounds__(D) pa_decode_merge_kernel(
     void *out_, const float *__restrict__ ws_acc, const float *__restrict__ ws_ml,
     const int32_t *__restrict__ context_lens, int num_q_heads, int partition_tokens,
-    int max_parts, int max_context_len, int cap) {
+    int max_parts, int max_context_len, int cap, int window) {
   const int hqi = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   int len = __ldg(context_lens + b);
   len = len < 0 ? 0 : min(min(len, cap), max_context_len);
-  const int nparts = (len + partition_tokens - 1) / partition_tokens;
+  const int nparts = (len - window_lo(len, window) + partition_tokens - 1) / partition_tokens;
   if (nparts <= 1) return;  // written by the partition kernel
   const size_t hq = (size_t)b * num_q_heads + hqi;
   const float *ml = ws_ml + hq * max_parts * 2;
@@ -1475,7 +1308,7 @@ size_t stream_workspace(int num_seqs, int num_q_heads, int num_kv_heads, int hea
 template <typename T, int D, int G>
 pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dtype dtype,
                         cudaStream_t stream) {
-  if (uses_stream_kernel(G, prm.block_size, prm.num_blocks, prm.num_kv_heads)) {
+  if (prm.window == 0 && uses_stream_kernel(G, prm.block_size, prm.num_blocks, prm.num_kv_heads)) {
     using C = tc::Cfg<D, G>;
     static size_t configured[kMaxDevices] = {};
     const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
@@ -1501,7 +1334,7 @@ pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dty
     dim3 mgrid((unsigned)prm.num_q_heads, (unsigned)num_seqs);
     pa_decode_merge_kernel<T, D><<<mgrid, D, 0, stream>>>(
         out, prm.ws_acc, prm.ws_ml, prm.context_lens, prm.num_q_heads, prm.partition_tokens,
-        prm.max_parts, prm.max_context_len, prm.max_blocks_per_seq * prm.block_size);
+        prm.max_parts, prm.max_context_len, prm.max_blocks_per_seq * prm.block_size, prm.window);
     if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
   }
   return PA_OK;
@@ -1608,7 +1441,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                       int num_blocks, float scale, pa_dtype dtype, void *workspace,
                       size_t workspace_bytes, int partition_tokens, void *stream,
-                      const FusedWrite *fw) {
+                      const FusedWrite *fw, int window) {
+  if (window < 0) return PA_ERR_INVALID;
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
       block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
       (dtype != PA_F16 && dtype != PA_BF16))
@@ -1628,7 +1462,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_UNSUPPORTED;
   const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
   const int max_parts = max_context_len > 0 ? (max_context_len + pt - 1) / pt : 1;
-  const bool streamk = uses_stream_kernel(group, block_size, num_blocks, num_kv_heads);
+  // a sliding window runs in the partition kernel
+  const bool streamk = window == 0 && uses_stream_kernel(group, block_size, num_blocks, num_kv_heads);
   const int nctas = streamk ? stream_grid(num_seqs, num_kv_heads, group, head_dim,
                                           max_context_len, partition_tokens)
                             : 0;
@@ -1663,6 +1498,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   prm.new_slots = fw ? fw->slots : nullptr;
   prm.k_cache_w = fw ? fw->k_cache : nullptr;
   prm.v_cache_w = fw ? fw->v_cache : nullptr;
+  prm.window = window;
   if (fw && !streamk) return PA_ERR_INVALID;  // only the even-split kernel writes
   prm.max_blocks_per_seq = max_blocks_per_seq;
   prm.max_context_len = max_context_len;
@@ -1693,7 +1529,34 @@ extern "C" pa_status pa_decode(void *out, const void *q, const void *k_cache, co
   return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                      max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                      num_blocks, scale, dtype, workspace, workspace_bytes, partition_tokens,
-                     stream, nullptr);
+                     stream, nullptr, 0);
+}
+
+extern "C" pa_status pa_decode_window(void *out, const void *q, const void *k_cache,
+                                      const void *v_cache, const int32_t *block_tables,
+                                      int max_blocks_per_seq, const int32_t *context_lens,
+                                      int max_context_len, int num_seqs, int num_q_heads,
+                                      int num_kv_heads, int head_dim, int block_size,
+                                      int num_blocks, float scale, int window, pa_dtype dtype,
+                                      void *workspace, size_t workspace_bytes,
+                                      int partition_tokens, void *stream) {
+  if (window <= 0) return PA_ERR_INVALID;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, partition_tokens,
+                     stream, nullptr, window);
+}
+
+extern "C" int pa_decode_window_launches(int num_seqs, int num_q_heads, int num_kv_heads,
+                                         int head_dim, int max_context_len, int window,
+                                         int partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+      head_dim <= 0 || window <= 0)
+    return 0;
+  // the partition kernel, and the merge kernel when the longest context has
+  // more than one partition (partitions are sized from max_context_len)
+  const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
+  return max_context_len > pt ? 2 : 1;
 }
 
 extern "C" int pa_decode_append_launches(int num_seqs, int num_q_heads, int num_kv_heads,
@@ -1707,6 +1570,44 @@ extern "C" int pa_decode_append_launches(int num_seqs, int num_q_heads, int num_
   return uses_stream_kernel(group, block_size, num_blocks, num_kv_heads) ? 1 : 1 + decode;
 }
 
+namespace {
+
+pa_status decode_append_impl(void *out, const void *q, const void *k_new, const void *v_new,
+                             const int64_t *slot_mapping, void *k_cache, void *v_cache,
+                             const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *context_lens, int max_context_len, int num_seqs,
+                             int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                             int num_blocks, float scale, pa_dtype dtype, void *workspace,
+                             size_t workspace_bytes, int partition_tokens, void *stream,
+                             int window) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+      block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (num_seqs == 0) return PA_OK;
+  if (!k_new || !v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+      !aligned(slot_mapping, 8))
+    return PA_ERR_INVALID;
+  const int group = num_q_heads / num_kv_heads;
+  if (window == 0 && uses_stream_kernel(group, block_size, num_blocks, num_kv_heads)) {
+    const FusedWrite fw{k_new, v_new, slot_mapping, k_cache, v_cache};
+    return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                       max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
+                       block_size, num_blocks, scale, dtype, workspace, workspace_bytes,
+                       partition_tokens, stream, &fw, 0);
+  }
+  // other shapes, and sliding windows: the write kernel, then the decode
+  const pa_status st = pa_reshape_and_cache(k_new, v_new, slot_mapping, num_seqs, k_cache,
+                                            v_cache, num_blocks, num_kv_heads, block_size,
+                                            head_dim, dtype, stream);
+  if (st != PA_OK) return st;
+  return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                     num_blocks, scale, dtype, workspace, workspace_bytes, partition_tokens,
+                     stream, nullptr, window);
+}
+
+}  // namespace
+
 extern "C" pa_status pa_decode_append(void *out, const void *q, const void *k_new,
                                       const void *v_new, const int64_t *slot_mapping,
                                       void *k_cache, void *v_cache, const int32_t *block_tables,
@@ -1716,30 +1617,28 @@ extern "C" pa_status pa_decode_append(void *out, const void *q, const void *k_ne
                                       int num_blocks, float scale, pa_dtype dtype,
                                       void *workspace, size_t workspace_bytes,
                                       int partition_tokens, void *stream) {
-  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
-      block_size <= 0 || num_blocks <= 0)
-    return PA_ERR_INVALID;
-  if (num_seqs == 0) return PA_OK;
-  if (!k_new || !v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16) ||
-      !aligned(slot_mapping, 8))
-    return PA_ERR_INVALID;
-  const int group = num_q_heads / num_kv_heads;
-  if (uses_stream_kernel(group, block_size, num_blocks, num_kv_heads)) {
-    const FusedWrite fw{k_new, v_new, slot_mapping, k_cache, v_cache};
-    return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                       max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
-                       block_size, num_blocks, scale, dtype, workspace, workspace_bytes,
-                       partition_tokens, stream, &fw);
-  }
-  // other shapes: the write kernel, then the decode
-  const pa_status st = pa_reshape_and_cache(k_new, v_new, slot_mapping, num_seqs, k_cache,
-                                            v_cache, num_blocks, num_kv_heads, block_size,
-                                            head_dim, dtype, stream);
-  if (st != PA_OK) return st;
-  return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
-                     max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                     num_blocks, scale, dtype, workspace, workspace_bytes, partition_tokens,
-                     stream, nullptr);
+  return decode_append_impl(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,
+                            max_blocks_per_seq, context_lens, max_context_len, num_seqs,
+                            num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                            dtype, workspace, workspace_bytes, partition_tokens, stream, 0);
+}
+
+extern "C" pa_status pa_decode_append_window(
+    void *out, const void *q, const void *k_new, const void *v_new, const int64_t *slot_mapping,
+    void *k_cache, void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+    const int32_t *context_lens, int max_context_len, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale, int window,
+    pa_dtype dtype, void *workspace, size_t workspace_bytes, int partition_tokens, void *stream) {
+  if (window <= 0) return PA_ERR_INVALID;
+  return decode_append_impl(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,
+                            max_blocks_per_seq, context_lens, max_context_len, num_seqs,
+                            num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                            dtype, workspace, workspace_bytes, partition_tokens, stream, window);
+}
+
+bool pa_internal_pool_tensor_map(CUtensorMap *map, const void *base, long long rows, int head_dim,
+                                 int box_rows, pa_dtype dtype) {
+  return pool_tensor_map(map, base, rows, head_dim, box_rows, dtype);
 }
 
 pa_status pa_internal_decode_status(cudaStream_t stream, int32_t *code) {
@@ -1758,11 +1657,13 @@ pa_status pa_internal_decode_status(cudaStream_t stream, int32_t *code) {
 
 extern "C" pa_status pa_device_status(void *stream, int32_t *code) {
   if (!code) return PA_ERR_INVALID;
-  int32_t a = 0, b = 0;
+  int32_t a = 0, b = 0, c = 0;
   pa_status st = pa_internal_cache_ops_status(static_cast<cudaStream_t>(stream), &a);
   if (st != PA_OK) return st;
   st = pa_internal_decode_status(static_cast<cudaStream_t>(stream), &b);
   if (st != PA_OK) return st;
-  *code = a | b;
+  st = pa_internal_prefill_status(static_cast<cudaStream_t>(stream), &c);
+  if (st != PA_OK) return st;
+  *code = a | b | c;
   return PA_OK;
 }

@@ -1,0 +1,505 @@
+// pa_prefill.cu -- paged attention for several query tokens per sequence
+// (prefill, or one chunk of a chunked prefill) on sm_100a.
+//
+// What it computes ("PagedAttention 核心思想解析", section 2.2: the rows of Q
+// are cut into blocks, each block is scored against the sequence's K/V blocks
+// found through the block table, and the partial results are merged by
+// position): sequence b holds n = context_lens[b] positions; its
+// m = q_start[b+1] - q_start[b] query tokens are its last m positions (their
+// K/V already written to the pool), and the token at position p attends to
+// positions [lo, p] -- lo = p + 1 - window under a sliding window, else 0.
+//
+// Design:
+//  * One CTA per (q head, 64 query tokens, sequence); the q heads of one kv
+//    head are neighbours in the grid, so the CTAs sharing a K/V tile run
+//    together and all but the first read it from L2. Tiles with the most keys
+//    (the last query tiles of a sequence) are launched first.
+//  * A producer warp streams the CTA's key tiles (64 keys) into a 2-stage ring
+//    with 2-D TMA copies of each (block, kv head) piece (128-byte swizzle; the
+//    same pool tensor maps as decode), guarded by full / empty mbarriers.
+//  * Four consumer warps own 16 query rows each. Per tile: S = Q K^T with
+//    mma.sync m16n8k16 (Q fragments stay in registers for the whole loop, K
+//    from ldmatrix on the swizzled panels), the causal / window mask on the
+//    tiles that need it, online softmax in the log2 domain, and O += P V with
+//    P rebuilt in registers as A fragments and V from ldmatrix.trans. The
+//    running sum uses the rounded weights, so the result is an exact weighted
+//    average of V. Rows of V past the sequence's last position (never written,
+//    may hold anything) are zeroed in shared memory before the product.
+//  * Every wait is bounded; block ids and lengths are range-checked and a bad
+//    one is skipped and reported in the device error word, never accessed.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "pa.h"
+#include "pa_internal.h"
+#include "pa_ptx.cuh"
+
+namespace {
+
+__device__ int g_prefill_error;
+
+constexpr int kQTile = 64;       // query tokens per CTA
+constexpr int kKTile = 64;       // keys per stage
+constexpr int kWarps = 4;        // consumer warps, 16 query rows each
+constexpr int kThreads = (kWarps + 1) * 32;
+constexpr int kStages = 2;
+constexpr int kPanelBytes = 64 * 128;  // 64 rows x 64 columns of 2 bytes, 128-byte swizzled
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+struct PrefillParams {
+  void *out;                  // [T][Hq][D]
+  const void *q;              // [T][Hq][D]
+  const int32_t *block_tables;
+  const int32_t *context_lens;
+  const int32_t *q_start;     // [B + 1]
+  int max_blocks_per_seq;
+  int max_context_len;
+  int num_tokens;
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int block_size;
+  int num_blocks;
+  int window;
+  int q_tiles;                // grid.y
+  float scale_log2;
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kQBytes = kPanels * kPanelBytes;          // 64 query rows
+  static constexpr int kStageBytes = 2 * kPanels * kPanelBytes;  // K panels, then V panels
+  static constexpr int kRingOffset = kQBytes;
+  static constexpr int kBarOffset = kRingOffset + kStages * kStageBytes;
+  static constexpr int kFlagOffset = kBarOffset + 2 * kStages * 8;
+  static constexpr int kBytes = 1024 + kFlagOffset + 16;  // + slack to align to 1 KB
+};
+
+__device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      atomicOr(&g_prefill_error, PA_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// First position the token at position p attends to.
+__device__ __forceinline__ int first_key(int p, int window) {
+  return window > 0 && p + 1 > window ? p + 1 - window : 0;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
+    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+    const PrefillParams p) {
+  using L = Layout<D>;
+  constexpr int KSTEPS = D / 16;  // k-steps of Q K^T
+  constexpr int NT_O = D / 8;     // n-tiles of the output row block
+
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + L::kBarOffset);
+  uint64_t *empty_bar = full_bar + kStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kFlagOffset);
+  const uint32_t qsm = smem_u32(smem);
+  const uint32_t ring = smem_u32(smem + L::kRingOffset);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x;
+  const int qt = p.q_tiles - 1 - (int)blockIdx.y;  // the longest tiles first
+  const int b = blockIdx.z;
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const int kvh = h / G;
+  const int bs = p.block_size;
+  const int cap = p.max_blocks_per_seq * bs;
+
+  // ---- this CTA's query rows and key range (the same in every thread)
+  int n = __ldg(p.context_lens + b);
+  const int qs0 = __ldg(p.q_start + b), qs1 = __ldg(p.q_start + b + 1);
+  int m = qs1 - qs0;
+  bool bad = false;
+  if (n < 0 || n > cap || n > p.max_context_len) {
+    bad = true;
+    n = n < 0 ? 0 : min(min(n, cap), p.max_context_len);
+  }
+  if (m < 0 || m > n || qs0 < 0 || qs1 > p.num_tokens) {
+    bad = true;
+    m = 0;
+  }
+  if (bad && tid == 0 && h == 0 && blockIdx.y == 0)
+    atomicOr(&g_prefill_error, PA_DEVERR_CONTEXT_LEN);
+  const int q0 = qt * kQTile;
+  if (q0 >= m) return;  // no query rows here (uniform)
+  const int rows = min(kQTile, m - q0);
+  const int p_first = n - m + q0;       // position of the first query row
+  const int p_last = p_first + rows - 1;
+  const int align = bs < kKTile ? bs : kKTile;
+  const int k_base = first_key(p_first, p.window) & ~(align - 1);  // block / 64-key aligned
+  const int ntiles = (p_last + 1 - k_base + kKTile - 1) / kKTile;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kWarps);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kWarps) {
+    // ======================================================================== producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)));
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
+    }
+    const int32_t *row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+    const int box_rows = align;
+    const uint32_t box_bytes = 2u * L::kPanels * box_rows * 128u;  // K and V
+    int issued = 0;
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % kStages;
+      if (i >= kStages && !wait_bounded(&empty_bar[s], ((i / kStages) & 1) ^ 1, abort_flag))
+        break;
+      __syncwarp();
+      const int t0 = k_base + i * kKTile;
+      const int t_end = min(t0 + kKTile, n);  // keys past n are never read
+      // boxes of this tile: whole blocks (block_size <= 64) or one 64-key slice
+      const int nbox = t_end > t0 ? (bs <= kKTile ? (t_end - 1) / bs - t0 / bs + 1 : 1) : 0;
+      int phys = -1;
+      bool ok = false;
+      if (lane < nbox) {
+        const int lb = t0 / bs + lane;
+        phys = lb < p.max_blocks_per_seq ? __ldg(row + lb) : -1;
+        ok = phys >= 0 && phys < p.num_blocks;
+        if (!ok) atomicOr(&g_prefill_error, PA_DEVERR_BLOCK_ID);
+      }
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes);
+      __syncwarp();
+      // one lane per (box, operand, panel): lane = box * 2 * kPanels + which * kPanels + pn
+      const int per_box = 2 * L::kPanels;
+      const int box = lane / per_box;
+      const int which = (lane / L::kPanels) % 2;
+      const int pn = lane % L::kPanels;
+      const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
+      if (box < nbox && ((okmask >> box) & 1u)) {
+        const int r0 = bs > kKTile ? t0 % bs : 0;
+        const int srow = bs > kKTile ? 0 : box * bs;
+        const int y = (box_phys * p.num_kv_heads + kvh) * bs + r0;
+        tma_load_2d(ring + s * L::kStageBytes + (which * L::kPanels + pn) * kPanelBytes + srow * 128,
+                    which ? &tmap_v : &tmap_k, pn * 64, y, &full_bar[s]);
+      }
+      issued = i + 1;
+    }
+    // do not leave while copies may still land in this CTA's shared memory
+    if (lane == 0) {
+      for (int i = max(0, issued - kStages); i < issued; ++i) {
+        const int s = i % kStages;
+        const unsigned long long t_start = global_ns();
+        while (!mbar_try_wait(&full_bar[s], (i / kStages) & 1)) {
+          if (global_ns() - t_start > kWaitLimitNs) {
+            atomicOr(&g_prefill_error, PA_DEVERR_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+    return;
+  }
+
+  // ========================================================================== consumers
+  const int g = lane >> 2, t = lane & 3;
+  const int wrow = warp * 16;
+  // positions of this thread's two query rows (rows past the chunk are clamped
+  // to the last position: computed, never stored)
+  const int pr0 = min(p_first + wrow + g, n - 1);
+  const int pr1 = min(p_first + wrow + g + 8, n - 1);
+  const int lo0 = first_key(pr0, p.window), lo1 = first_key(pr1, p.window);
+  const int p_warp_first = p_first + wrow;
+  const int p_warp_last = min(p_first + wrow + 15, n - 1);
+
+  // ---- Q rows of this warp -> swizzled shared memory -> A fragments (kept)
+  {
+    const T *qg = static_cast<const T *>(p.q);
+    constexpr int kChunks = D / 8;  // 16-byte chunks per row
+    for (int c = lane; c < 16 * kChunks; c += 32) {
+      const int r = c / kChunks, ch = c % kChunks;
+      const int qrow = wrow + r;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (qrow < rows)
+        v = __ldg(reinterpret_cast<const uint4 *>(
+                      qg + ((size_t)(qs0 + q0 + qrow) * p.num_q_heads + h) * D) + ch);
+      *reinterpret_cast<uint4 *>(smem + (ch / 8) * kPanelBytes + qrow * 128 +
+                                 (((ch % 8) ^ (qrow & 7)) << 4)) = v;
+    }
+    __syncwarp();
+  }
+  uint32_t qa[KSTEPS][4];
+  {
+    const int r = wrow + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk)
+      ldsm_x4(swz(qsm + (kk / 4) * kPanelBytes, r, 2 * (kk % 4) + (lane >> 4)), qa[kk]);
+  }
+
+  float o[NT_O][4];
+#pragma unroll
+  for (int x = 0; x < NT_O; ++x) o[x][0] = o[x][1] = o[x][2] = o[x][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  const int kb_row = (lane & 7) + 8 * (lane >> 4);         // K ldmatrix: key row in 16
+  const int kb_chk = (lane >> 3) & 1;                      //             d chunk in pair
+  const int vb_row = (lane & 7) + 8 * ((lane >> 3) & 1);   // V ldmatrix.trans: key row
+  const int vb_chk = lane >> 4;                            //                   d chunk
+
+  for (int i = 0; i < ntiles; ++i) {
+    const int s = i % kStages;
+    const bool landed = wait_bounded(&full_bar[s], (i / kStages) & 1, abort_flag);
+    __syncwarp();
+    const int t0 = k_base + i * kKTile;
+    const uint32_t kst = ring + s * L::kStageBytes;
+    const uint32_t vst = kst + L::kPanels * kPanelBytes;
+    // rows of V outside every row's keys -- past the sequence's end (never
+    // loaded, or unwritten slots) or before the first row's window (released
+    // slots) -- may hold anything: zero them before any warp multiplies by them
+    const int nvalid = min(kKTile, n - t0);
+    const int nskip = max(0, first_key(p_first, p.window) - t0);
+    if (nvalid < kKTile || nskip > 0) {
+      unsigned char *vz = smem + L::kRingOffset + s * L::kStageBytes + L::kPanels * kPanelBytes;
+      for (int r = warp * 4 + (lane >> 3); r < kKTile; r += 16) {
+        if (r >= nskip && r < nvalid) continue;
+#pragma unroll
+        for (int pn = 0; pn < L::kPanels; ++pn)
+          *reinterpret_cast<uint4 *>(vz + pn * kPanelBytes + r * 128 + (lane & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+    }
+    // a warp whose rows all precede this tile, or whose windows all start after
+    // it, has nothing to add
+    if (landed && t0 <= p_warp_last && t0 + kKTile > first_key(p_warp_first, p.window)) {
+      // ---- S = Q K^T: 16 rows x 64 keys (8 n-tiles of 8 keys)
+      float sc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < KSTEPS; ++kk) {
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {  // pairs of n-tiles
+          uint32_t kb[4];
+          ldsm_x4(swz(kst + (kk / 4) * kPanelBytes, np * 16 + kb_row, 2 * (kk % 4) + kb_chk), kb);
+          Mma<T>::run(sc[2 * np], qa[kk], kb[0], kb[1]);
+          Mma<T>::run(sc[2 * np + 1], qa[kk], kb[2], kb[3]);
+        }
+      }
+      // ---- scale, mask, online softmax (log2 domain)
+      const bool need_mask = t0 + kKTile - 1 > p_warp_first ||
+                             (p.window > 0 && t0 < first_key(p_warp_last, p.window));
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int kp = t0 + nt * 8 + 2 * t + e;
+          float a = sc[nt][e] * p.scale_log2, c = sc[nt][2 + e] * p.scale_log2;
+          if (need_mask) {
+            a = (kp <= pr0 && kp >= lo0) ? a : -INFINITY;
+            c = (kp <= pr1 && kp >= lo1) ? c : -INFINITY;
+          }
+          sc[nt][e] = a;
+          sc[nt][2 + e] = c;
+          mx0 = fmaxf(mx0, a);
+          mx1 = fmaxf(mx1, c);
+        }
+      }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
+      const float al0 = m0 == -INFINITY ? 0.f : exp2f(m0 - b0);
+      const float al1 = m1 == -INFINITY ? 0.f : exp2f(m1 - b1);
+      m0 = mn0;
+      m1 = mn1;
+      // P as A fragments of the 4 k-steps of P V (keys 16kk .. 16kk + 15)
+      uint32_t pa[4][4];
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int nt = 2 * kk + half;
+          float r00, r01, r10, r11;
+          pa[kk][half * 2] = Mma<T>::pack(exp2f(sc[nt][0] - b0), exp2f(sc[nt][1] - b0), r00, r01);
+          pa[kk][half * 2 + 1] =
+              Mma<T>::pack(exp2f(sc[nt][2] - b1), exp2f(sc[nt][3] - b1), r10, r11);
+          rs0 += r00 + r01;
+          rs1 += r10 + r11;
+        }
+      }
+      l0 = l0 * al0 + rs0;
+      l1 = l1 * al1 + rs1;
+#pragma unroll
+      for (int x = 0; x < NT_O; ++x) {
+        o[x][0] *= al0;
+        o[x][1] *= al0;
+        o[x][2] *= al1;
+        o[x][3] *= al1;
+      }
+      // ---- O += P V: for each pair of 8-wide d n-tiles, 4 k-steps of 16 keys
+#pragma unroll
+      for (int x = 0; x < NT_O / 2; ++x) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint32_t vb[4];
+          ldsm_x4_trans(swz(vst + (x / 4) * kPanelBytes, kk * 16 + vb_row, 2 * (x % 4) + vb_chk), vb);
+          Mma<T>::run(o[2 * x], pa[kk], vb[0], vb[1]);
+          Mma<T>::run(o[2 * x + 1], pa[kk], vb[2], vb[3]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[s]);
+  }
+
+  // ---- normalise, stage the warp's rows in shared memory, store them
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+  // the Q staging rows of this warp are free again (its fragments are in registers)
+#pragma unroll
+  for (int x = 0; x < NT_O; ++x) {
+    const int col = x * 8 + 2 * t;  // element column; chunk col / 8, offset (col % 8) * 2
+    float r;
+    const uint32_t w0 = Mma<T>::pack(o[x][0] * inv0, o[x][1] * inv0, r, r);
+    const uint32_t w1 = Mma<T>::pack(o[x][2] * inv1, o[x][3] * inv1, r, r);
+    const int r0 = wrow + g, r1 = wrow + g + 8;
+    *reinterpret_cast<uint32_t *>(smem + (col / 64) * kPanelBytes + r0 * 128 +
+                                  ((((col % 64) / 8) ^ (r0 & 7)) << 4) + (col % 8) * 2) = w0;
+    *reinterpret_cast<uint32_t *>(smem + (col / 64) * kPanelBytes + r1 * 128 +
+                                  ((((col % 64) / 8) ^ (r1 & 7)) << 4) + (col % 8) * 2) = w1;
+  }
+  __syncwarp();
+  {
+    T *og = static_cast<T *>(p.out);
+    constexpr int kChunks = D / 8;
+    for (int c = lane; c < 16 * kChunks; c += 32) {
+      const int r = c / kChunks, ch = c % kChunks;
+      const int qrow = wrow + r;
+      if (qrow >= rows) continue;
+      const uint4 v = *reinterpret_cast<const uint4 *>(smem + (ch / 8) * kPanelBytes + qrow * 128 +
+                                                       (((ch % 8) ^ (qrow & 7)) << 4));
+      *(reinterpret_cast<uint4 *>(og + ((size_t)(qs0 + q0 + qrow) * p.num_q_heads + h) * D) + ch) = v;
+    }
+  }
+}
+
+template <typename T, int D>
+pa_status launch(const PrefillParams &prm, const void *k_cache, const void *v_cache,
+                 pa_dtype dtype, cudaStream_t stream) {
+  using L = Layout<D>;
+  CUtensorMap tk, tv;
+  const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
+  const int box_rows = prm.block_size < kKTile ? prm.block_size : kKTile;
+  if (!pa_internal_pool_tensor_map(&tk, k_cache, rows, D, box_rows, dtype) ||
+      !pa_internal_pool_tensor_map(&tv, v_cache, rows, D, box_rows, dtype))
+    return PA_ERR_CUDA;
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(pa_prefill_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             L::kBytes) != cudaSuccess)
+      return PA_ERR_CUDA;
+    configured[dev] = true;
+  }
+  dim3 grid((unsigned)prm.num_q_heads, (unsigned)prm.q_tiles, (unsigned)prm.num_seqs);
+  pa_prefill_kernel<T, D><<<grid, kThreads, L::kBytes, stream>>>(tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) & (a - 1)) == 0; }
+
+}  // namespace
+
+extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *context_lens, const int32_t *q_start,
+                                int num_seqs, int num_tokens, int max_q_len,
+                                int max_context_len, int num_q_heads, int num_kv_heads,
+                                int head_dim, int block_size, int num_blocks, float scale,
+                                int window, pa_dtype dtype, void *stream) {
+  if (num_seqs < 0 || num_tokens < 0 || max_q_len < 0 || max_context_len < 0 || window < 0 ||
+      num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads || block_size <= 0 ||
+      num_blocks <= 0 || max_blocks_per_seq <= 0 || (dtype != PA_F16 && dtype != PA_BF16))
+    return PA_ERR_INVALID;
+  if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+  // TMA boxes are whole blocks or 64-key slices of one
+  if (block_size < 8 || (block_size & (block_size - 1))) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || num_tokens == 0 || max_q_len == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !q_start)
+    return PA_ERR_INVALID;
+  if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(q_start, 4))
+    return PA_ERR_INVALID;
+  const long long rows = (long long)num_blocks * num_kv_heads * block_size;
+  if (rows > INT32_MAX || num_seqs > 65535 || num_q_heads > 65535) return PA_ERR_INVALID;
+  const int q_tiles = (max_q_len + kQTile - 1) / kQTile;
+  if (q_tiles > 65535) return PA_ERR_INVALID;
+  PrefillParams prm;
+  prm.out = out;
+  prm.q = q;
+  prm.block_tables = block_tables;
+  prm.context_lens = context_lens;
+  prm.q_start = q_start;
+  prm.max_blocks_per_seq = max_blocks_per_seq;
+  prm.max_context_len = max_context_len;
+  prm.num_tokens = num_tokens;
+  prm.num_seqs = num_seqs;
+  prm.num_q_heads = num_q_heads;
+  prm.num_kv_heads = num_kv_heads;
+  prm.block_size = block_size;
+  prm.num_blocks = num_blocks;
+  prm.window = window;
+  prm.q_tiles = q_tiles;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PA_BF16)
+    return head_dim == 128 ? launch<__nv_bfloat16, 128>(prm, k_cache, v_cache, dtype, st)
+                           : launch<__nv_bfloat16, 64>(prm, k_cache, v_cache, dtype, st);
+  return head_dim == 128 ? launch<__half, 128>(prm, k_cache, v_cache, dtype, st)
+                         : launch<__half, 64>(prm, k_cache, v_cache, dtype, st);
+}
+
+// Read and clear this file's error word (stream-ordered; synchronises the stream).
+pa_status pa_internal_prefill_status(cudaStream_t stream, int32_t *code) {
+  int value = 0;
+  const int zero = 0;
+  if (cudaMemcpyFromSymbolAsync(&value, g_prefill_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                stream) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaMemcpyToSymbolAsync(g_prefill_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice,
+                              stream) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return PA_ERR_CUDA;
+  *code = value;
+  return PA_OK;
+}

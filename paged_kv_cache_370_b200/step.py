@@ -22,10 +22,13 @@ from . import abi
 class DecodeStep:
     def __init__(self, *, k_cache, v_cache, q, k_new, v_new, slot_mapping, block_tables,
                  context_lens, max_context_len: int, scale: float, partition_tokens: int = 0,
-                 copy_pairs=None, out=None, fused: bool = False):
+                 copy_pairs=None, out=None, fused: bool = False, window: int = 0):
         """``fused``: write the new tokens inside the decode (pa_decode_append);
-        k_new/v_new then hold one token per sequence, at position len - 1."""
+        k_new/v_new then hold one token per sequence, at position len - 1.
+        ``window`` > 0: attend to each sequence's last ``window`` positions only
+        (pa_decode_window / pa_decode_append_window)."""
         self.fused = fused
+        self.window = int(window)
         self.k_cache, self.v_cache = k_cache, v_cache
         self.q, self.k_new, self.v_new = q, k_new, v_new
         self.slot_mapping = slot_mapping
@@ -49,6 +52,12 @@ class DecodeStep:
         self.append_launches = abi.pa_decode_append_launches(B, hq, hkv, d, bs, nb,
                                                              self.max_context_len,
                                                              self.partition_tokens)
+        if self.window > 0:  # the partition kernel (and merge), after a separate write
+            self.decode_launches = abi.pa_decode_window_launches(B, hq, hkv, d,
+                                                                 self.max_context_len,
+                                                                 self.window,
+                                                                 self.partition_tokens)
+            self.append_launches = 1 + self.decode_launches
         self.partition = self.partition_tokens or abi.pa_decode_default_partition(
             B, hkv, self.max_context_len)
 
@@ -68,11 +77,23 @@ class DecodeStep:
                                  self.v_cache, stream)
 
     def attend(self, stream=None):
+        if self.window > 0:
+            abi.pa_decode_window(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
+                                 self.context_lens, self.max_context_len, self.scale, self.window,
+                                 self.workspace, self.partition_tokens, stream)
+            return
         abi.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
                       self.context_lens, self.max_context_len, self.scale, self.workspace,
                       self.partition_tokens, stream)
 
     def append(self, stream=None):
+        if self.window > 0:
+            abi.pa_decode_append_window(self.out, self.q, self.k_new, self.v_new,
+                                        self.slot_mapping, self.k_cache, self.v_cache,
+                                        self.block_tables, self.context_lens,
+                                        self.max_context_len, self.scale, self.window,
+                                        self.workspace, self.partition_tokens, stream)
+            return
         abi.pa_decode_append(self.out, self.q, self.k_new, self.v_new, self.slot_mapping,
                              self.k_cache, self.v_cache, self.block_tables, self.context_lens,
                              self.max_context_len, self.scale, self.workspace,
@@ -99,7 +120,7 @@ class HostDecodeStep:
 
     def __init__(self, *, k_cache, v_cache, q, k_new, v_new, slot_mapping, block_tables,
                  context_lens, max_context_len: int, scale: float, partition_tokens: int = 0,
-                 copy_pairs=None, fused: bool = False):
+                 copy_pairs=None, fused: bool = False, window: int = 0):
         dev = k_cache.device
         parts = {"q": q, "k_new": k_new, "v_new": v_new, "slot_mapping": slot_mapping,
                  "block_tables": block_tables, "context_lens": context_lens}
@@ -124,7 +145,7 @@ class HostDecodeStep:
                                context_lens=views["context_lens"],
                                max_context_len=max_context_len, scale=scale,
                                partition_tokens=partition_tokens,
-                               copy_pairs=views.get("copy_pairs"), fused=fused)
+                               copy_pairs=views.get("copy_pairs"), fused=fused, window=window)
         self.h_out = torch.empty(tuple(q.shape), dtype=q.dtype).pin_memory()
 
     @property

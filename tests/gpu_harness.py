@@ -41,7 +41,7 @@ class GpuBatch:
     last token and decodes."""
 
     def __init__(self, batch, partition_tokens: int = 0, device="cuda", tables=None,
-                 fused: bool = False):
+                 fused: bool = False, window: int = 0, step_tables=None):
         self.batch = batch
         bs, dt = batch.block_size, batch.dtype
         shape = (batch.num_blocks, batch.num_kv_heads, bs, batch.head_dim)
@@ -75,10 +75,11 @@ class GpuBatch:
         self.step = DecodeStep(
             k_cache=self.k_cache, v_cache=self.v_cache, q=to_dev(batch.q, dt, device),
             k_new=new_k, v_new=new_v, slot_mapping=torch.from_numpy(new_slots).to(device),
-            block_tables=torch.from_numpy(np.ascontiguousarray(self.tables_np)).to(device),
+            block_tables=torch.from_numpy(np.ascontiguousarray(
+                self.tables_np if step_tables is None else step_tables)).to(device),
             context_lens=torch.from_numpy(batch.context_lens).to(device),
             max_context_len=max(batch.max_context_len, 1), scale=float(batch.scale),
-            partition_tokens=partition_tokens, fused=fused)
+            partition_tokens=partition_tokens, fused=fused, window=window)
 
     def run(self):
         out = self.step.run()

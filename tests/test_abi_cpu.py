@@ -317,6 +317,19 @@ def test_decode_rejects_bad_arguments_before_launch():
     assert L.pa_copy_blocks(None, None, None, 0, 8, 4, 16, 128, 1, None) == 0
     assert L.pa_copy_blocks(None, None, None, 2, 8, 4, 16, 0, 1, None) == -1
 
+    def call_window(w, **kw):
+        a = dict(args, hq=8, B=0, **kw)
+        return L.pa_decode_window(a["out"], a["q"], a["k"], a["v"], a["bt"], a["mbps"], a["cl"],
+                                  a["maxlen"], a["B"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"],
+                                  a["scale"], w, a["dt"], a["ws"], a["wsb"], a["pt"], a["st"])
+
+    assert call_window(0) == abi.PA_ERR_INVALID     # a window holds at least one position
+    assert call_window(-3) == abi.PA_ERR_INVALID
+    assert call_window(5) == abi.PA_OK              # empty batch: nothing to do
+    # swap: a null space or unaligned pools are refused before any launch
+    assert L.pa_swap_out(None, None, None, 8, None, 0, None) == abi.PA_ERR_INVALID
+    assert L.pa_swap_in(None, None, None, 8, None, 0, None) == abi.PA_ERR_INVALID
+
 
 def test_workspace_size():
     # a fixed 64 KiB counter region, then room for the larger of the two kernels' scratch
