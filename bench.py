@@ -63,7 +63,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama8b",
-                    choices=["llama8b", "long_skew", "mixed", "shared_prompt", "swap"])
+                    choices=["llama8b", "long_skew", "mixed", "shared_prompt", "swap", "prefill"])
     ap.add_argument("--block-size", type=int, default=16, help="block size of the mixed workload")
     ap.add_argument("--variants", type=int, default=4, help="batches rotated (llama8b)")
     ap.add_argument("--partition-tokens", type=int, default=0)
@@ -665,6 +665,121 @@ def run_swap(args):
             "gpu_launches": 2 * args.steps}
 
 
+# ---------------------------------------------------------------------------------- prefill
+def prefill_flops(batch, window=0) -> float:
+    """Algorithmic FLOPs of causal paged prefill attention: for every (query
+    token, q head), 2*D for its scores and 2*D for its weighted V per key it
+    attends to (positions [lo, p])."""
+    qs = batch.meta["q_start"]
+    keys = 0
+    for b in range(batch.num_seqs):
+        n, m = int(batch.context_lens[b]), int(qs[b + 1] - qs[b])
+        p = np.arange(n - m, n, dtype=np.int64)
+        lo = np.maximum(p + 1 - window, 0) if window > 0 else np.zeros_like(p)
+        keys += int((p + 1 - lo).sum())
+    return 4.0 * batch.head_dim * batch.num_q_heads * keys
+
+
+def run_prefill(args):
+    """Chunked prefill on the Llama-3.1-8B shapes (16 sequences x 512 new tokens
+    after up to 1,536 history tokens): one step = the chunk's K/V write
+    (pa_reshape_and_cache) + pa_prefill, graph-replayed over 4 rotating batches."""
+    import torch
+    from paged_kv_cache_370_b200 import abi
+    dev = torch.device("cuda", 0)
+    nv, per = 4, 16384  # 4 batches, each drawing distinct ids from its own quarter of the pool
+    batches = [synth.llama8b_prefill(seed=synth.SEED_BASE + 7 + 10 * v, num_blocks=per)
+               for v in range(nv)]
+    b0 = batches[0]
+    shape = (nv * per, b0.num_kv_heads, b0.block_size, b0.head_dim)
+    kc = torch.zeros(shape, dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    steps = []
+    for v, b in enumerate(batches):
+        tables = (b.block_tables + v * per).astype(np.int32)
+        b.block_tables = tables
+        slots = abi.pa_slot_mapping(tables, b.context_lens, b.block_size)
+        qs = b.meta["q_start"]
+        new_rows = np.concatenate([np.arange(b.seq_start[i + 1] - (qs[i + 1] - qs[i]),
+                                             b.seq_start[i + 1]) for i in range(b.num_seqs)])
+        hist = np.setdiff1d(np.arange(b.total_tokens), new_rows)
+        k_all, v_all = to_dev(b.k, "bf16", torch, dev), to_dev(b.v, "bf16", torch, dev)
+        abi.pa_reshape_and_cache(k_all[torch.from_numpy(hist).to(dev)].contiguous(),
+                                 v_all[torch.from_numpy(hist).to(dev)].contiguous(),
+                                 torch.from_numpy(slots[hist]).to(dev), kc, vc)
+        nidx = torch.from_numpy(new_rows).to(dev)
+        st = {"k_new": k_all[nidx].contiguous(), "v_new": v_all[nidx].contiguous(),
+              "slots": torch.from_numpy(slots[new_rows]).to(dev),
+              "q": to_dev(b.q, "bf16", torch, dev), "tables": torch.from_numpy(tables).to(dev),
+              "lens": torch.from_numpy(b.context_lens).to(dev),
+              "q_start": torch.from_numpy(qs.astype(np.int32)).to(dev),
+              "max_q": int(b.meta["q_lens"].max()), "max_len": b.max_context_len,
+              "scale": float(b.scale), "flops": prefill_flops(b, args.window)}
+        st["out"] = torch.empty_like(st["q"])
+        steps.append(st)
+        del k_all, v_all
+
+    def write(st):
+        abi.pa_reshape_and_cache(st["k_new"], st["v_new"], st["slots"], kc, vc)
+
+    def attend(st):
+        abi.pa_prefill(st["out"], st["q"], kc, vc, st["tables"], st["lens"], st["q_start"],
+                       st["max_q"], st["max_len"], st["scale"], args.window)
+
+    g_round = capture(lambda: [f(st) for st in steps for f in (write, attend)], torch)
+    g_att = capture(lambda: [attend(st) for st in steps], torch)
+    for _ in range(max(3, args.warmup // 10)):
+        g_round.replay()
+    torch.cuda.synchronize()
+    rounds = max(1, args.steps // len(steps))
+    clocks = ClockSampler(os.environ.get("PA_BUS_ID"))
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    e0.record()
+    for _ in range(rounds):
+        g_round.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    step_ms = e0.elapsed_time(e1) / (rounds * len(steps))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record()
+    for _ in range(rounds):
+        g_att.replay()
+    a1.record()
+    torch.cuda.synchronize()
+    clocks.stop()
+    att_ms = a0.elapsed_time(a1) / (rounds * len(steps))
+    flops = float(np.mean([st["flops"] for st in steps]))
+    peak = 1394.0
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = float(json.load(f)["bf16_tflops_sustained"])
+        kind = "measured sustained bf16 (cuBLAS, seconds-long loop)"
+    except (OSError, KeyError, ValueError):
+        kind = "fallback"
+    tflops = flops / (att_ms * 1e-3) / 1e12
+    tokens = float(np.mean([int(st["q"].shape[0]) for st in steps]))
+    code = abi.pa_device_status()
+    return {"metric": "paged prefill attention TFLOP/s (causal, bf16 in, fp32 accumulate)",
+            "value": round(flops / (step_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": rounds * len(steps), "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "Llama-3.1-8B-shaped chunked prefill", "num_seqs": 16,
+                       "chunk_tokens": 512, "history": "uniform [0, 1536]",
+                       "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128, "block_size": 16,
+                       "window": args.window, "batches_rotated": len(steps)},
+            "query_tokens_per_s": round(tokens / (step_ms * 1e-3), 1),
+            "roofline": {"bound": "tensor", "kernel": "pa_prefill", "achieved": round(tflops, 2),
+                         "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                         "peak_kind": kind, "flops_per_launch": flops,
+                         "avg_launch_ms": round(att_ms, 5), "traffic": None},
+            "gpu_launches": 2 * rounds * len(steps), "clocks": clocks.summary(t0, t1),
+            "device_error_word": code}
+
+
 # ------------------------------------------------------------------------------------- main
 def main():
     args = parse_args()
@@ -674,9 +789,10 @@ def main():
             return 0
         print(json.dumps(run_reference(args, rank, world)), flush=True)
         return 0
-    if args.workload == "swap":
+    if args.workload in ("swap", "prefill"):
         if rank == 0:
-            print(json.dumps(run_swap(args)), flush=True)
+            fn = run_swap if args.workload == "swap" else run_prefill
+            print(json.dumps(fn(args)), flush=True)
         return 0
     dist = None
     if world > 1:
