@@ -687,7 +687,8 @@ def run_prefill(args):
     import torch
     from paged_kv_cache_370_b200 import abi
     dev = torch.device("cuda", 0)
-    nv, per = 4, 16384  # 4 batches, each drawing distinct ids from its own quarter of the pool
+    # 4 batches, each drawing distinct ids from its own quarter of the pool
+    nv, per = 4, max(2048, args.pool_blocks // 4)
     batches = [synth.llama8b_prefill(seed=synth.SEED_BASE + 7 + 10 * v, num_blocks=per)
                for v in range(nv)]
     b0 = batches[0]

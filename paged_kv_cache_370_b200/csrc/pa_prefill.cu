@@ -35,10 +35,17 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <type_traits>
 
 #include "pa.h"
 #include "pa_internal.h"
 #include "pa_ptx.cuh"
+
+// Which kernel pa_prefill runs: 1 = tcgen05 (tensor memory accumulators), 0 =
+// mma.sync (register accumulators).
+#ifndef PA_PREFILL_TCGEN05
+#define PA_PREFILL_TCGEN05 1
+#endif
 
 namespace {
 
@@ -412,6 +419,347 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
   }
 }
 
+// ============================================================ tcgen05 kernel (5th-gen tensor cores)
+// Same computation, one CTA per (q head, 128 query tokens, sequence), with the
+// two products on tcgen05.mma (M = 128 query rows, one elected issuing thread)
+// and both accumulators in tensor memory:
+//   warp 0      stages 64-key K/V tiles with TMA into a 3-stage ring (as above);
+//   warp 1      allocates TMEM; its lane 0 issues S_j = Q K_j^T (TMEM, double
+//               buffered) and, one tile behind, O += P_{j-1} V_{j-1} (TMEM), and
+//               commits each group to an mbarrier;
+//   warps 2-3   copy the Q tile into shared memory (128-byte swizzled, K-major);
+//   warps 4-7   one thread per query row: read its S row from TMEM, mask, online
+//               softmax in the log2 domain, write its P row (bf16 / fp16,
+//               swizzled) to shared memory for the next product; O is rescaled in
+//               TMEM only when a row's max grows by more than 2^8 (the weights
+//               against the stale max stay <= 2^8, and the final division by the
+//               matching sum makes the result exact either way); finally O / l
+//               from TMEM to global memory.
+namespace t5 {
+
+constexpr int kM = 128;        // query rows per CTA (tcgen05 M)
+constexpr int kN = 64;         // keys per tile
+constexpr int kStages = 3;
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 256;  // S buffers at columns 0 and 64, O at 128
+constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
+
+template <int D>
+struct Lay {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kQPanel = kM * 128;                    // 128 rows x 128 bytes
+  static constexpr int kQBytes = kPanels * kQPanel;
+  static constexpr int kKVPanel = kN * 128;                   // 64 rows x 128 bytes
+  static constexpr int kStageBytes = 2 * kPanels * kKVPanel;  // K panels, then V panels
+  static constexpr int kPBytes = kM * 128;                    // 128 rows x 64 keys
+  static constexpr int kRingOff = kQBytes;
+  static constexpr int kPOff = kRingOff + kStages * kStageBytes;
+  static constexpr int kBarOff = kPOff + 2 * kPBytes;
+  // full[3] empty[3] q_ready s_full[2] s_free[2] p_full[2] pv_done[2] mma_done
+  static constexpr int kNumBars = 2 * kStages + 10;
+  static constexpr int kTmemOff = kBarOff + kNumBars * 8;
+  static constexpr int kFlagOff = kTmemOff + 8;
+  static constexpr int kBytes = 1024 + kFlagOff + 16;
+};
+
+}  // namespace t5
+
+template <typename T, int D>
+__global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
+    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
+    const PrefillParams p) {
+  using L = t5::Lay<D>;
+  constexpr int kM = t5::kM, kN = t5::kN, NS = t5::kStages;
+  constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
+  constexpr uint32_t kIdescS = umma_idesc_f16(kFmt, 0, 0, kN, kM);  // Q (K-major) . K (K-major)
+  constexpr uint32_t kIdescO = umma_idesc_f16(kFmt, 0, 1, D, kM);   // P (K-major) . V (MN-major)
+
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+  uint64_t *full_bar = bars, *empty_bar = bars + NS, *q_ready = bars + 2 * NS;
+  uint64_t *s_full = q_ready + 1, *s_free = s_full + 2, *p_full = s_free + 2;
+  uint64_t *pv_done = p_full + 2, *mma_done = pv_done + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemOff);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
+  const uint32_t q_sm = smem_u32(smem);
+  const uint32_t ring = smem_u32(smem + L::kRingOff);
+  const uint32_t p_sm = smem_u32(smem + L::kPOff);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x;
+  const int qt = p.q_tiles - 1 - (int)blockIdx.y;  // the longest tiles first
+  const int b = blockIdx.z;
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const int kvh = h / G;
+  const int bs = p.block_size;
+  const int cap = p.max_blocks_per_seq * bs;
+
+  // ---- this CTA's query rows and key range (the same in every thread)
+  int n = __ldg(p.context_lens + b);
+  const int qs0 = __ldg(p.q_start + b), qs1 = __ldg(p.q_start + b + 1);
+  int m = qs1 - qs0;
+  bool bad = false;
+  if (n < 0 || n > cap || n > p.max_context_len) {
+    bad = true;
+    n = n < 0 ? 0 : min(min(n, cap), p.max_context_len);
+  }
+  if (m < 0 || m > n || qs0 < 0 || qs1 > p.num_tokens) {
+    bad = true;
+    m = 0;
+  }
+  if (bad && tid == 0 && h == 0 && blockIdx.y == 0)
+    atomicOr(&g_prefill_error, PA_DEVERR_CONTEXT_LEN);
+  const int q0 = qt * kM;
+  if (q0 >= m) return;  // no query rows here (uniform; before any TMEM is taken)
+  const int rows = min(kM, m - q0);
+  const int p_first = n - m + q0;
+  const int p_last = p_first + rows - 1;
+  const int align = bs < kN ? bs : kN;
+  const int k_base = first_key(p_first, p.window) & ~(align - 1);
+  const int ntiles = (p_last + 1 - k_base + kN - 1) / kN;
+
+  if (tid == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);  // one tcgen05.commit per use
+    }
+    mbar_init(q_ready, 64);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, t5::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================================================================== producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)));
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
+    }
+    const int32_t *row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+    const uint32_t box_bytes = 2u * L::kPanels * align * 128u;  // K and V of one box
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % NS;
+      if (i >= NS && !wait_bounded(&empty_bar[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
+      __syncwarp();
+      const int t0 = k_base + i * kN;
+      const int t_end = min(t0 + kN, n);
+      const int nbox = t_end > t0 ? (bs <= kN ? (t_end - 1) / bs - t0 / bs + 1 : 1) : 0;
+      int phys = -1;
+      bool ok = false;
+      if (lane < nbox) {
+        const int lb = t0 / bs + lane;
+        phys = lb < p.max_blocks_per_seq ? __ldg(row + lb) : -1;
+        ok = phys >= 0 && phys < p.num_blocks;
+        if (!ok) atomicOr(&g_prefill_error, PA_DEVERR_BLOCK_ID);
+      }
+      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      if (lane == 0) mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes);
+      __syncwarp();
+      const int box = lane / (2 * L::kPanels);
+      const int which = (lane / L::kPanels) % 2;
+      const int pn = lane % L::kPanels;
+      const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
+      if (box < nbox && ((okmask >> box) & 1u)) {
+        const int r0 = bs > kN ? t0 % bs : 0;
+        const int srow = bs > kN ? 0 : box * bs;
+        const int y = (box_phys * p.num_kv_heads + kvh) * bs + r0;
+        tma_load_2d(ring + s * L::kStageBytes + (which * L::kPanels + pn) * L::kKVPanel + srow * 128,
+                    which ? &tmap_v : &tmap_k, pn * 64, y, &full_bar[s]);
+      }
+    }
+  } else if (warp == 1) {
+    // ====================================================================== MMA issuer
+    if (lane == 0) {
+      bool go = wait_bounded(q_ready, 0, abort_flag);
+      tc_fence_after();
+      for (int j = 0; j <= ntiles && go; ++j) {
+        if (j < ntiles) {  // S_j = Q K_j^T into S buffer j % 2
+          const int st = j % NS, sb = j & 1;
+          go = wait_bounded(&full_bar[st], (j / NS) & 1, abort_flag);
+          if (go && j >= 2) go = wait_bounded(&s_free[sb], ((j - 2) / 2) & 1, abort_flag);
+          if (!go) break;
+          tc_fence_after();
+          const uint32_t kaddr = ring + st * L::kStageBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_f16(tmem + sb * kN,
+                     umma_desc_sw128(q_sm + (kk / 4) * L::kQPanel + (kk % 4) * 32, 16, 1024),
+                     umma_desc_sw128(kaddr + (kk / 4) * L::kKVPanel + (kk % 4) * 32, 16, 1024),
+                     kIdescS, kk > 0);
+          umma_commit(&s_full[sb]);
+        }
+        if (j >= 1) {  // O += P_{j-1} V_{j-1}
+          const int jp = j - 1, st = jp % NS, pb = jp & 1;
+          go = wait_bounded(&p_full[pb], (jp / 2) & 1, abort_flag);
+          if (!go) break;
+          tc_fence_after();
+          const uint32_t vaddr = ring + st * L::kStageBytes + L::kPanels * L::kKVPanel;
+#pragma unroll
+          for (int kk = 0; kk < kN / 16; ++kk)
+            umma_f16(tmem + 128,
+                     umma_desc_sw128(p_sm + pb * L::kPBytes + kk * 32, 16, 1024),
+                     umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
+                     kIdescO, jp > 0 || kk > 0);
+          umma_commit(&pv_done[pb]);
+          umma_commit(&empty_bar[st]);
+        }
+      }
+      // every product issued so far has finished before TMEM is released
+      umma_commit(mma_done);
+      wait_bounded(mma_done, 0, abort_flag);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ======================================================================= Q loaders
+    const T *qg = static_cast<const T *>(p.q);
+    constexpr int kChunks = D / 8;
+    for (int c = tid - 64; c < kM * kChunks; c += 64) {
+      const int r = c / kChunks, ch = c % kChunks;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < rows)
+        v = __ldg(reinterpret_cast<const uint4 *>(
+                      qg + ((size_t)(qs0 + q0 + r) * p.num_q_heads + h) * D) + ch);
+      *reinterpret_cast<uint4 *>(smem + (ch / 8) * L::kQPanel + r * 128 +
+                                 (((ch % 8) ^ (r & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(q_ready);
+  } else {
+    // ========================================================== softmax, one row each
+    const int r = tid - 128;                      // query row == TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)((warp - 4) * 32) << 16);
+    const int pr = min(p_first + r, n - 1);       // rows past the chunk: computed, not stored
+    const int lo = first_key(pr, p.window);
+    const int lo_first = first_key(p_first, p.window);
+    float m_ref = -INFINITY, l = 0.f;
+    for (int j = 0; j < ntiles; ++j) {
+      const int sb = j & 1, st = j % NS;
+      const int t0 = k_base + j * kN;
+      wait_bounded(&s_full[sb], (j / 2) & 1, abort_flag);
+      tc_fence_after();
+      uint32_t sv[64];
+      tmem_ld32(trow + sb * kN, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(trow + sb * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s_free[sb]);
+      float mx = -INFINITY;
+      // the mask only matters on tiles that reach past a row of this warp or
+      // start before a row's window (warp-uniform)
+      const int wr0 = min(p_first + (warp - 4) * 32, n - 1);
+      const int wr1 = min(p_first + (warp - 4) * 32 + 31, n - 1);
+      if (t0 + kN - 1 > wr0 || (p.window > 0 && t0 < first_key(wr1, p.window))) {
+#pragma unroll
+        for (int c = 0; c < kN; ++c) {
+          const int kp = t0 + c;
+          const float x = (kp <= pr && kp >= lo) ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
+          sv[c] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kN; ++c) {
+          const float x = __uint_as_float(sv[c]) * p.scale_log2;
+          sv[c] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      }
+      // move the reference max when it grew past the lazy bound (warp-uniform
+      // TMEM traffic: lanes that keep theirs scale by 1)
+      const bool grow = mx > m_ref + t5::kLazyRescale || (m_ref == -INFINITY && mx > -INFINITY);
+      if (__any_sync(0xffffffffu, grow && m_ref > -INFINITY)) {
+        wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) / 2) & 1, abort_flag);  // O holds P_{j-1} V_{j-1}
+        tc_fence_after();
+        const float alpha = grow && m_ref > -INFINITY ? exp2f(m_ref - mx) : 1.f;
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          uint32_t o[32];
+          tmem_ld32(trow + 128 + c4 * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(trow + 128 + c4 * 32, o);
+        }
+        tmem_wait_st();
+        l *= alpha;
+      }
+      if (grow) m_ref = mx;
+      const float base = m_ref == -INFINITY ? 0.f : m_ref;
+      // this tile's P row -> P buffer sb (free once P_{j-2} V_{j-2} is done)
+      if (j >= 2) wait_bounded(&pv_done[sb], ((j - 2) / 2) & 1, abort_flag);
+      unsigned char *prow = smem + L::kPOff + sb * L::kPBytes + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float a, c;
+          w[e] = Mma<T>::pack(exp2f(__uint_as_float(sv[ch * 8 + 2 * e]) - base),
+                              exp2f(__uint_as_float(sv[ch * 8 + 2 * e + 1]) - base), a, c);
+          l += a + c;
+        }
+        *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      // rows of V outside every row's keys may hold anything: zero them
+      const int nvalid = min(kN, n - t0);
+      const int nskip = max(0, lo_first - t0);
+      if (nvalid < kN || nskip > 0) {
+        unsigned char *vz = smem + L::kRingOff + st * L::kStageBytes + L::kPanels * L::kKVPanel;
+        for (int c = r; c < kN * 8 * L::kPanels; c += 128) {
+          const int vr = c / (8 * L::kPanels), pn = (c / 8) % L::kPanels, ch = c % 8;
+          if (vr >= nskip && vr < nvalid) continue;
+          *reinterpret_cast<uint4 *>(vz + pn * L::kKVPanel + vr * 128 + (ch << 4)) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&p_full[sb]);
+    }
+    // ---- O / l -> global memory
+    wait_bounded(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) / 2) & 1, abort_flag);
+    tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    T *og = static_cast<T *>(p.out);
+#pragma unroll
+    for (int c4 = 0; c4 < D / 32; ++c4) {
+      uint32_t o[32];
+      tmem_ld32(trow + 128 + c4 * 32, o);
+      tmem_wait_ld();
+      if (r < rows) {
+        uint4 *dst = reinterpret_cast<uint4 *>(og + ((size_t)(qs0 + q0 + r) * p.num_q_heads + h) * D +
+                                               c4 * 32);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t w[4];
+          float a, c;
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = Mma<T>::pack(__uint_as_float(o[q4 * 8 + 2 * e]) * inv,
+                                __uint_as_float(o[q4 * 8 + 2 * e + 1]) * inv, a, c);
+          dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_free(tmem, t5::kTmemCols);
+}
+
 template <typename T, int D>
 pa_status launch(const PrefillParams &prm, const void *k_cache, const void *v_cache,
                  pa_dtype dtype, cudaStream_t stream) {
@@ -433,6 +781,32 @@ pa_status launch(const PrefillParams &prm, const void *k_cache, const void *v_ca
   }
   dim3 grid((unsigned)prm.num_q_heads, (unsigned)prm.q_tiles, (unsigned)prm.num_seqs);
   pa_prefill_kernel<T, D><<<grid, kThreads, L::kBytes, stream>>>(tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D>
+pa_status launch_tc(const PrefillParams &prm_in, int max_q_len, const void *k_cache,
+                    const void *v_cache, pa_dtype dtype, cudaStream_t stream) {
+  using L = t5::Lay<D>;
+  PrefillParams prm = prm_in;
+  prm.q_tiles = (max_q_len + t5::kM - 1) / t5::kM;
+  CUtensorMap tk, tv;
+  const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
+  const int box_rows = prm.block_size < t5::kN ? prm.block_size : t5::kN;
+  if (!pa_internal_pool_tensor_map(&tk, k_cache, rows, D, box_rows, dtype) ||
+      !pa_internal_pool_tensor_map(&tv, v_cache, rows, D, box_rows, dtype))
+    return PA_ERR_CUDA;
+  static bool configured[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+  if (!configured[dev]) {
+    if (cudaFuncSetAttribute(pa_prefill_tc_kernel<T, D>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+      return PA_ERR_CUDA;
+    configured[dev] = true;
+  }
+  dim3 grid((unsigned)prm.num_q_heads, (unsigned)prm.q_tiles, (unsigned)prm.num_seqs);
+  pa_prefill_tc_kernel<T, D><<<grid, t5::kThreads, L::kBytes, stream>>>(tk, tv, prm);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -482,11 +856,19 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
   prm.q_tiles = q_tiles;
   prm.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+#if PA_PREFILL_TCGEN05
+  if (dtype == PA_BF16)
+    return head_dim == 128 ? launch_tc<__nv_bfloat16, 128>(prm, max_q_len, k_cache, v_cache, dtype, st)
+                           : launch_tc<__nv_bfloat16, 64>(prm, max_q_len, k_cache, v_cache, dtype, st);
+  return head_dim == 128 ? launch_tc<__half, 128>(prm, max_q_len, k_cache, v_cache, dtype, st)
+                         : launch_tc<__half, 64>(prm, max_q_len, k_cache, v_cache, dtype, st);
+#else
   if (dtype == PA_BF16)
     return head_dim == 128 ? launch<__nv_bfloat16, 128>(prm, k_cache, v_cache, dtype, st)
                            : launch<__nv_bfloat16, 64>(prm, k_cache, v_cache, dtype, st);
   return head_dim == 128 ? launch<__half, 128>(prm, k_cache, v_cache, dtype, st)
                          : launch<__half, 64>(prm, k_cache, v_cache, dtype, st);
+#endif
 }
 
 // Read and clear this file's error word (stream-ordered; synchronises the stream).
