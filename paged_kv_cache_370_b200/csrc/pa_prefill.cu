@@ -103,6 +103,15 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, vol
   }
 }
 
+// 2^x by the hardware's approximate base-2 exponential (PTX ex2.approx.ftz, one
+// instruction; its error is far below the rounding of the 16-bit weights it
+// feeds, and -inf gives 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // First position the token at position p attends to.
 __device__ __forceinline__ int first_key(int p, int window) {
   return window > 0 && p + 1 > window ? p + 1 - window : 0;
@@ -420,43 +429,46 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
 }
 
 // ============================================================ tcgen05 kernel (5th-gen tensor cores)
-// Same computation, one CTA per (q head, 128 query tokens, sequence), with the
-// two products on tcgen05.mma (M = 128 query rows, one elected issuing thread)
-// and both accumulators in tensor memory:
-//   warp 0      stages 64-key K/V tiles with TMA into a 3-stage ring (as above);
-//   warp 1      allocates TMEM; its lane 0 issues S_j = Q K_j^T (TMEM, double
-//               buffered) and, one tile behind, O += P_{j-1} V_{j-1} (TMEM), and
-//               commits each group to an mbarrier;
-//   warps 2-3   copy the Q tile into shared memory (128-byte swizzled, K-major);
-//   warps 4-7   one thread per query row: read its S row from TMEM, mask, online
-//               softmax in the log2 domain, write its P row (bf16 / fp16,
-//               swizzled) to shared memory for the next product; O is rescaled in
-//               TMEM only when a row's max grows by more than 2^8 (the weights
-//               against the stale max stay <= 2^8, and the final division by the
-//               matching sum makes the result exact either way); finally O / l
-//               from TMEM to global memory.
+// Same computation, one CTA per (q head, 256 query tokens, sequence), with the
+// two products on tcgen05.mma and every accumulator in tensor memory. The 256
+// rows form two groups of 128 (one tcgen05 M each); the groups share every K/V
+// tile and take turns on the tensor core, so one group's softmax overlaps the
+// other group's products.
+//   warp 0      stages 64-key K/V tiles with TMA into a 2-stage ring;
+//   warp 1      allocates TMEM (512 columns: per group two S buffers and O); its
+//               lane 0 issues, per tile, S = Q K^T for each group and, one tile
+//               behind, O += P V for each group, committing each to an mbarrier;
+//   warps 2-9   one thread per query row (group = (warp - 2) / 4, TMEM lane =
+//               32 * (warp % 4) + lane): copy its Q row into shared memory, then
+//               per tile read its S row from TMEM, mask, online softmax in the
+//               log2 domain, write its P row (swizzled) for the next product.
+//               O is rescaled in TMEM only when the row max grows by more than
+//               2^8 (the weights against the stale max stay <= 2^8 and the final
+//               division by the matching sum keeps the result exact); at the end
+//               O / l goes from TMEM to global memory.
 namespace t5 {
 
-constexpr int kM = 128;        // query rows per CTA (tcgen05 M)
+constexpr int kM = 128;        // query rows per group (tcgen05 M)
+constexpr int kGroups = 2;
 constexpr int kN = 64;         // keys per tile
-constexpr int kStages = 3;
-constexpr int kThreads = 256;
-constexpr uint32_t kTmemCols = 256;  // S buffers at columns 0 and 64, O at 128
+constexpr int kStages = 2;
+constexpr int kThreads = (2 + 4 * kGroups) * 32;
+constexpr uint32_t kTmemCols = 512;  // group g: S buffers at 256g + {0, 64}, O at 256g + 128
 constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
 
 template <int D>
 struct Lay {
   static constexpr int kPanels = D / 64;
-  static constexpr int kQPanel = kM * 128;                    // 128 rows x 128 bytes
+  static constexpr int kQPanel = kGroups * kM * 128;          // 256 rows x 128 bytes
   static constexpr int kQBytes = kPanels * kQPanel;
   static constexpr int kKVPanel = kN * 128;                   // 64 rows x 128 bytes
   static constexpr int kStageBytes = 2 * kPanels * kKVPanel;  // K panels, then V panels
   static constexpr int kPBytes = kM * 128;                    // 128 rows x 64 keys
   static constexpr int kRingOff = kQBytes;
-  static constexpr int kPOff = kRingOff + kStages * kStageBytes;
-  static constexpr int kBarOff = kPOff + 2 * kPBytes;
-  // full[3] empty[3] q_ready s_full[2] s_free[2] p_full[2] pv_done[2] mma_done
-  static constexpr int kNumBars = 2 * kStages + 10;
+  static constexpr int kPOff = kRingOff + kStages * kStageBytes;  // [group][buffer]
+  static constexpr int kBarOff = kPOff + kGroups * 2 * kPBytes;
+  // full[S] empty[S] q_ready mma_done, then per group s_full[2] s_free[2] p_full[2] pv_done[2]
+  static constexpr int kNumBars = 2 * kStages + 2 + 8 * kGroups;
   static constexpr int kTmemOff = kBarOff + kNumBars * 8;
   static constexpr int kFlagOff = kTmemOff + 8;
   static constexpr int kBytes = 1024 + kFlagOff + 16;
@@ -469,7 +481,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const PrefillParams p) {
   using L = t5::Lay<D>;
-  constexpr int kM = t5::kM, kN = t5::kN, NS = t5::kStages;
+  constexpr int kM = t5::kM, kN = t5::kN, NS = t5::kStages, NG = t5::kGroups;
   constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t kIdescS = umma_idesc_f16(kFmt, 0, 0, kN, kM);  // Q (K-major) . K (K-major)
   constexpr uint32_t kIdescO = umma_idesc_f16(kFmt, 0, 1, D, kM);   // P (K-major) . V (MN-major)
@@ -479,8 +491,12 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
   uint64_t *full_bar = bars, *empty_bar = bars + NS, *q_ready = bars + 2 * NS;
-  uint64_t *s_full = q_ready + 1, *s_free = s_full + 2, *p_full = s_free + 2;
-  uint64_t *pv_done = p_full + 2, *mma_done = pv_done + 2;
+  uint64_t *mma_done = q_ready + 1;
+  // per group g: s_full[g][2], s_free[g][2], p_full[g][2], pv_done[g][2]
+  auto s_full = [&](int g, int i) { return mma_done + 1 + g * 8 + i; };
+  auto s_free = [&](int g, int i) { return mma_done + 1 + g * 8 + 2 + i; };
+  auto p_full = [&](int g, int i) { return mma_done + 1 + g * 8 + 4 + i; };
+  auto pv_done = [&](int g, int i) { return mma_done + 1 + g * 8 + 6 + i; };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
   const uint32_t q_sm = smem_u32(smem);
@@ -511,28 +527,35 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   }
   if (bad && tid == 0 && h == 0 && blockIdx.y == 0)
     atomicOr(&g_prefill_error, PA_DEVERR_CONTEXT_LEN);
-  const int q0 = qt * kM;
+  const int q0 = qt * NG * kM;
   if (q0 >= m) return;  // no query rows here (uniform; before any TMEM is taken)
-  const int rows = min(kM, m - q0);
+  const int rows = min(NG * kM, m - q0);
   const int p_first = n - m + q0;
-  const int p_last = p_first + rows - 1;
   const int align = bs < kN ? bs : kN;
   const int k_base = first_key(p_first, p.window) & ~(align - 1);
-  const int ntiles = (p_last + 1 - k_base + kN - 1) / kN;
+  // tiles each group needs (up to its last row); group 1 may have no rows
+  int gtiles[NG];
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    const int grows = min(kM, rows - g * kM);
+    gtiles[g] = grows > 0 ? (p_first + g * kM + grows - 1 + 1 - k_base + kN - 1) / kN : 0;
+  }
+  const int ntiles = gtiles[NG - 1] > 0 ? gtiles[NG - 1] : gtiles[0];
 
   if (tid == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);  // one tcgen05.commit per use
     }
-    mbar_init(q_ready, 64);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128);
-      mbar_init(&pv_done[i], 1);
-    }
+    mbar_init(q_ready, 4 * 32 * NG);
     mbar_init(mma_done, 1);
+    for (int g = 0; g < NG; ++g)
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(s_full(g, i), 1);
+        mbar_init(s_free(g, i), 128);
+        mbar_init(p_full(g, i), 128);
+        mbar_init(pv_done(g, i), 1);
+      }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -582,39 +605,72 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     }
   } else if (warp == 1) {
     // ====================================================================== MMA issuer
+    // Issues whatever is ready, in any order: S_j of a group as soon as K_j has
+    // landed and the group has read S_{j-2} (double-buffered S), P_j V_j of a
+    // group as soon as its softmax wrote P_j; a tile's stage goes back to the
+    // producer once every group that reads it has issued its P V.
     if (lane == 0) {
       bool go = wait_bounded(q_ready, 0, abort_flag);
       tc_fence_after();
-      for (int j = 0; j <= ntiles && go; ++j) {
-        if (j < ntiles) {  // S_j = Q K_j^T into S buffer j % 2
-          const int st = j % NS, sb = j & 1;
-          go = wait_bounded(&full_bar[st], (j / NS) & 1, abort_flag);
-          if (go && j >= 2) go = wait_bounded(&s_free[sb], ((j - 2) / 2) & 1, abort_flag);
-          if (!go) break;
-          tc_fence_after();
-          const uint32_t kaddr = ring + st * L::kStageBytes;
+      int ns[NG], npv[NG];
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_f16(tmem + sb * kN,
-                     umma_desc_sw128(q_sm + (kk / 4) * L::kQPanel + (kk % 4) * 32, 16, 1024),
-                     umma_desc_sw128(kaddr + (kk / 4) * L::kKVPanel + (kk % 4) * 32, 16, 1024),
-                     kIdescS, kk > 0);
-          umma_commit(&s_full[sb]);
+      for (int g = 0; g < NG; ++g) ns[g] = npv[g] = 0;
+      int released = 0;
+      unsigned long long idle_since = global_ns();
+      while (go) {
+        bool done = true, progress = false;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+          if (npv[g] < gtiles[g]) done = false;
+          const int js = ns[g];
+          if (js < gtiles[g] && mbar_try_wait(&full_bar[js % NS], (js / NS) & 1) &&
+              (js < 2 || mbar_try_wait(s_free(g, js & 1), ((js - 2) / 2) & 1))) {
+            tc_fence_after();
+            const uint32_t kaddr = ring + (js % NS) * L::kStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_f16(tmem + g * 256 + (js & 1) * kN,
+                       umma_desc_sw128(q_sm + (kk / 4) * L::kQPanel + g * kM * 128 + (kk % 4) * 32,
+                                       16, 1024),
+                       umma_desc_sw128(kaddr + (kk / 4) * L::kKVPanel + (kk % 4) * 32, 16, 1024),
+                       kIdescS, kk > 0);
+            umma_commit(s_full(g, js & 1));
+            ++ns[g];
+            progress = true;
+          }
+          const int jp = npv[g];
+          if (jp < ns[g] && mbar_try_wait(p_full(g, jp & 1), (jp / 2) & 1)) {
+            tc_fence_after();
+            const uint32_t vaddr = ring + (jp % NS) * L::kStageBytes + L::kPanels * L::kKVPanel;
+#pragma unroll
+            for (int kk = 0; kk < kN / 16; ++kk)
+              umma_f16(tmem + g * 256 + 128,
+                       umma_desc_sw128(p_sm + (g * 2 + (jp & 1)) * L::kPBytes + kk * 32, 16, 1024),
+                       umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
+                       kIdescO, jp > 0 || kk > 0);
+            umma_commit(pv_done(g, jp & 1));
+            ++npv[g];
+            progress = true;
+          }
         }
-        if (j >= 1) {  // O += P_{j-1} V_{j-1}
-          const int jp = j - 1, st = jp % NS, pb = jp & 1;
-          go = wait_bounded(&p_full[pb], (jp / 2) & 1, abort_flag);
-          if (!go) break;
-          tc_fence_after();
-          const uint32_t vaddr = ring + st * L::kStageBytes + L::kPanels * L::kKVPanel;
+        // release, in order, every tile all of whose readers have issued P V
+        while (released < ntiles) {
+          bool all = true;
 #pragma unroll
-          for (int kk = 0; kk < kN / 16; ++kk)
-            umma_f16(tmem + 128,
-                     umma_desc_sw128(p_sm + pb * L::kPBytes + kk * 32, 16, 1024),
-                     umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
-                     kIdescO, jp > 0 || kk > 0);
-          umma_commit(&pv_done[pb]);
-          umma_commit(&empty_bar[st]);
+          for (int g = 0; g < NG; ++g)
+            if (released < gtiles[g] && npv[g] <= released) all = false;
+          if (!all) break;
+          umma_commit(&empty_bar[released % NS]);
+          ++released;
+        }
+        if (done) break;
+        const unsigned long long now = global_ns();
+        if (progress) {
+          idle_since = now;
+        } else if (now - idle_since > kWaitLimitNs || *abort_flag) {
+          *abort_flag = 1;
+          atomicOr(&g_prefill_error, PA_DEVERR_TIMEOUT);
+          break;
         }
       }
       // every product issued so far has finished before TMEM is released
@@ -622,45 +678,49 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       wait_bounded(mma_done, 0, abort_flag);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ======================================================================= Q loaders
-    const T *qg = static_cast<const T *>(p.q);
-    constexpr int kChunks = D / 8;
-    for (int c = tid - 64; c < kM * kChunks; c += 64) {
-      const int r = c / kChunks, ch = c % kChunks;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (r < rows)
-        v = __ldg(reinterpret_cast<const uint4 *>(
-                      qg + ((size_t)(qs0 + q0 + r) * p.num_q_heads + h) * D) + ch);
-      *reinterpret_cast<uint4 *>(smem + (ch / 8) * L::kQPanel + r * 128 +
-                                 (((ch % 8) ^ (r & 7)) << 4)) = v;
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(q_ready);
   } else {
-    // ========================================================== softmax, one row each
-    const int r = tid - 128;                      // query row == TMEM lane
-    const uint32_t trow = tmem + ((uint32_t)((warp - 4) * 32) << 16);
-    const int pr = min(p_first + r, n - 1);       // rows past the chunk: computed, not stored
+    // ====================================================== softmax, one row per thread
+    const int grp = (warp - 2) / 4;
+    const int r = 32 * (warp % 4) + lane;          // row in the group == TMEM lane
+    const int R = grp * kM + r;                    // row in the CTA
+    const uint32_t trow = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + grp * 256;
+    const int my_tiles = gtiles[grp];
+    // this row of Q -> shared memory (128-byte swizzled, K-major)
+    {
+      const T *qg = static_cast<const T *>(p.q);
+      constexpr int kChunks = D / 8;
+#pragma unroll 4
+      for (int ch = 0; ch < kChunks; ++ch) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (R < rows)
+          v = __ldg(reinterpret_cast<const uint4 *>(
+                        qg + ((size_t)(qs0 + q0 + R) * p.num_q_heads + h) * D) + ch);
+        *reinterpret_cast<uint4 *>(smem + (ch / 8) * L::kQPanel + R * 128 +
+                                   (((ch % 8) ^ (R & 7)) << 4)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(q_ready);
+    }
+    const int pr = min(p_first + R, n - 1);        // rows past the chunk: computed, not stored
     const int lo = first_key(pr, p.window);
     const int lo_first = first_key(p_first, p.window);
+    const int wr0 = min(p_first + grp * kM + 32 * (warp % 4), n - 1);
+    const int wr1 = min(p_first + grp * kM + 32 * (warp % 4) + 31, n - 1);
     float m_ref = -INFINITY, l = 0.f;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = 0; j < my_tiles; ++j) {
       const int sb = j & 1, st = j % NS;
       const int t0 = k_base + j * kN;
-      wait_bounded(&s_full[sb], (j / 2) & 1, abort_flag);
+      wait_bounded(s_full(grp, sb), (j / 2) & 1, abort_flag);
       tc_fence_after();
       uint32_t sv[64];
       tmem_ld32(trow + sb * kN, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld32(trow + sb * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&s_free[sb]);
+      mbar_arrive(s_free(grp, sb));
       float mx = -INFINITY;
       // the mask only matters on tiles that reach past a row of this warp or
       // start before a row's window (warp-uniform)
-      const int wr0 = min(p_first + (warp - 4) * 32, n - 1);
-      const int wr1 = min(p_first + (warp - 4) * 32 + 31, n - 1);
       if (t0 + kN - 1 > wr0 || (p.window > 0 && t0 < first_key(wr1, p.window))) {
 #pragma unroll
         for (int c = 0; c < kN; ++c) {
@@ -681,7 +741,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       // TMEM traffic: lanes that keep theirs scale by 1)
       const bool grow = mx > m_ref + t5::kLazyRescale || (m_ref == -INFINITY && mx > -INFINITY);
       if (__any_sync(0xffffffffu, grow && m_ref > -INFINITY)) {
-        wait_bounded(&pv_done[(j - 1) & 1], ((j - 1) / 2) & 1, abort_flag);  // O holds P_{j-1} V_{j-1}
+        wait_bounded(pv_done(grp, (j - 1) & 1), ((j - 1) / 2) & 1, abort_flag);  // O has P_{j-1} V_{j-1}
         tc_fence_after();
         const float alpha = grow && m_ref > -INFINITY ? exp2f(m_ref - mx) : 1.f;
 #pragma unroll
@@ -698,22 +758,23 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       }
       if (grow) m_ref = mx;
       const float base = m_ref == -INFINITY ? 0.f : m_ref;
-      // this tile's P row -> P buffer sb (free once P_{j-2} V_{j-2} is done)
-      if (j >= 2) wait_bounded(&pv_done[sb], ((j - 2) / 2) & 1, abort_flag);
-      unsigned char *prow = smem + L::kPOff + sb * L::kPBytes + r * 128;
+      // this tile's P row -> P buffer (grp, sb), free once P_{j-2} V_{j-2} is done
+      if (j >= 2) wait_bounded(pv_done(grp, sb), ((j - 2) / 2) & 1, abort_flag);
+      unsigned char *prow = smem + L::kPOff + (grp * 2 + sb) * L::kPBytes + r * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float a, c;
-          w[e] = Mma<T>::pack(exp2f(__uint_as_float(sv[ch * 8 + 2 * e]) - base),
-                              exp2f(__uint_as_float(sv[ch * 8 + 2 * e + 1]) - base), a, c);
+          w[e] = Mma<T>::pack(ex2_approx(__uint_as_float(sv[ch * 8 + 2 * e]) - base),
+                              ex2_approx(__uint_as_float(sv[ch * 8 + 2 * e + 1]) - base), a, c);
           l += a + c;
         }
         *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      // rows of V outside every row's keys may hold anything: zero them
+      // rows of V outside every row's keys may hold anything: zero them (both
+      // groups zero the same rows of a shared stage; the writes are identical)
       const int nvalid = min(kN, n - t0);
       const int nskip = max(0, lo_first - t0);
       if (nvalid < kN || nskip > 0) {
@@ -726,30 +787,32 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(&p_full[sb]);
+      mbar_arrive(p_full(grp, sb));
     }
     // ---- O / l -> global memory
-    wait_bounded(&pv_done[(ntiles - 1) & 1], ((ntiles - 1) / 2) & 1, abort_flag);
-    tc_fence_after();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    T *og = static_cast<T *>(p.out);
+    if (my_tiles > 0) {
+      wait_bounded(pv_done(grp, (my_tiles - 1) & 1), ((my_tiles - 1) / 2) & 1, abort_flag);
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      T *og = static_cast<T *>(p.out);
 #pragma unroll
-    for (int c4 = 0; c4 < D / 32; ++c4) {
-      uint32_t o[32];
-      tmem_ld32(trow + 128 + c4 * 32, o);
-      tmem_wait_ld();
-      if (r < rows) {
-        uint4 *dst = reinterpret_cast<uint4 *>(og + ((size_t)(qs0 + q0 + r) * p.num_q_heads + h) * D +
-                                               c4 * 32);
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t o[32];
+        tmem_ld32(trow + 128 + c4 * 32, o);
+        tmem_wait_ld();
+        if (R < rows) {
+          uint4 *dst = reinterpret_cast<uint4 *>(
+              og + ((size_t)(qs0 + q0 + R) * p.num_q_heads + h) * D + c4 * 32);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t w[4];
-          float a, c;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w[4];
+            float a, c;
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w[e] = Mma<T>::pack(__uint_as_float(o[q4 * 8 + 2 * e]) * inv,
-                                __uint_as_float(o[q4 * 8 + 2 * e + 1]) * inv, a, c);
-          dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int e = 0; e < 4; ++e)
+              w[e] = Mma<T>::pack(__uint_as_float(o[q4 * 8 + 2 * e]) * inv,
+                                  __uint_as_float(o[q4 * 8 + 2 * e + 1]) * inv, a, c);
+            dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
     }
@@ -789,7 +852,7 @@ pa_status launch_tc(const PrefillParams &prm_in, int max_q_len, const void *k_ca
                     const void *v_cache, pa_dtype dtype, cudaStream_t stream) {
   using L = t5::Lay<D>;
   PrefillParams prm = prm_in;
-  prm.q_tiles = (max_q_len + t5::kM - 1) / t5::kM;
+  prm.q_tiles = (max_q_len + t5::kGroups * t5::kM - 1) / (t5::kGroups * t5::kM);
   CUtensorMap tk, tv;
   const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
   const int box_rows = prm.block_size < t5::kN ? prm.block_size : t5::kN;
