@@ -444,8 +444,9 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
 //               log2 domain, write its P row (swizzled) for the next product.
 //               O is rescaled in TMEM only when the row max grows by more than
 //               2^8 (the weights against the stale max stay <= 2^8 and the final
-//               division by the matching sum keeps the result exact); at the end
-//               O / l goes from TMEM to global memory.
+//               division by the matching sum keeps the result exact); l sums the
+//               weights before their rounding to 16 bits; at the end O / l goes
+//               from TMEM to global memory.
 namespace t5 {
 
 constexpr int kM = 128;        // query rows per group (tcgen05 M)
@@ -718,6 +719,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(s_free(grp, sb));
+      // max of the raw scores (the scale is positive); masked keys become -inf
       float mx = -INFINITY;
       // the mask only matters on tiles that reach past a row of this warp or
       // start before a row's window (warp-uniform)
@@ -725,18 +727,15 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
 #pragma unroll
         for (int c = 0; c < kN; ++c) {
           const int kp = t0 + c;
-          const float x = (kp <= pr && kp >= lo) ? __uint_as_float(sv[c]) * p.scale_log2 : -INFINITY;
+          const float x = (kp <= pr && kp >= lo) ? __uint_as_float(sv[c]) : -INFINITY;
           sv[c] = __float_as_uint(x);
           mx = fmaxf(mx, x);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < kN; ++c) {
-          const float x = __uint_as_float(sv[c]) * p.scale_log2;
-          sv[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+        for (int c = 0; c < kN; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
       }
+      mx *= p.scale_log2;  // log2 domain
       // move the reference max when it grew past the lazy bound (warp-uniform
       // TMEM traffic: lanes that keep theirs scale by 1)
       const bool grow = mx > m_ref + t5::kLazyRescale || (m_ref == -INFINITY && mx > -INFINITY);
@@ -757,8 +756,9 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         l *= alpha;
       }
       if (grow) m_ref = mx;
-      const float base = m_ref == -INFINITY ? 0.f : m_ref;
-      // this tile's P row -> P buffer (grp, sb), free once P_{j-2} V_{j-2} is done
+      const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
+      // this tile's P row -> P buffer (grp, sb), free once P_{j-2} V_{j-2} is done;
+      // weight = 2^(s * scale_log2 - m_ref), one FMA and one exp2 per key
       if (j >= 2) wait_bounded(pv_done(grp, sb), ((j - 2) / 2) & 1, abort_flag);
       unsigned char *prow = smem + L::kPOff + (grp * 2 + sb) * L::kPBytes + r * 128;
 #pragma unroll
@@ -766,10 +766,11 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         uint32_t w[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          float a, c;
-          w[e] = Mma<T>::pack(ex2_approx(__uint_as_float(sv[ch * 8 + 2 * e]) - base),
-                              ex2_approx(__uint_as_float(sv[ch * 8 + 2 * e + 1]) - base), a, c);
-          l += a + c;
+          const float a = ex2_approx(fmaf(__uint_as_float(sv[ch * 8 + 2 * e]), p.scale_log2, nbase));
+          const float c = ex2_approx(fmaf(__uint_as_float(sv[ch * 8 + 2 * e + 1]), p.scale_log2, nbase));
+          float ra, rc;
+          w[e] = Mma<T>::pack(a, c, ra, rc);
+          l += a + c;  // the sum of the unrounded weights (|rounding| <= 2^-9 relative each)
         }
         *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
