@@ -71,6 +71,8 @@ def parse_args():
                     help="llama8b pool size (smaller for profiler captures)")
     ap.add_argument("--window", type=int, default=0,
                     help="sliding window: attend to each sequence's last W positions (0: all)")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="no programmatic early start of each decode kernel")
     ap.add_argument("--no-fuse", action="store_true",
                     help="separate KV-write kernel instead of pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
@@ -202,7 +204,10 @@ def _workload_config(args, batches, pt):
                 "batches_rotated": len(batches),
                 "l2": f"inputs larger than L2: {len(batches)} rotating batches, "
                       f"{sum(decode_step_bytes(x.context_lens, 32, 8, 128, 16)['kv'] for x in batches) / 1e9:.2f} GB of KV",
-                "timing": "CUDA graphs replayed back to back; CUDA events on the stream"}
+                "timing": "CUDA graphs replayed back to back; CUDA events on the stream",
+                "launch": ("plain stream order" if args.no_overlap or args.no_fuse else
+                           "programmatic early start: each decode kernel's start-up overlaps "
+                           "the previous kernel's tail (pa_decode_append_overlapped)")}
     if args.workload == "long_skew":
         return {"workload": "long-context skew decode", "num_seqs": 8, "num_q_heads": 32,
                 "num_kv_heads": 8, "head_dim": 128, "block_size": 16,
@@ -251,7 +256,7 @@ def device_steps(args, batches, torch, device):
                           context_lens=torch.from_numpy(b.context_lens).to(device),
                           max_context_len=b.max_context_len, scale=float(b.scale),
                           partition_tokens=args.partition_tokens, fused=not args.no_fuse,
-                          window=args.window)
+                          window=args.window, overlapped=not args.no_overlap)
         del k_all, v_all
         steps.append(step)
         infos.append(_byte_info(b.context_lens, b.num_q_heads, b.num_kv_heads, b.head_dim,

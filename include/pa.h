@@ -306,6 +306,27 @@ pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *
                      int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale,
                      int window, pa_dtype dtype, void *stream);
 
+/* ------------------------------------------------------------------------------------------
+ * pa_decode_append_overlapped -- pa_decode_append whose kernel may start before the kernel
+ * launched before it on the same stream has finished (programmatic dependent launch), so
+ * its start-up -- scanning the lengths, locating its tiles, fetching the first block ids --
+ * overlaps the end of that kernel. It reads context_lens, block_tables and slot_mapping
+ * before waiting for the preceding kernel, and q, k_new, v_new and the pools after.
+ * Contract: those three arrays must not be written by the immediately preceding kernel
+ * (e.g. they are uploaded or prepared before it). Same arguments and results as
+ * pa_decode_append; without the even-split kernel (block size, GQA group) it is
+ * pa_decode_append.
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_decode_append_overlapped(void *out, const void *q, const void *k_new,
+                                      const void *v_new, const int64_t *slot_mapping,
+                                      void *k_cache, void *v_cache, const int32_t *block_tables,
+                                      int max_blocks_per_seq, const int32_t *context_lens,
+                                      int max_context_len, int num_seqs, int num_q_heads,
+                                      int num_kv_heads, int head_dim, int block_size,
+                                      int num_blocks, float scale, pa_dtype dtype,
+                                      void *workspace, size_t workspace_bytes,
+                                      int partition_tokens, void *stream);
+
 /* Kernels one pa_decode_append call with these arguments launches (0 if none). */
 int pa_decode_append_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                               int block_size, int num_blocks, int max_context_len,

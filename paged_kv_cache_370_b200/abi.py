@@ -61,6 +61,8 @@ def _load() -> ctypes.CDLL:
         "pa_decode_append": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, P, sz,
                                  i, P]),
         "pa_decode_append_launches": (i, [i, i, i, i, i, i, i, i]),
+        "pa_decode_append_overlapped": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f,
+                                            i, P, sz, i, P]),
         "pa_decode_window": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P, sz, i, P]),
         "pa_decode_window_launches": (i, [i, i, i, i, i, i, i]),
         "pa_prefill": (i, [P, P, P, P, P, i, P, P, i, i, i, i, i, i, i, i, i, f, i, i, P]),
@@ -325,6 +327,24 @@ def pa_decode_append(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block
         B, hq, hkv, d, bs, nb, float(scale), _dtype_code(q), _dev_ptr(workspace, "workspace"),
         ws_bytes, int(partition_tokens), _stream(stream))
     _check(st, "pa_decode_append")
+
+
+def pa_decode_append_overlapped(out, q, k_new, v_new, slot_mapping, k_cache, v_cache,
+                                block_tables, context_lens, max_context_len, scale,
+                                workspace=None, partition_tokens=0, stream=None):
+    """pa_decode_append whose kernel may start during the preceding kernel's tail; the
+    lengths, tables and slots must not be written by that preceding kernel."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = _lib.pa_decode_append_overlapped(
+        _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_new, "k_new"), _dev_ptr(v_new, "v_new"),
+        _dev_ptr(slot_mapping, "slot_mapping"), _dev_ptr(k_cache, "k_cache"),
+        _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),
+        int(block_tables.shape[1]), _dev_ptr(context_lens, "context_lens"), int(max_context_len),
+        B, hq, hkv, d, bs, nb, float(scale), _dtype_code(q), _dev_ptr(workspace, "workspace"),
+        ws_bytes, int(partition_tokens), _stream(stream))
+    _check(st, "pa_decode_append_overlapped")
 
 
 def pa_decode_append_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,

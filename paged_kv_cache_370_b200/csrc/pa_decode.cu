@@ -139,6 +139,8 @@ struct DecodeParams {
   // sliding window (partition kernel only): a sequence of length len attends
   // to positions [len - window, len) (0: every position)
   int window;
+  // even-split kernel launched as a programmatic dependent of the preceding kernel
+  int early_start;
 };
 
 // First position attended by a sequence of length len under a window of w
@@ -755,6 +757,13 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
     }
+    // Everything above read only the lengths, the block tables and the slots.
+    // Launched as a programmatic dependent (pa_decode_append_overlapped), the
+    // kernel may have started before the preceding kernel finished: wait for it
+    // here, before the first read of q, the new rows or the pools (no-op
+    // otherwise), then let the next kernel start its own prologue.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % NS;
       // stage free? (after a give-up the loop runs on without waiting: no early exits)
@@ -858,6 +867,8 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
   }
 
   // ======================================================================= consumers
+  // (their bounded waits start once the preceding kernel is done: see the producer)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int g = lane >> 2;  // fragment row group
   const int t = lane & 3;   // this lane's heads are 2t and 2t+1
   const int wrow = warp * 16;
@@ -1319,8 +1330,18 @@ pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dty
       return PA_ERR_CUDA;
     if (!ensure_smem(tc::pa_decode_stream_kernel<T, D, G>, (size_t)C::kBytes, configured))
       return PA_ERR_CUDA;
-    tc::pa_decode_stream_kernel<T, D, G>
-        <<<(unsigned)prm.grid_ctas, tc::kThreads, C::kBytes, stream>>>(tk, tv, prm);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)prm.grid_ctas);
+    cfg.blockDim = dim3(tc::kThreads);
+    cfg.dynamicSmemBytes = C::kBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = prm.early_start ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, tc::pa_decode_stream_kernel<T, D, G>, tk, tv, prm) != cudaSuccess)
+      return PA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
   using L = Smem<T, D, G>;
@@ -1441,7 +1462,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                       int num_blocks, float scale, pa_dtype dtype, void *workspace,
                       size_t workspace_bytes, int partition_tokens, void *stream,
-                      const FusedWrite *fw, int window) {
+                      const FusedWrite *fw, int window, bool early_start = false) {
   if (window < 0) return PA_ERR_INVALID;
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
       block_size <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
@@ -1499,6 +1520,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   prm.k_cache_w = fw ? fw->k_cache : nullptr;
   prm.v_cache_w = fw ? fw->v_cache : nullptr;
   prm.window = window;
+  prm.early_start = early_start ? 1 : 0;
   if (fw && !streamk) return PA_ERR_INVALID;  // only the even-split kernel writes
   prm.max_blocks_per_seq = max_blocks_per_seq;
   prm.max_context_len = max_context_len;
@@ -1579,7 +1601,7 @@ pa_status decode_append_impl(void *out, const void *q, const void *k_new, const 
                              int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                              int num_blocks, float scale, pa_dtype dtype, void *workspace,
                              size_t workspace_bytes, int partition_tokens, void *stream,
-                             int window) {
+                             int window, bool early_start = false) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
       block_size <= 0 || num_blocks <= 0)
     return PA_ERR_INVALID;
@@ -1593,7 +1615,7 @@ pa_status decode_append_impl(void *out, const void *q, const void *k_new, const 
     return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                        max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
                        block_size, num_blocks, scale, dtype, workspace, workspace_bytes,
-                       partition_tokens, stream, &fw, 0);
+                       partition_tokens, stream, &fw, 0, early_start);
   }
   // other shapes, and sliding windows: the write kernel, then the decode
   const pa_status st = pa_reshape_and_cache(k_new, v_new, slot_mapping, num_seqs, k_cache,
@@ -1621,6 +1643,18 @@ extern "C" pa_status pa_decode_append(void *out, const void *q, const void *k_ne
                             max_blocks_per_seq, context_lens, max_context_len, num_seqs,
                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                             dtype, workspace, workspace_bytes, partition_tokens, stream, 0);
+}
+
+extern "C" pa_status pa_decode_append_overlapped(
+    void *out, const void *q, const void *k_new, const void *v_new, const int64_t *slot_mapping,
+    void *k_cache, void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+    const int32_t *context_lens, int max_context_len, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale, pa_dtype dtype,
+    void *workspace, size_t workspace_bytes, int partition_tokens, void *stream) {
+  return decode_append_impl(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,
+                            max_blocks_per_seq, context_lens, max_context_len, num_seqs,
+                            num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                            dtype, workspace, workspace_bytes, partition_tokens, stream, 0, true);
 }
 
 extern "C" pa_status pa_decode_append_window(

@@ -22,13 +22,18 @@ from . import abi
 class DecodeStep:
     def __init__(self, *, k_cache, v_cache, q, k_new, v_new, slot_mapping, block_tables,
                  context_lens, max_context_len: int, scale: float, partition_tokens: int = 0,
-                 copy_pairs=None, out=None, fused: bool = False, window: int = 0):
+                 copy_pairs=None, out=None, fused: bool = False, window: int = 0,
+                 overlapped: bool = False):
         """``fused``: write the new tokens inside the decode (pa_decode_append);
         k_new/v_new then hold one token per sequence, at position len - 1.
         ``window`` > 0: attend to each sequence's last ``window`` positions only
         (pa_decode_window / pa_decode_append_window)."""
         self.fused = fused
         self.window = int(window)
+        # fused steps only: the kernel may start during the preceding kernel's tail
+        # (pa_decode_append_overlapped); the lengths, tables and slots must not be
+        # written by that kernel
+        self.overlapped = overlapped
         self.k_cache, self.v_cache = k_cache, v_cache
         self.q, self.k_new, self.v_new = q, k_new, v_new
         self.slot_mapping = slot_mapping
@@ -94,10 +99,10 @@ class DecodeStep:
                                         self.max_context_len, self.scale, self.window,
                                         self.workspace, self.partition_tokens, stream)
             return
-        abi.pa_decode_append(self.out, self.q, self.k_new, self.v_new, self.slot_mapping,
-                             self.k_cache, self.v_cache, self.block_tables, self.context_lens,
-                             self.max_context_len, self.scale, self.workspace,
-                             self.partition_tokens, stream)
+        fn = abi.pa_decode_append_overlapped if self.overlapped else abi.pa_decode_append
+        fn(self.out, self.q, self.k_new, self.v_new, self.slot_mapping, self.k_cache,
+           self.v_cache, self.block_tables, self.context_lens, self.max_context_len, self.scale,
+           self.workspace, self.partition_tokens, stream)
 
     def run(self, stream=None):
         self.copy(stream)

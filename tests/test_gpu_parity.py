@@ -218,6 +218,35 @@ def test_fused_write_full(make):
     assert torch.equal(ref.v_cache.view(torch.int16), g.v_cache.view(torch.int16))
 
 
+def test_overlapped_launch_gives_the_same_bits():
+    """pa_decode_append_overlapped (the kernel may start during the preceding
+    kernel's tail) returns the bits of pa_decode_append, also when its launches
+    follow each other back to back and inside a CUDA graph."""
+    batch = synth.llama8b()
+    ref = GpuBatch(batch, fused=True)
+    want = ref.run().clone()
+    del ref
+    g = GpuBatch(batch, fused=True)
+    g.step.overlapped = True
+    for _ in range(3):  # each launch follows the previous one on the stream
+        g.step.append()
+    torch.cuda.synchronize()
+    assert torch.equal(g.step.out.view(torch.int16), want.view(torch.int16))
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            g.step.append()
+            g.step.append()
+    torch.cuda.current_stream().wait_stream(s)
+    g.step.out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(g.step.out.view(torch.int16), want.view(torch.int16))
+    _status_clean()
+
+
 def test_fused_write_reports_bad_slots():
     batch = synth.small_random(16, 3, [40, 70, 9], 8, 2, 128, 16, 20, "bf16")
     g = GpuBatch(batch, fused=True)
