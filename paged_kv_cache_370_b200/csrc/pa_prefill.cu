@@ -452,7 +452,12 @@ namespace t5 {
 constexpr int kM = 128;        // query rows per group (tcgen05 M)
 constexpr int kGroups = 2;
 constexpr int kN = 64;         // keys per tile
-constexpr int kStages = 2;
+// K/V ring depth and P buffers per group (3 x 1 or 2 x 2 fit the 227 KB limit)
+#ifndef PA_PREFILL_TC_STAGES
+#define PA_PREFILL_TC_STAGES 3
+#endif
+constexpr int kStages = PA_PREFILL_TC_STAGES;
+constexpr int kPBufs = kStages >= 3 ? 1 : 2;
 constexpr int kThreads = (2 + 4 * kGroups) * 32;
 constexpr uint32_t kTmemCols = 512;  // group g: S buffers at 256g + {0, 64}, O at 256g + 128
 constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
@@ -467,7 +472,7 @@ struct Lay {
   static constexpr int kPBytes = kM * 128;                    // 128 rows x 64 keys
   static constexpr int kRingOff = kQBytes;
   static constexpr int kPOff = kRingOff + kStages * kStageBytes;  // [group][buffer]
-  static constexpr int kBarOff = kPOff + kGroups * 2 * kPBytes;
+  static constexpr int kBarOff = kPOff + kGroups * kPBufs * kPBytes;
   // full[S] empty[S] q_ready mma_done, then per group s_full[2] s_free[2] p_full[2] pv_done[2]
   static constexpr int kNumBars = 2 * kStages + 2 + 8 * kGroups;
   static constexpr int kTmemOff = kBarOff + kNumBars * 8;
@@ -646,7 +651,8 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
 #pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk)
               umma_f16(tmem + g * 256 + 128,
-                       umma_desc_sw128(p_sm + (g * 2 + (jp & 1)) * L::kPBytes + kk * 32, 16, 1024),
+                       umma_desc_sw128(p_sm + (g * t5::kPBufs + jp % t5::kPBufs) * L::kPBytes + kk * 32,
+                                       16, 1024),
                        umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
                        kIdescO, jp > 0 || kk > 0);
             umma_commit(pv_done(g, jp & 1));
@@ -757,10 +763,15 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       }
       if (grow) m_ref = mx;
       const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
-      // this tile's P row -> P buffer (grp, sb), free once P_{j-2} V_{j-2} is done;
-      // weight = 2^(s * scale_log2 - m_ref), one FMA and one exp2 per key
-      if (j >= 2) wait_bounded(pv_done(grp, sb), ((j - 2) / 2) & 1, abort_flag);
-      unsigned char *prow = smem + L::kPOff + (grp * 2 + sb) * L::kPBytes + r * 128;
+      // this tile's P row -> the group's P buffer; weight = 2^(s * scale_log2 - m_ref),
+      // one FMA and one exp2 per key
+      // (one buffer: free once P_{j-1} V_{j-1} is done; two: once P_{j-2} V_{j-2} is)
+      if (j >= t5::kPBufs) {
+        const int jr = j - t5::kPBufs;
+        wait_bounded(pv_done(grp, jr & 1), (jr / 2) & 1, abort_flag);
+      }
+      unsigned char *prow =
+          smem + L::kPOff + (grp * t5::kPBufs + j % t5::kPBufs) * L::kPBytes + r * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t w[4];
