@@ -52,7 +52,6 @@ namespace {
 __device__ int g_prefill_error;
 
 constexpr int kQTile = 64;       // query tokens per CTA
-constexpr int kKTile = 64;       // keys per stage
 constexpr int kWarps = 4;        // consumer warps, 16 query rows each
 constexpr int kThreads = (kWarps + 1) * 32;
 constexpr int kStages = 2;
@@ -122,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const PrefillParams p) {
   using L = Layout<D>;
+  constexpr int kKTile = 64;      // keys per stage
   constexpr int KSTEPS = D / 16;  // k-steps of Q K^T
   constexpr int NT_O = D / 8;     // n-tiles of the output row block
 
@@ -840,6 +840,7 @@ pa_status launch(const PrefillParams &prm, const void *k_cache, const void *v_ca
                  pa_dtype dtype, cudaStream_t stream) {
   using L = Layout<D>;
   CUtensorMap tk, tv;
+  constexpr int kKTile = 64;  // keys per stage
   const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
   const int box_rows = prm.block_size < kKTile ? prm.block_size : kKTile;
   if (!pa_internal_pool_tensor_map(&tk, k_cache, rows, D, box_rows, dtype) ||
