@@ -76,6 +76,9 @@ def parse_args():
     ap.add_argument("--no-fuse", action="store_true",
                     help="separate KV-write kernel instead of pa_decode_append")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--round-reps", type=int, default=4,
+                    help="each captured round holds this many steps of every rotated batch "
+                         "(device-resident and host-fed timing alike)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -204,7 +207,9 @@ def _workload_config(args, batches, pt):
                 "batches_rotated": len(batches),
                 "l2": f"inputs larger than L2: {len(batches)} rotating batches, "
                       f"{sum(decode_step_bytes(x.context_lens, 32, 8, 128, 16)['kv'] for x in batches) / 1e9:.2f} GB of KV",
-                "timing": "CUDA graphs replayed back to back; CUDA events on the stream",
+                "timing": f"CUDA graphs of {len(batches) * max(1, args.round_reps)} steps "
+                          "(the batches in rotation) replayed back to back; CUDA events "
+                          "on the stream",
                 "launch": ("plain stream order" if args.no_overlap or args.no_fuse else
                            "programmatic early start: each decode kernel's start-up overlaps "
                            "the previous kernel's tail (pa_decode_append_overlapped)")}
@@ -381,10 +386,13 @@ def run_ours(args, rank, world, local, dist):
         pre(s) if has_pre(s) else None
         s.append() if s.fused else s.attend()
 
-    # one graph per round: a step of every batch, back to back (a serving loop
-    # launches a whole decode step as one graph); and the decode launches alone
-    g_round = capture(lambda: [one_step(s) for s in steps], torch)
-    g_dec_only = capture(lambda: [s.append() if s.fused else s.attend() for s in steps], torch)
+    # one graph per round: round_reps steps of every batch in rotation, back to
+    # back (a serving loop launches whole decode steps as graphs); and the decode
+    # launches alone
+    R = V * max(1, args.round_reps)
+    g_round = capture(lambda: [one_step(steps[i % V]) for i in range(R)], torch)
+    g_dec_only = capture(lambda: [s.append() if s.fused else s.attend()
+                                  for s in (steps[i % V] for i in range(R))], torch)
 
     def barrier():
         if dist is not None:
@@ -392,14 +400,14 @@ def run_ours(args, rank, world, local, dist):
         torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
-    for i in range(max(1, args.warmup // V)):
+    for i in range(max(1, args.warmup // R)):
         g_round.replay()
-    for i in range(args.warmup % V):
+    for i in range(args.warmup % R):
         if g_write[i % V] is not None:
             g_write[i % V].replay()
         g_dec[i % V].replay()
     K = args.steps
-    rounds, rest = divmod(K, V)
+    rounds, rest = divmod(K, R)
     props = torch.cuda.get_device_properties(device)
     bus = getattr(props, "pci_bus_id", None)
     bus_str = None
@@ -427,14 +435,14 @@ def run_ours(args, rank, world, local, dist):
     sampler.stop()
     total_ms = start_ev.elapsed_time(end_ev)
     # ---- per-kernel durations (same launches, separately timed with events)
-    reps = max(1, min(200, K // V))
+    reps = max(1, min(50, K // R))
     ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ka.record(stream)
     for _ in range(reps):
         g_dec_only.replay()
     kb.record(stream)
     torch.cuda.synchronize()
-    dec_ms = [ka.elapsed_time(kb) / (reps * V)]
+    dec_ms = [ka.elapsed_time(kb) / (reps * R)]
     pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     wr_ms = [0.0]
     if any(g is not None for g in g_write):
@@ -503,44 +511,54 @@ def run_ours(args, rank, world, local, dist):
 
 
 def run_e2e(args, steps, infos, torch, device, dist, world):
-    """The same steps fed from pinned host buffers, output copied back, graph-replayed."""
-    from paged_kv_cache_370_b200.step import HostDecodeStep
-    hsteps = []
-    for s in steps:
-        hsteps.append(HostDecodeStep(k_cache=s.k_cache, v_cache=s.v_cache, q=s.q, k_new=s.k_new,
-                                     v_new=s.v_new, slot_mapping=s.slot_mapping,
-                                     block_tables=s.block_tables, context_lens=s.context_lens,
-                                     max_context_len=s.max_context_len, scale=s.scale,
-                                     partition_tokens=s.partition_tokens,
-                                     copy_pairs=s.copy_pairs, fused=s.fused))
-    graphs = [capture(h.run, torch) for h in hsteps]
-    g_round = capture(lambda: [h.run() for h in hsteps], torch)
-    V = len(graphs)
-    for i in range(max(1, args.warmup // V)):
-        g_round.replay()
+    """The same steps fed from pinned host buffers through the library's
+    HostStepPipeline: two rounds of R host-fed steps taking turns, each round's
+    uploads, kernels and downloads replayed as graphs on three streams."""
+    from paged_kv_cache_370_b200.step import HostDecodeStep, HostStepPipeline
+    V = len(steps)
+    R = V * max(1, args.round_reps)
+
+    def host_step(s):
+        return HostDecodeStep(k_cache=s.k_cache, v_cache=s.v_cache, q=s.q, k_new=s.k_new,
+                              v_new=s.v_new, slot_mapping=s.slot_mapping,
+                              block_tables=s.block_tables, context_lens=s.context_lens,
+                              max_context_len=s.max_context_len, scale=s.scale,
+                              partition_tokens=s.partition_tokens, copy_pairs=s.copy_pairs,
+                              fused=s.fused, window=s.window, overlapped=s.overlapped)
+
+    rounds = [[host_step(steps[i % V]) for i in range(R)] for _ in range(2)]
+    pipe = HostStepPipeline(rounds)
+    pipe.capture()
+    # a step count that is not a whole number of rounds ends with serial host steps
+    tail = [capture(h.run, torch) for h in rounds[0][:V]]
+    pipe.run(max(2, args.warmup // R))
+    torch.cuda.synchronize()
     K = args.steps
-    rounds, rest = divmod(K, V)
+    n_rounds, rest = divmod(K, R)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for _ in range(rounds):
-        g_round.replay()
+    pipe.run(n_rounds)
     for i in range(rest):
-        graphs[i].replay()
+        tail[i % V].replay()
     b.record()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     my_bytes = sum(infos[i % V]["decode"]["total"] for i in range(K))
     ms, total = rank_aggregate(a.elapsed_time(b), float(my_bytes), dist, device)
+    h0 = rounds[0]
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms / K, 5),
-            "h2d_bytes_per_step": int(np.mean([hsteps[i % V].h2d_bytes for i in range(K)])),
-            "d2h_bytes_per_step": int(hsteps[0].d2h_bytes),
-            "how": "pinned host inputs copied in and output copied out every step, "
-                   "graph-replayed through the library's HostDecodeStep"}
+            "h2d_bytes_per_step": int(np.mean([h0[i % V].h2d_bytes for i in range(K)])),
+            "d2h_bytes_per_step": int(h0[0].d2h_bytes),
+            "how": "pinned host inputs copied in and output copied out every step through the "
+                   f"library's HostStepPipeline: rounds of {R} steps, each round's uploads, "
+                   "kernels and downloads replayed as CUDA graphs on three streams, the next "
+                   "round's uploads and the previous round's downloads under this round's "
+                   "kernels"}
 
 
 # --------------------------------------------------------------------------- CPU (oracle)

@@ -11,6 +11,8 @@ paged attention of each sequence's query over its whole history ("å¤§è¯­è¨€æ¨¡åž
 the library's kernels on the current stream. ``HostDecodeStep`` is the same
 step fed from pinned host buffers: it copies the step's inputs to the device,
 runs the step and copies the output back, all stream-ordered.
+``HostStepPipeline`` runs many host-fed steps with their copies hidden under
+other steps' kernels.
 """
 from __future__ import annotations
 
@@ -125,7 +127,8 @@ class HostDecodeStep:
 
     def __init__(self, *, k_cache, v_cache, q, k_new, v_new, slot_mapping, block_tables,
                  context_lens, max_context_len: int, scale: float, partition_tokens: int = 0,
-                 copy_pairs=None, fused: bool = False, window: int = 0):
+                 copy_pairs=None, fused: bool = False, window: int = 0,
+                 overlapped: bool = False):
         dev = k_cache.device
         parts = {"q": q, "k_new": k_new, "v_new": v_new, "slot_mapping": slot_mapping,
                  "block_tables": block_tables, "context_lens": context_lens}
@@ -150,8 +153,11 @@ class HostDecodeStep:
                                context_lens=views["context_lens"],
                                max_context_len=max_context_len, scale=scale,
                                partition_tokens=partition_tokens,
-                               copy_pairs=views.get("copy_pairs"), fused=fused, window=window)
+                               copy_pairs=views.get("copy_pairs"), fused=fused, window=window,
+                               overlapped=overlapped)
         self.h_out = torch.empty(tuple(q.shape), dtype=q.dtype).pin_memory()
+        self._in_ready = torch.cuda.Event()
+        self._done = torch.cuda.Event()
 
     @property
     def h2d_bytes(self) -> int:
@@ -169,3 +175,124 @@ class HostDecodeStep:
         out = self.step.run()
         self.h_out.copy_(out, non_blocking=True)
         return self.h_out
+
+    def enqueue(self, copy_in, compute, copy_out):
+        """The same step spread over three streams so that consecutive steps overlap:
+        the upload on ``copy_in``, the kernels on ``compute`` once the upload landed,
+        the download on ``copy_out`` once the kernels finished. Steps enqueued one
+        after another on the same three streams pipeline: the next step's upload and
+        the previous step's download run under this step's kernels, while the
+        kernels themselves stay in order on ``compute`` (each step reads the pools
+        the previous one wrote). The caller must not enqueue the same step again
+        before its previous use completed (its buffers are reused); ``h_out`` holds
+        the result once ``copy_out`` has passed this point."""
+        with torch.cuda.stream(copy_in):
+            self.d_in.copy_(self.h_in, non_blocking=True)
+            self._in_ready.record(copy_in)
+        compute.wait_event(self._in_ready)
+        with torch.cuda.stream(compute):
+            self.step.run()
+            self._done.record(compute)
+        copy_out.wait_event(self._done)
+        with torch.cuda.stream(copy_out):
+            self.h_out.copy_(self.step.out, non_blocking=True)
+        return self.h_out
+
+    def upload(self):
+        self.d_in.copy_(self.h_in, non_blocking=True)
+
+    def download(self):
+        self.h_out.copy_(self.step.out, non_blocking=True)
+
+
+class HostStepPipeline:
+    """Host-fed steps run back to back with every copy under some step's kernels.
+
+    The steps come in two sets (rounds) that take turns. Each round has three
+    CUDA graphs: the uploads of its steps' inputs, its steps' kernels, and the
+    downloads of its steps' outputs. ``run`` replays them on three streams so that
+    round r+1's uploads and round r-1's downloads run while round r's kernels do.
+    Because the graph of kernels has no copy nodes in it, each decode kernel keeps
+    its programmatic dependency on the one before it (the early start of an
+    ``overlapped`` step). Rounds' kernels run in order on the caller's stream, so
+    the steps see the pools in the order given.
+
+    A round's buffers are reused two rounds later: its uploads wait for its
+    previous kernels to finish, and its kernels for its previous downloads."""
+
+    def __init__(self, rounds):
+        if len(rounds) != 2 or not all(rounds):
+            raise ValueError("two non-empty rounds of HostDecodeStep are needed")
+        self.rounds = [list(r) for r in rounds]
+        self.s_in = torch.cuda.Stream()
+        self.s_out = torch.cuda.Stream()
+        self._graphs = None
+        self._up = [torch.cuda.Event() for _ in range(2)]
+        self._comp = [torch.cuda.Event() for _ in range(2)]
+        self._down = [torch.cuda.Event() for _ in range(2)]
+
+    @property
+    def steps_per_round(self):
+        return [len(r) for r in self.rounds]
+
+    def launches(self, round_index: int) -> int:
+        return sum(h.launches() for h in self.rounds[round_index])
+
+    def capture(self):
+        """Capture the six graphs (after one eager pass that warms every launch path)."""
+        cur = torch.cuda.current_stream()
+        side = torch.cuda.Stream()
+        side.wait_stream(cur)
+        phases = []
+        with torch.cuda.stream(side):
+            for r in self.rounds:
+                for h in r:
+                    h.upload()
+                for h in r:
+                    h.step.run()
+                for h in r:
+                    h.download()
+            torch.cuda.synchronize()
+            for r in self.rounds:
+                gs = []
+                for fn in (lambda r=r: [h.upload() for h in r],
+                           lambda r=r: [h.step.run() for h in r],
+                           lambda r=r: [h.download() for h in r]):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=side):
+                        fn()
+                    gs.append(g)
+                phases.append(gs)
+        cur.wait_stream(side)
+        torch.cuda.synchronize()
+        self._graphs = phases
+        # nothing is in flight: every round's buffers are free
+        for e in self._comp + self._down:
+            e.record(cur)
+
+    def run(self, n_rounds: int):
+        """Enqueue ``n_rounds`` rounds (alternating sets) on the current stream and
+        the two copy streams; on return the current stream is ordered after every
+        copy. Results are in each step's ``h_out`` once the stream passes."""
+        if self._graphs is None:
+            self.capture()
+        cs = torch.cuda.current_stream()
+        self.s_in.wait_stream(cs)
+        self.s_out.wait_stream(cs)
+        for i in range(n_rounds):
+            x = i % 2
+            up, comp, down = self._graphs[x]
+            self.s_in.wait_event(self._comp[x])
+            with torch.cuda.stream(self.s_in):
+                up.replay()
+            self._up[x].record(self.s_in)
+            cs.wait_event(self._up[x])
+            cs.wait_event(self._down[x])
+            comp.replay()
+            self._comp[x].record(cs)
+            self.s_out.wait_event(self._comp[x])
+            with torch.cuda.stream(self.s_out):
+                down.replay()
+            self._down[x].record(self.s_out)
+        cs.wait_stream(self.s_in)
+        cs.wait_stream(self.s_out)
