@@ -447,6 +447,44 @@ pa_status pa_alloc_fill_tables(const pa_alloc *a, const int64_t *seq_ids, int n,
                                int32_t *block_tables, int max_blocks_per_seq, int32_t pad,
                                int32_t *context_lens);
 
+/* Prefix caching of full blocks [P3, section "分页还顺带解决了什么": requests
+ * whose prompts begin alike point their first blocks at the same physical
+ * blocks; only blocks that are completely filled are shared; P1, section 9:
+ * a common prompt prefix's KV is cached].
+ *
+ * pa_alloc_add_seq_cached adds a sequence holding the prompt tokens[0 ..
+ * num_tokens) (token ids; only compared for equality). Its leading full
+ * blocks are looked up: logical block i is shared when a cached block holds
+ * exactly tokens[0 .. (i+1) * block_size) (the same ids in the same order,
+ * from position 0). The lookup covers the full blocks that lie within the
+ * first num_tokens - 1 tokens, so at least the last prompt token is always
+ * left to compute, and stops at the first block that is not cached. Shared
+ * blocks gain a reference; the rest are taken from the free list. Then every
+ * full block the prompt fills that is not yet cached under its prefix is
+ * registered (a prefix is cached on one block at most). *num_cached_tokens =
+ * shared blocks * block_size: the positions whose K/V are already in the
+ * pool. The caller writes positions [*num_cached_tokens, num_tokens) (e.g.
+ * pa_reshape_and_cache) before any kernel reads them; a request added later
+ * in the same step may share these blocks, and stream order makes the write
+ * land first. Tokens appended by pa_alloc_append_slot are not registered.
+ * All or nothing: PA_ERR_OUT_OF_BLOCKS leaves the state unchanged.
+ *
+ * A cached block whose last reference is dropped (pa_alloc_free_seq,
+ * pa_alloc_slide_window, pa_alloc_swap_out) keeps its contents and stays
+ * cached, counted as free. Blocks are taken first from the free blocks that
+ * hold no cached prefix; when there are none, the cached free block released
+ * longest ago is reused, and only its own prefix is forgotten: a longer
+ * prefix still cached on another block is found again once a request caches
+ * the shorter one anew.
+ *
+ * pa_alloc_cached_blocks: blocks holding a cached prefix, and how many of
+ * those are free (evictable). pa_alloc_reset_prefix_cache forgets every
+ * cached prefix (the blocks themselves are untouched). */
+pa_status pa_alloc_add_seq_cached(pa_alloc *a, int64_t seq_id, const int32_t *tokens,
+                                  int num_tokens, int *num_cached_tokens);
+pa_status pa_alloc_cached_blocks(const pa_alloc *a, int *cached_blocks, int *cached_free_blocks);
+pa_status pa_alloc_reset_prefix_cache(pa_alloc *a);
+
 pa_status pa_alloc_ref_count(const pa_alloc *a, int32_t block, int *ref_count);
 
 /* Free blocks; token slots that hold a token; allocated slots that do not

@@ -34,13 +34,27 @@ It restates, one step at a time, what the pages say a block manager does:
   host count = the group's references), the device block loses those
   references, and the tables then name host blocks; swapping in is the
   mirror image. A block also used outside the group stays where it is for
-  the others, so the group gets its own copy.
+  the others, so the group gets its own copy;
+* prefix caching: requests whose prompts begin with the same tokens point
+  their first blocks at the same physical blocks, and only completely
+  filled blocks are shared (third page, section "分页还顺带解决了什么"); the
+  KV of a common prompt prefix is kept as a cache (first page, section 9).
+  Here a cached block stands for the whole token prefix up to its end. A
+  new prompt shares, from its start, every full block whose prefix is
+  cached, except that the block holding the prompt's last token is never
+  looked up (that token's attention must be computed); then each full block
+  of the prompt whose prefix is not cached yet is recorded. A cached block
+  nobody uses any more stays cached and counts as free; it is reused only
+  when no plain free block is left, the one released longest ago first, and
+  only its own prefix is then forgotten.
 
 Which physical id the free list hands out is not fixed by the pages; this
 model pops the most recently freed block (a LIFO stack). Tests compare the
 product allocator with this model only up to a relabelling of ids.
 """
 from __future__ import annotations
+
+from collections import OrderedDict
 
 
 RELEASED = -1  # table entry of a block given back by the sliding window
@@ -67,6 +81,10 @@ class BlockManagerModel:
         self.swapped: set[int] = set()
         self.host_free: list[int] = []
         self.host_ref: list[int] = []
+        # prefix cache: token prefix (whole blocks) -> the block holding its last block
+        self.cached: dict[tuple, int] = {}
+        self.prefix_of: dict[int, tuple] = {}
+        self.idle: OrderedDict[int, None] = OrderedDict()  # unused cached blocks, oldest first
 
     # -- allocation ---------------------------------------------------------------------------
     def _blocks_for(self, num_tokens: int) -> int:
@@ -74,11 +92,23 @@ class BlockManagerModel:
         return -(-num_tokens // self.block_size)
 
     def _pop(self) -> int:
-        if not self.free:
+        if self.free:
+            blk = self.free.pop()
+        elif self.idle:
+            blk = next(iter(self.idle))  # the unused cached block released longest ago
+            del self.idle[blk]
+            del self.cached[self.prefix_of.pop(blk)]
+        else:
             raise OutOfBlocks("free list is empty")
-        blk = self.free.pop()
         self.ref[blk] = 1
         return blk
+
+    def _release(self, blk: int):
+        """blk's last reference is gone."""
+        if blk in self.prefix_of:
+            self.idle[blk] = None
+        else:
+            self.free.append(blk)
 
     def add_seq(self, seq: int, num_tokens: int) -> list[int]:
         """A new request: take the blocks its prompt needs, all or none."""
@@ -87,11 +117,53 @@ class BlockManagerModel:
         if num_tokens < 0:
             raise ValueError("negative length")
         need = self._blocks_for(num_tokens)
-        if need > len(self.free):
-            raise OutOfBlocks(f"need {need} blocks, {len(self.free)} free")
+        if need > self.num_free():
+            raise OutOfBlocks(f"need {need} blocks, {self.num_free()} free")
         self.tables[seq] = [self._pop() for _ in range(need)]
         self.lens[seq] = num_tokens
         return list(self.tables[seq])
+
+    def add_seq_cached(self, seq: int, tokens) -> int:
+        """A new request with prompt ``tokens``: share its cached leading full
+        blocks, take the rest from the free list (all or none), record its full
+        blocks. Returns the number of positions already held (shared blocks x
+        block size)."""
+        if seq in self.tables:
+            raise BadState(f"sequence {seq} exists")
+        tokens = [int(t) for t in tokens]
+        n, bs = len(tokens), self.block_size
+        shared = []
+        for i in range(max(n - 1, 0) // bs):  # full blocks before the last token
+            blk = self.cached.get(tuple(tokens[:(i + 1) * bs]))
+            if blk is None:
+                break
+            shared.append(blk)
+        need = self._blocks_for(n) - len(shared)
+        unused = sum(1 for b in shared if self.ref[b] == 0)  # counted as free until shared
+        if need > self.num_free() - unused:
+            raise OutOfBlocks(f"need {need} blocks, {self.num_free() - unused} free")
+        for b in shared:
+            self.idle.pop(b, None)
+            self.ref[b] += 1
+        table = shared + [self._pop() for _ in range(need)]
+        for i in range(len(shared), n // bs):
+            key = tuple(tokens[:(i + 1) * bs])
+            if key not in self.cached:
+                self.cached[key] = table[i]
+                self.prefix_of[table[i]] = key
+        self.tables[seq] = table
+        self.lens[seq] = n
+        return len(shared) * bs
+
+    def cached_blocks(self):
+        """(blocks holding a cached prefix, of which unused)."""
+        return len(self.cached), len(self.idle)
+
+    def reset_prefix_cache(self):
+        self.free.extend(self.idle)
+        self.idle.clear()
+        self.cached.clear()
+        self.prefix_of.clear()
 
     def fork(self, parent: int, child: int):
         """The child shares every block of the parent; each gains a reference."""
@@ -132,7 +204,8 @@ class BlockManagerModel:
         go back on the free list."""
         if seq not in self.tables:
             raise BadState(f"no sequence {seq}")
-        ref, free = (self.host_ref, self.host_free) if seq in self.swapped else (self.ref, self.free)
+        host = seq in self.swapped
+        ref = self.host_ref if host else self.ref
         for blk in reversed(self.tables.pop(seq)):
             if blk == RELEASED:
                 continue
@@ -140,7 +213,10 @@ class BlockManagerModel:
                 raise BadState("reference count underflow")
             ref[blk] -= 1
             if ref[blk] == 0:
-                free.append(blk)
+                if host:
+                    self.host_free.append(blk)
+                else:
+                    self._release(blk)
         del self.lens[seq]
         self.swapped.discard(seq)
 
@@ -161,7 +237,7 @@ class BlockManagerModel:
             table[i] = RELEASED
             self.ref[blk] -= 1
             if self.ref[blk] == 0:
-                self.free.append(blk)
+                self._release(blk)
                 freed += 1
         return freed
 
@@ -189,17 +265,21 @@ class BlockManagerModel:
                     refs[blk] = 0
                     order.append(blk)
                 refs[blk] += 1
-        src_ref, src_free = (self.ref, self.free) if out else (self.host_ref, self.host_free)
-        dst_ref, dst_free = (self.host_ref, self.host_free) if out else (self.ref, self.free)
-        if len(order) > len(dst_free):
-            raise OutOfBlocks(f"need {len(order)} blocks on the other side, {len(dst_free)} free")
+        src_ref = self.ref if out else self.host_ref
+        dst_ref = self.host_ref if out else self.ref
+        room = len(self.host_free) if out else self.num_free()
+        if len(order) > room:
+            raise OutOfBlocks(f"need {len(order)} blocks on the other side, {room} free")
         moved, pairs = {}, []
         for blk in order:
-            new = dst_free.pop()
+            new = self.host_free.pop() if out else self._pop()
             dst_ref[new] = refs[blk]
             src_ref[blk] -= refs[blk]
             if src_ref[blk] == 0:
-                src_free.append(blk)
+                if out:
+                    self._release(blk)
+                else:
+                    self.host_free.append(blk)
             moved[blk] = new
             pairs.append((blk, new))
         for s in seqs:
@@ -233,7 +313,7 @@ class BlockManagerModel:
         return list(self.tables[seq])
 
     def num_free(self) -> int:
-        return len(self.free)
+        return len(self.free) + len(self.idle)
 
     def stats(self):
         """(free blocks, token slots holding a valid token, slots allocated but empty).
@@ -250,6 +330,6 @@ class BlockManagerModel:
                     continue
                 f = min(self.block_size, n - i * self.block_size)
                 filled[blk] = max(filled.get(blk, 0), max(f, 0))
-        used_blocks = self.num_blocks - len(self.free)
+        used_blocks = self.num_blocks - self.num_free()
         used_tokens = sum(filled.values())
-        return len(self.free), used_tokens, used_blocks * self.block_size - used_tokens
+        return self.num_free(), used_tokens, used_blocks * self.block_size - used_tokens

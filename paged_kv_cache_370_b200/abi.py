@@ -90,6 +90,9 @@ def _load() -> ctypes.CDLL:
         "pa_alloc_swap_in": (i, [P, P, i, P, i, P]),
         "pa_alloc_is_swapped": (i, [P, i64, P]),
         "pa_alloc_host_free": (i, [P, P]),
+        "pa_alloc_add_seq_cached": (i, [P, i64, P, i, P]),
+        "pa_alloc_cached_blocks": (i, [P, P, P]),
+        "pa_alloc_reset_prefix_cache": (i, [P]),
         "pa_alloc_block_table": (i, [P, i64, P, i, P, P]),
         "pa_alloc_fill_tables": (i, [P, P, i, P, i, ctypes.c_int32, P]),
         "pa_alloc_ref_count": (i, [P, ctypes.c_int32, P]),
@@ -415,6 +418,27 @@ class BlockManager:
 
     def add_seq(self, seq_id: int, num_tokens: int):
         _check(_lib.pa_alloc_add_seq(self._h, seq_id, num_tokens), "pa_alloc_add_seq")
+
+    def add_seq_cached(self, seq_id: int, tokens) -> int:
+        """A new sequence holding the prompt ``tokens`` (token ids), sharing the
+        leading full blocks whose whole prefix is cached; returns how many
+        positions are already in the pool (the caller writes the rest)."""
+        tok = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32).reshape(-1))
+        n = ctypes.c_int(0)
+        _check(_lib.pa_alloc_add_seq_cached(self._h, seq_id, _np_ptr(tok) if len(tok) else None,
+                                            len(tok), ctypes.byref(n)),
+               "pa_alloc_add_seq_cached")
+        return n.value
+
+    def cached_blocks(self) -> tuple[int, int]:
+        """(blocks holding a cached prefix, of which free)."""
+        c, f = ctypes.c_int(0), ctypes.c_int(0)
+        _check(_lib.pa_alloc_cached_blocks(self._h, ctypes.byref(c), ctypes.byref(f)),
+               "pa_alloc_cached_blocks")
+        return c.value, f.value
+
+    def reset_prefix_cache(self):
+        _check(_lib.pa_alloc_reset_prefix_cache(self._h), "pa_alloc_reset_prefix_cache")
 
     def fork(self, parent: int, child: int):
         _check(_lib.pa_alloc_fork(self._h, parent, child), "pa_alloc_fork")

@@ -14,10 +14,23 @@
 //
 // The free list is a LIFO stack of block ids: a freed block is the next one
 // handed out, which keeps recently used blocks warm in L2.
+//
+// Prefix caching ("大语言模型推理内存管理算法 paged attention", section 9;
+// "08. PagedAttention：把 KV Cache 分页管理", section "分页还顺带解决了什么":
+// requests whose prompts begin alike share their first, completely filled
+// blocks). A cached block stands for one token prefix: every token from
+// position 0 to the end of the block. The prefixes form a trie whose nodes are
+// keyed by (parent node, the block's own tokens) and checked in full on every
+// lookup, so a hit never rests on the hash alone; a node may have no block
+// (its block was reused) while longer prefixes below it are still cached. A
+// cached block whose last reference goes keeps its contents and waits,
+// counted as free, in a list ordered by release time; it is reused (oldest
+// first) only when no plain free block is left.
 
 #include "pa.h"
 
 #include <algorithm>
+#include <cstring>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -38,19 +51,156 @@ struct Sequence {
 struct pa_alloc {
   int num_blocks = 0;
   int block_size = 0;
-  std::vector<int32_t> free_stack;  // back() is handed out next
+  std::vector<int32_t> free_stack;  // free blocks holding no cached prefix; back() next
   std::vector<int32_t> ref_count;   // per physical block
   std::unordered_map<int64_t, Sequence> seqs;
   std::vector<int32_t> host_free;   // host swap-space blocks, back() handed out next
   std::vector<int32_t> host_ref;    // per host block
 
-  int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
+  // ---- prefix cache: a trie of token prefixes, one node per distinct
+  // prefix of whole blocks that is cached or has a cached extension
+  struct Node {
+    int64_t parent = -1;  // the node of the prefix one block shorter; -1 at the root
+    int32_t block = -1;   // the block holding this prefix's last block_size tokens, or -1
+    int32_t children = 0;
+  };
+  std::vector<Node> nodes;
+  std::vector<int32_t> node_tokens;     // [node][block_size]: the node's own tokens
+  std::vector<int64_t> spare_nodes;     // deleted node slots
+  std::unordered_multimap<uint64_t, int64_t> index;  // key hash -> node
+  std::vector<int64_t> node_of;         // per block: its node, or -1
+  int64_t cached = 0;                   // blocks holding a cached prefix
+  // free cached blocks, oldest release first: an intrusive list through lru_next/lru_prev
+  std::vector<int32_t> lru_prev, lru_next;
+  int32_t lru_head = -1, lru_tail = -1;
+  int64_t lru_size = 0;
 
-  int32_t pop() {
-    int32_t b = free_stack.back();
-    free_stack.pop_back();
+  int64_t blocks_for(int64_t tokens) const { return (tokens + block_size - 1) / block_size; }
+  int64_t num_free() const { return (int64_t)free_stack.size() + lru_size; }
+  bool cache_ready() const { return !node_of.empty(); }
+
+  void cache_init() {
+    if (cache_ready()) return;
+    node_of.assign(num_blocks, -1);
+    lru_prev.assign(num_blocks, -1);
+    lru_next.assign(num_blocks, -1);
+  }
+
+  // FNV-1a (Fowler, Noll, Vo) over the parent node and the block's tokens.
+  uint64_t key_hash(int64_t parent, const int32_t *tok) const {
+    uint64_t h = 1469598103934665603ull;
+    auto eat = [&h](const void *p, size_t n) {
+      const unsigned char *c = static_cast<const unsigned char *>(p);
+      for (size_t i = 0; i < n; ++i) {
+        h ^= c[i];
+        h *= 1099511628211ull;
+      }
+    };
+    eat(&parent, sizeof parent);
+    eat(tok, sizeof(int32_t) * (size_t)block_size);
+    return h;
+  }
+
+  const int32_t *tokens_of(int64_t n) const { return &node_tokens[(size_t)n * block_size]; }
+
+  // The node for (parent, tok), or -1; the key is checked in full.
+  int64_t find(int64_t parent, const int32_t *tok) const {
+    if (!cache_ready()) return -1;
+    auto range = index.equal_range(key_hash(parent, tok));
+    for (auto it = range.first; it != range.second; ++it) {
+      const int64_t n = it->second;
+      if (nodes[n].parent == parent &&
+          std::memcmp(tokens_of(n), tok, sizeof(int32_t) * block_size) == 0)
+        return n;
+    }
+    return -1;
+  }
+
+  int64_t find_or_add(int64_t parent, const int32_t *tok) {
+    int64_t n = find(parent, tok);
+    if (n >= 0) return n;
+    if (!spare_nodes.empty()) {
+      n = spare_nodes.back();
+      spare_nodes.pop_back();
+    } else {
+      n = (int64_t)nodes.size();
+      nodes.emplace_back();
+      node_tokens.resize(node_tokens.size() + block_size);
+    }
+    nodes[n] = Node{parent, -1, 0};
+    std::memcpy(&node_tokens[(size_t)n * block_size], tok, sizeof(int32_t) * block_size);
+    index.emplace(key_hash(parent, tok), n);
+    if (parent >= 0) nodes[parent].children += 1;
+    return n;
+  }
+
+  // Delete nodes that hold no block and lead to none, from n towards the root.
+  void prune(int64_t n) {
+    while (n >= 0 && nodes[n].block < 0 && nodes[n].children == 0) {
+      auto range = index.equal_range(key_hash(nodes[n].parent, tokens_of(n)));
+      for (auto it = range.first; it != range.second; ++it)
+        if (it->second == n) {
+          index.erase(it);
+          break;
+        }
+      const int64_t up = nodes[n].parent;
+      spare_nodes.push_back(n);
+      if (up >= 0) nodes[up].children -= 1;
+      n = up;
+    }
+  }
+
+  // Block b no longer holds its prefix (it is about to be reused).
+  void uncache(int32_t b) {
+    const int64_t n = node_of[b];
+    nodes[n].block = -1;
+    node_of[b] = -1;
+    --cached;
+    prune(n);
+  }
+
+  void lru_unlink(int32_t b) {
+    if (lru_prev[b] >= 0) lru_next[lru_prev[b]] = lru_next[b]; else lru_head = lru_next[b];
+    if (lru_next[b] >= 0) lru_prev[lru_next[b]] = lru_prev[b]; else lru_tail = lru_prev[b];
+    lru_prev[b] = lru_next[b] = -1;
+    --lru_size;
+  }
+
+  void lru_append(int32_t b) {
+    lru_prev[b] = lru_tail;
+    lru_next[b] = -1;
+    if (lru_tail >= 0) lru_next[lru_tail] = b; else lru_head = b;
+    lru_tail = b;
+    ++lru_size;
+  }
+
+  // A free block with reference count 1. The caller checked num_free() > 0.
+  int32_t take() {
+    int32_t b;
+    if (!free_stack.empty()) {
+      b = free_stack.back();
+      free_stack.pop_back();
+    } else {
+      b = lru_head;  // the cached block released longest ago
+      lru_unlink(b);
+      uncache(b);
+    }
     ref_count[b] = 1;
     return b;
+  }
+
+  // Block b's count has just reached zero.
+  void release(int32_t b) {
+    if (cache_ready() && node_of[b] >= 0)
+      lru_append(b);
+    else
+      free_stack.push_back(b);
+  }
+
+  // A cached block gains a reference (leaving the free list if it was there).
+  void reuse(int32_t b) {
+    if (ref_count[b] == 0) lru_unlink(b);
+    ref_count[b] += 1;
   }
 };
 
@@ -75,12 +225,81 @@ pa_status pa_alloc_add_seq(pa_alloc *a, int64_t seq_id, int num_tokens) {
   if (!a || num_tokens < 0) return PA_ERR_INVALID;
   if (a->seqs.count(seq_id)) return PA_ERR_STATE;
   int64_t need = a->blocks_for(num_tokens);
-  if (need > (int64_t)a->free_stack.size()) return PA_ERR_OUT_OF_BLOCKS;
+  if (need > a->num_free()) return PA_ERR_OUT_OF_BLOCKS;
   Sequence s;
   s.blocks.reserve(need);
-  for (int64_t i = 0; i < need; ++i) s.blocks.push_back(a->pop());
+  for (int64_t i = 0; i < need; ++i) s.blocks.push_back(a->take());
   s.len = num_tokens;
   a->seqs.emplace(seq_id, std::move(s));
+  return PA_OK;
+}
+
+pa_status pa_alloc_add_seq_cached(pa_alloc *a, int64_t seq_id, const int32_t *tokens,
+                                  int num_tokens, int *num_cached_tokens) {
+  if (!a || num_tokens < 0 || (num_tokens && !tokens)) return PA_ERR_INVALID;
+  if (a->seqs.count(seq_id)) return PA_ERR_STATE;
+  a->cache_init();
+  const int bs = a->block_size;
+  const int64_t need = a->blocks_for(num_tokens);
+  // the cached prefix: full blocks within the first num_tokens - 1 tokens, from the start
+  const int64_t lookable = num_tokens > 0 ? (int64_t)(num_tokens - 1) / bs : 0;
+  std::vector<int32_t> hits;
+  int64_t node = -1, idle_hits = 0;
+  for (int64_t i = 0; i < lookable; ++i) {
+    const int64_t n = a->find(node, tokens + i * bs);
+    if (n < 0 || a->nodes[n].block < 0) break;
+    const int32_t b = a->nodes[n].block;
+    hits.push_back(b);
+    if (a->ref_count[b] == 0) ++idle_hits;  // counted as free now, not after the reuse
+    node = n;
+  }
+  if (need - (int64_t)hits.size() > a->num_free() - idle_hits) return PA_ERR_OUT_OF_BLOCKS;
+  Sequence s;
+  s.blocks.reserve(need);
+  for (int32_t b : hits) {  // before any take(), so no eviction can reach them
+    a->reuse(b);
+    s.blocks.push_back(b);
+  }
+  for (int64_t i = (int64_t)hits.size(); i < need; ++i) s.blocks.push_back(a->take());
+  // cache the full blocks this prompt fills whose prefix no block holds yet
+  const int64_t full = num_tokens / bs;
+  for (int64_t i = (int64_t)hits.size(); i < full; ++i) {
+    node = a->find_or_add(node, tokens + i * bs);
+    if (a->nodes[node].block >= 0) continue;  // held by another block already
+    a->nodes[node].block = s.blocks[i];
+    a->node_of[s.blocks[i]] = node;
+    ++a->cached;
+  }
+  s.len = num_tokens;
+  a->seqs.emplace(seq_id, std::move(s));
+  if (num_cached_tokens) *num_cached_tokens = (int)((int64_t)hits.size() * bs);
+  return PA_OK;
+}
+
+pa_status pa_alloc_cached_blocks(const pa_alloc *a, int *cached_blocks, int *cached_free_blocks) {
+  if (!a) return PA_ERR_INVALID;
+  if (cached_blocks) *cached_blocks = (int)a->cached;
+  if (cached_free_blocks) *cached_free_blocks = (int)a->lru_size;
+  return PA_OK;
+}
+
+pa_status pa_alloc_reset_prefix_cache(pa_alloc *a) {
+  if (!a) return PA_ERR_INVALID;
+  if (!a->cache_ready()) return PA_OK;
+  for (int32_t b = a->lru_head; b >= 0;) {  // free cached blocks become plain free blocks
+    const int32_t next = a->lru_next[b];
+    a->lru_prev[b] = a->lru_next[b] = -1;
+    a->free_stack.push_back(b);
+    b = next;
+  }
+  a->lru_head = a->lru_tail = -1;
+  a->lru_size = 0;
+  std::fill(a->node_of.begin(), a->node_of.end(), -1);
+  a->nodes.clear();
+  a->node_tokens.clear();
+  a->spare_nodes.clear();
+  a->index.clear();
+  a->cached = 0;
   return PA_OK;
 }
 
@@ -107,14 +326,14 @@ pa_status pa_alloc_append_slot(pa_alloc *a, int64_t seq_id, int64_t *slot, int64
   int64_t src = -1, dst = -1;
   if (logical == (int64_t)s.blocks.size()) {
     // the last block is full (or there is none): take a new one
-    if (a->free_stack.empty()) return PA_ERR_OUT_OF_BLOCKS;
-    s.blocks.push_back(a->pop());
+    if (a->num_free() == 0) return PA_ERR_OUT_OF_BLOCKS;
+    s.blocks.push_back(a->take());
   } else {
     int32_t blk = s.blocks[logical];
     if (a->ref_count[blk] > 1) {
       // shared block: copy on write
-      if (a->free_stack.empty()) return PA_ERR_OUT_OF_BLOCKS;
-      int32_t fresh = a->pop();
+      if (a->num_free() == 0) return PA_ERR_OUT_OF_BLOCKS;
+      int32_t fresh = a->take();
       a->ref_count[blk] -= 1;
       s.blocks[logical] = fresh;
       src = blk;
@@ -149,12 +368,16 @@ pa_status pa_alloc_free_seq(pa_alloc *a, int64_t seq_id) {
   auto it = a->seqs.find(seq_id);
   if (it == a->seqs.end()) return PA_ERR_STATE;
   const std::vector<int32_t> &blocks = it->second.blocks;
-  std::vector<int32_t> &ref = it->second.swapped ? a->host_ref : a->ref_count;
-  std::vector<int32_t> &free_list = it->second.swapped ? a->host_free : a->free_stack;
+  const bool host = it->second.swapped;
+  std::vector<int32_t> &ref = host ? a->host_ref : a->ref_count;
   for (int32_t b : blocks)
     if (b != kReleased && ref[b] <= 0) return PA_ERR_STATE;  // would underflow: refuse, change nothing
   for (auto r = blocks.rbegin(); r != blocks.rend(); ++r) {
-    if (*r != kReleased && --ref[*r] == 0) free_list.push_back(*r);
+    if (*r == kReleased || --ref[*r] != 0) continue;
+    if (host)
+      a->host_free.push_back(*r);
+    else
+      a->release(*r);
   }
   a->seqs.erase(it);
   return PA_OK;
@@ -175,7 +398,7 @@ pa_status pa_alloc_slide_window(pa_alloc *a, int64_t seq_id, int window, int *fr
     if (a->ref_count[b] <= 0) return PA_ERR_STATE;
     s.blocks[i] = kReleased;
     if (--a->ref_count[b] == 0) {
-      a->free_stack.push_back(b);
+      a->release(b);
       ++n;
     }
   }
@@ -239,8 +462,8 @@ pa_status pa_alloc_stats(const pa_alloc *a, int *free_blocks, int64_t *used_toke
   }
   int64_t used = 0;
   for (const auto &kv : fill) used += kv.second;
-  const int64_t used_blocks = a->num_blocks - (int64_t)a->free_stack.size();
-  if (free_blocks) *free_blocks = (int)a->free_stack.size();
+  const int64_t used_blocks = a->num_blocks - a->num_free();
+  if (free_blocks) *free_blocks = (int)a->num_free();
   if (used_tokens) *used_tokens = used;
   if (wasted_tokens) *wasted_tokens = used_blocks * a->block_size - used;
   return PA_OK;
@@ -280,20 +503,29 @@ static pa_status swap_group(pa_alloc *a, const int64_t *seq_ids, int n, int64_t 
       if (refs[b]++ == 0) order.push_back(b);
     }
   std::vector<int32_t> &src_ref = out ? a->ref_count : a->host_ref;
-  std::vector<int32_t> &src_free = out ? a->free_stack : a->host_free;
   std::vector<int32_t> &dst_ref = out ? a->host_ref : a->ref_count;
-  std::vector<int32_t> &dst_free = out ? a->host_free : a->free_stack;
   for (int32_t b : order)
     if (src_ref[b] < refs[b]) return PA_ERR_STATE;
-  if (order.size() > dst_free.size()) return PA_ERR_OUT_OF_BLOCKS;
+  const int64_t dst_free = out ? (int64_t)a->host_free.size() : a->num_free();
+  if ((int64_t)order.size() > dst_free) return PA_ERR_OUT_OF_BLOCKS;
   if ((int)order.size() > cap) return PA_ERR_INVALID;
   std::unordered_map<int32_t, int32_t> moved;
   for (size_t i = 0; i < order.size(); ++i) {
     const int32_t b = order[i];
-    const int32_t d = dst_free.back();
-    dst_free.pop_back();
+    int32_t d;
+    if (out) {
+      d = a->host_free.back();
+      a->host_free.pop_back();
+    } else {
+      d = a->take();
+    }
     dst_ref[d] = refs[b];
-    if ((src_ref[b] -= refs[b]) == 0) src_free.push_back(b);
+    if ((src_ref[b] -= refs[b]) == 0) {
+      if (out)
+        a->release(b);
+      else
+        a->host_free.push_back(b);
+    }
     moved[b] = d;
     pairs[2 * i] = b;
     pairs[2 * i + 1] = d;

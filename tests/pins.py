@@ -28,7 +28,7 @@ import torch
 import oracle
 import synth
 from conftest import read_golden
-from oracle.allocator_model import BlockManagerModel
+from oracle.allocator_model import BlockManagerModel, OutOfBlocks
 
 NAN_BITS = {"f16": 0x7E00, "bf16": 0x7FC0}
 
@@ -655,6 +655,123 @@ def pin_allocator_swap():
     assert m.num_free() == 8
 
 
+def pin_allocator_prefix_cache():
+    """Prefix caching worked by hand (third page, section "分页还顺带解决了什么":
+    requests that begin alike point their first blocks at the same physical
+    blocks, and only completely filled blocks are shared; first page, section
+    9: the common prefix's KV is cached). Block size 4, 8 blocks; S is a
+    10-token system prompt 1..10."""
+    m = BlockManagerModel(8, 4)
+    S = list(range(1, 11))
+    # A = S + [11, 12]: nothing cached yet; its 3 full blocks get cached
+    assert m.add_seq_cached(0, S + [11, 12]) == 0
+    assert m.cached_blocks() == (3, 0) and m.num_free() == 5
+    a = m.block_table(0)
+    # B = S + [21] (11 tokens): blocks [1..4] and [1..8] are A's
+    assert m.add_seq_cached(1, S + [21]) == 8
+    assert m.block_table(1)[:2] == a[:2] and m.block_table(1)[2] not in a
+    assert [m.ref[b] for b in a] == [2, 2, 1] and m.num_free() == 4
+    # C = S + [11, 12, 13]: all three of A's blocks precede its last token
+    assert m.add_seq_cached(2, S + [11, 12, 13]) == 12
+    assert m.block_table(2)[:3] == a and m.num_free() == 3
+    # D = A's own prompt: its last token sits in block 3, which is computed again
+    assert m.add_seq_cached(3, S + [11, 12]) == 8
+    assert m.block_table(3)[2] not in a
+    assert m.cached_blocks() == (3, 0)          # block 3's prefix stays on A's block
+    assert [m.ref[b] for b in a] == [4, 4, 2] and m.num_free() == 2
+    for seq in (0, 1, 2, 3):
+        m.free_seq(seq)
+    # everything is free; A's blocks keep their prefixes, freed in the order
+    # a[2] (when C went), a[1] and a[0] (when D went)
+    assert m.num_free() == 8 and m.cached_blocks() == (3, 3)
+    assert m.add_seq_cached(4, S + [11, 12]) == 8          # served from the cache
+    assert m.block_table(4)[:2] == a[:2] and m.cached_blocks() == (3, 1)
+    m.free_seq(4)                                          # a[1], a[0] released again, after a[2]
+    # a 24-token request without caching needs 6 blocks: the 5 plain free ones,
+    # then the cached block released longest ago, a[2]
+    m.add_seq(5, 24)
+    assert a[2] in m.block_table(5) and m.cached_blocks() == (2, 2) and m.num_free() == 2
+    m.add_seq(6, 4)                                        # then a[1]
+    assert m.block_table(6) == [a[1]] and m.cached_blocks() == (1, 1)
+    # S + [31] would share a[0] and need 2 more blocks; only a[0] is free
+    try:
+        m.add_seq_cached(7, S + [31])
+        raise AssertionError("expected OutOfBlocks")
+    except OutOfBlocks:
+        pass
+    assert m.cached_blocks() == (1, 1) and m.num_free() == 1 and 7 not in m.tables
+    m.free_seq(5)
+    assert m.add_seq_cached(7, S + [31]) == 4              # [1..8] left with a[1]
+    h = m.block_table(7)
+    assert h[0] == a[0] and m.cached_blocks() == (2, 0)    # ... and is cached again on h[1]
+    assert m.add_seq_cached(8, S + [11, 12, 13]) == 8      # [1..12] left with a[2]
+    assert m.block_table(8)[:2] == h[:2] and m.cached_blocks() == (3, 0)
+    assert m.num_free() == 2
+    # a shared block that is free stops being free when shared: 3 blocks, one
+    # plain free and one cached [1..4] free; 1..4, 6..9, 10 shares that block and
+    # needs 2 more, but only 1 is left
+    m = BlockManagerModel(3, 4)
+    assert m.add_seq_cached(0, [1, 2, 3, 4, 5]) == 0
+    m.free_seq(0)
+    m.add_seq(1, 4)
+    assert m.num_free() == 2 and m.cached_blocks() == (1, 1)
+    try:
+        m.add_seq_cached(2, [1, 2, 3, 4, 6, 7, 8, 9, 10])
+        raise AssertionError("expected OutOfBlocks")
+    except OutOfBlocks:
+        pass
+    assert m.num_free() == 2 and m.cached_blocks() == (1, 1) and 2 not in m.tables
+
+
+def pin_allocator_prefix_cache_reconnect():
+    """A cached prefix whose shorter prefix lost its block is found again once a
+    request caches the shorter one anew: the KV of a full block depends only on
+    the tokens from position 0 to its end. Block size 4, 6 blocks."""
+    m = BlockManagerModel(6, 4)
+    assert m.add_seq_cached(0, list(range(1, 13))) == 0    # 3 blocks, 3 prefixes cached
+    q = m.block_table(0)
+    assert m.slide_window(0, 4) == 2                       # blocks [1..4], [1..8] released
+    assert m.cached_blocks() == (3, 2) and m.num_free() == 5
+    m.add_seq(1, 12)                                       # the 3 plain free blocks
+    m.add_seq(2, 4)                                        # reuses q[0]: [1..4] forgotten
+    assert m.block_table(2) == [q[0]] and m.cached_blocks() == (2, 1)
+    m.free_seq(1)
+    assert m.add_seq_cached(3, [1, 2, 3, 4, 99]) == 0      # [1..4] not cached: computed
+    r = m.block_table(3)
+    assert m.cached_blocks() == (3, 1)                     # and cached again on r[0]
+    assert m.add_seq_cached(4, list(range(1, 9)) + [100]) == 8
+    assert m.block_table(4)[:2] == [r[0], q[1]]            # [1..8] still on q[1]
+    assert m.cached_blocks() == (3, 0) and m.num_free() == 0
+
+
+def pin_allocator_prefix_cache_bruteforce():
+    """With a pool that never runs short and nothing freed, every full block a
+    prompt fills stays cached, so a new prompt of n tokens reuses exactly the
+    longest whole-block common prefix it has with any earlier prompt, capped at
+    the full blocks before its last token -- counted here by comparing the
+    token lists directly -- and takes its other blocks fresh."""
+    rng = np.random.default_rng(12)
+    bs = 4
+    m = BlockManagerModel(4096, bs)
+    stems = [list(rng.integers(0, 5, size=24)) for _ in range(3)]
+    prompts, fresh = [], 0
+    for k in range(120):
+        stem = stems[int(rng.integers(0, 3))]
+        cut = int(rng.integers(0, 25))
+        p = [int(t) for t in stem[:cut]] + [int(t) for t in rng.integers(0, 5, size=int(rng.integers(0, 9)))]
+        best = 0
+        for r in prompts:
+            lcp = 0
+            while lcp < min(len(r), len(p)) and r[lcp] == p[lcp]:
+                lcp += 1
+            best = max(best, lcp // bs)
+        want = min(best, max(len(p) - 1, 0) // bs) * bs
+        assert m.add_seq_cached(k, p) == want, (k, p)
+        fresh += -(-len(p) // bs) - want // bs
+        prompts.append(p)
+    assert m.num_free() == 4096 - fresh
+
+
 ALL_ORACLE_PINS = [
     pin_f16_decoder, pin_bf16_decoder, pin_worked_example_slots, pin_bs16_tables, pin_dense,
     pin_len1_returns_v, pin_identical_keys_mean_v, pin_bruteforce_fsum, pin_relabel, pin_poison,
@@ -664,4 +781,5 @@ ALL_ORACLE_PINS = [
     pin_prefill_bruteforce_fsum, pin_prefill_relabel,
 ]
 ALL_MODEL_PINS = [pin_allocator_worked_example, pin_allocator_capacity, pin_allocator_cow,
-                  pin_allocator_sliding_window, pin_allocator_swap]
+                  pin_allocator_sliding_window, pin_allocator_swap, pin_allocator_prefix_cache,
+                  pin_allocator_prefix_cache_reconnect, pin_allocator_prefix_cache_bruteforce]

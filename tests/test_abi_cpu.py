@@ -180,12 +180,34 @@ def test_random_trace_matches_model_up_to_relabelling(seed):
     model.set_host_blocks(nh)
     prod.set_host_blocks(nh)
     live, next_id = [], 0
-    ops = ["add", "fork", "append", "append", "append", "free", "window", "swap_out", "swap_in"]
-    for _ in range(2000):
+    ops = ["add", "fork", "append", "append", "append", "free", "window", "swap_out", "swap_in",
+           "cached", "cached"]
+    # prompts for prefix caching: a few shared stems over a small vocabulary
+    stems = [[int(t) for t in rng.integers(0, 3, size=48)] for _ in range(3)]
+    for step in range(2000):
         op = rng.choice(ops)
         resident = [s for s in live if s not in model.swapped]
         swapped = [s for s in live if s in model.swapped]
-        if op == "add" or not resident:
+        if step % 500 == 499:
+            model.reset_prefix_cache()
+            prod.reset_prefix_cache()
+        if op == "cached":
+            stem = stems[int(rng.integers(0, len(stems)))]
+            toks = stem[:int(rng.integers(0, 49))] + \
+                [int(t) for t in rng.integers(0, 3, size=int(rng.integers(0, 12)))]
+            try:
+                got = model.add_seq_cached(next_id, toks)
+                ok = True
+            except ModelOOM:
+                ok = False
+            if ok:
+                assert prod.add_seq_cached(next_id, toks) == got
+                live.append(next_id)
+            else:
+                with pytest.raises(OutOfBlocks):
+                    prod.add_seq_cached(next_id, toks)
+            next_id += 1
+        elif op == "add" or not resident:
             n = int(rng.integers(0, 40))
             try:
                 model.add_seq(next_id, n)
@@ -252,6 +274,51 @@ def test_random_trace_matches_model_up_to_relabelling(seed):
         assert _relabel_consistent(model, prod, [s for s in live if s not in model.swapped])
         assert _relabel_consistent(model, prod, [s for s in live if s in model.swapped], host=True)
         assert model.stats() == prod.stats()
+        assert model.cached_blocks() == prod.cached_blocks()
+
+
+def test_prefix_cache_worked_example():
+    """The hand-worked prefix-caching example on the product (block size 4, 8
+    blocks, system prompt 1..10): shared blocks, the recomputed last block,
+    release order and reuse of cached blocks, all-or-nothing."""
+    m = BlockManager(8, 4)
+    S = list(range(1, 11))
+    assert m.add_seq_cached(0, S + [11, 12]) == 0
+    a = m.block_table(0)
+    assert m.add_seq_cached(1, S + [21]) == 8 and m.block_table(1)[:2] == a[:2]
+    assert m.add_seq_cached(2, S + [11, 12, 13]) == 12 and m.block_table(2)[:3] == a
+    assert m.add_seq_cached(3, S + [11, 12]) == 8 and m.block_table(3)[2] not in a
+    assert [m.ref_count(b) for b in a] == [4, 4, 2] and m.cached_blocks() == (3, 0)
+    for seq in range(4):
+        m.free_seq(seq)
+    assert m.num_free() == 8 and m.cached_blocks() == (3, 3)
+    assert m.add_seq_cached(4, S + [11, 12]) == 8
+    m.free_seq(4)
+    m.add_seq(5, 24)
+    assert a[2] in m.block_table(5) and m.cached_blocks() == (2, 2)
+    m.add_seq(6, 4)
+    assert m.block_table(6) == [a[1]]
+    with pytest.raises(OutOfBlocks):
+        m.add_seq_cached(7, S + [31])
+    assert m.cached_blocks() == (1, 1) and m.num_free() == 1
+    m.free_seq(5)
+    assert m.add_seq_cached(7, S + [31]) == 4
+    assert m.add_seq_cached(8, S + [11, 12, 13]) == 8
+    assert m.cached_blocks() == (3, 0) and m.num_free() == 2
+    for seq in (6, 7, 8):
+        m.free_seq(seq)
+    assert m.cached_blocks() == (3, 3)
+    m.reset_prefix_cache()
+    assert m.cached_blocks() == (0, 0) and m.num_free() == 8
+    assert m.add_seq_cached(9, S + [11]) == 0
+
+
+def test_prefix_cache_arguments():
+    m = BlockManager(8, 4)
+    assert m.add_seq_cached(0, []) == 0 and m.block_table(0) == []
+    with pytest.raises(PAError):
+        m.add_seq_cached(0, [1, 2, 3])           # the sequence exists
+    assert m.add_seq_cached(1, [5]) == 0 and m.add_seq_cached(2, [5]) == 0
 
 
 def test_swap_group_shares_blocks_once():

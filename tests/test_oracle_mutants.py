@@ -68,3 +68,49 @@ def test_pins_catch_mutant(name, tmp_path):
                 caught.append((pin.__name__, type(e).__name__))
                 break
     assert caught, f"no pin caught the planted mistake {name}"
+
+
+# Plausible mistakes in the block-manager model (oracle/allocator_model.py);
+# the model pins must catch each.
+MODEL_MUTANTS = {
+    "cow_at_three_users": ("if self.ref[blk] > 1:", "if self.ref[blk] > 2:"),
+    "window_releases_partial_block": ("for i in range(start // self.block_size):",
+                                      "for i in range(-(-start // self.block_size)):"),
+    "prefix_lookup_reaches_last_token": ("for i in range(max(n - 1, 0) // bs):",
+                                         "for i in range(n // bs):"),
+    "prefix_partial_block_cached": ("for i in range(len(shared), n // bs):",
+                                    "for i in range(len(shared), -(-n // bs)):"),
+    "prefix_evicts_newest": ("blk = next(iter(self.idle))", "blk = next(reversed(self.idle))"),
+    "prefix_idle_not_free": ("return len(self.free) + len(self.idle)", "return len(self.free)"),
+    "prefix_hit_left_idle": ("self.idle.pop(b, None)", "pass"),
+    "prefix_hits_not_counted": ("unused = sum(1 for b in shared if self.ref[b] == 0)",
+                                "unused = 0"),
+    "prefix_not_kept_after_free": ("if blk in self.prefix_of:\n            self.idle[blk] = None",
+                                   "if False:\n            self.idle[blk] = None"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MODEL_MUTANTS))
+def test_model_pins_catch_mutant(name, tmp_path, monkeypatch):
+    import importlib.util
+
+    import oracle.allocator_model as am
+    old, new = MODEL_MUTANTS[name]
+    src = open(am.__file__).read()
+    assert src.count(old) == 1, f"anchor of mutant {name} not found once in allocator_model.py"
+    path = os.path.join(tmp_path, "allocator_model_mutant.py")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    spec = importlib.util.spec_from_file_location("allocator_model_mutant", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    monkeypatch.setattr(pins, "BlockManagerModel", mod.BlockManagerModel)
+    monkeypatch.setattr(pins, "OutOfBlocks", mod.OutOfBlocks)
+    caught = []
+    for pin in pins.ALL_MODEL_PINS:
+        try:
+            pin()
+        except Exception as e:  # noqa: BLE001 -- any failure of a pin counts
+            caught.append((pin.__name__, type(e).__name__))
+            break
+    assert caught, f"no model pin caught the planted mistake {name}"
