@@ -430,18 +430,23 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
 
 // ============================================================ tcgen05 kernel (5th-gen tensor cores)
 // Same computation, one CTA per (q head, 256 query tokens, sequence), with the
-// two products on tcgen05.mma and every accumulator in tensor memory. The 256
-// rows form two groups of 128 (one tcgen05 M each); the groups share every K/V
-// tile and take turns on the tensor core, so one group's softmax overlaps the
-// other group's products.
-//   warp 0      stages 64-key K/V tiles with TMA into a 2-stage ring;
+// two products on tcgen05.mma and every operand of P V but V in tensor memory.
+// The 256 rows form two groups of 128 (one tcgen05 M each); the groups share
+// every K/V tile and take turns on the tensor core, so one group's softmax
+// overlaps the other group's products.
+//   warp 0      stages 64-key K/V tiles with TMA into a 4-stage ring;
 //   warp 1      allocates TMEM (512 columns: per group two S buffers and O); its
 //               lane 0 issues, per tile, S = Q K^T for each group and, one tile
-//               behind, O += P V for each group, committing each to an mbarrier;
+//               behind, O += P V for each group with P read from TMEM,
+//               committing each to an mbarrier;
 //   warps 2-9   one thread per query row (group = (warp - 2) / 4, TMEM lane =
 //               32 * (warp % 4) + lane): copy its Q row into shared memory, then
 //               per tile read its S row from TMEM, mask, online softmax in the
-//               log2 domain, write its P row (swizzled) for the next product.
+//               log2 domain, and write its P row (16-bit, two per column) over
+//               the S row it came from. S being double-buffered, so is P: the
+//               softmax never waits for a P V to finish; the next S into a
+//               buffer is issued after the P V that reads it (the tensor core
+//               runs its operations in issue order).
 //               O is rescaled in TMEM only when the row max grows by more than
 //               2^8 (the weights against the stale max stay <= 2^8 and the final
 //               division by the matching sum keeps the result exact); l sums the
@@ -452,14 +457,14 @@ namespace t5 {
 constexpr int kM = 128;        // query rows per group (tcgen05 M)
 constexpr int kGroups = 2;
 constexpr int kN = 64;         // keys per tile
-// K/V ring depth and P buffers per group (3 x 1 or 2 x 2 fit the 227 KB limit)
+// K/V ring depth (4 x 32 KB + 64 KB of Q at D = 128 fit the 227 KB limit)
 #ifndef PA_PREFILL_TC_STAGES
-#define PA_PREFILL_TC_STAGES 3
+#define PA_PREFILL_TC_STAGES 4
 #endif
 constexpr int kStages = PA_PREFILL_TC_STAGES;
-constexpr int kPBufs = kStages >= 3 ? 1 : 2;
 constexpr int kThreads = (2 + 4 * kGroups) * 32;
-constexpr uint32_t kTmemCols = 512;  // group g: S buffers at 256g + {0, 64}, O at 256g + 128
+// group g: S/P buffers at 256g + {0, 64} (P in the first 32 columns), O at 256g + 128
+constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
 
 template <int D>
@@ -469,12 +474,10 @@ struct Lay {
   static constexpr int kQBytes = kPanels * kQPanel;
   static constexpr int kKVPanel = kN * 128;                   // 64 rows x 128 bytes
   static constexpr int kStageBytes = 2 * kPanels * kKVPanel;  // K panels, then V panels
-  static constexpr int kPBytes = kM * 128;                    // 128 rows x 64 keys
   static constexpr int kRingOff = kQBytes;
-  static constexpr int kPOff = kRingOff + kStages * kStageBytes;  // [group][buffer]
-  static constexpr int kBarOff = kPOff + kGroups * kPBufs * kPBytes;
-  // full[S] empty[S] q_ready mma_done, then per group s_full[2] s_free[2] p_full[2] pv_done[2]
-  static constexpr int kNumBars = 2 * kStages + 2 + 8 * kGroups;
+  static constexpr int kBarOff = kRingOff + kStages * kStageBytes;
+  // full[S] empty[S] q_ready mma_done, then per group s_full[2] p_full[2] pv_done[2]
+  static constexpr int kNumBars = 2 * kStages + 2 + 6 * kGroups;
   static constexpr int kTmemOff = kBarOff + kNumBars * 8;
   static constexpr int kFlagOff = kTmemOff + 8;
   static constexpr int kBytes = 1024 + kFlagOff + 16;
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   constexpr int kM = t5::kM, kN = t5::kN, NS = t5::kStages, NG = t5::kGroups;
   constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t kIdescS = umma_idesc_f16(kFmt, 0, 0, kN, kM);  // Q (K-major) . K (K-major)
-  constexpr uint32_t kIdescO = umma_idesc_f16(kFmt, 0, 1, D, kM);   // P (K-major) . V (MN-major)
+  constexpr uint32_t kIdescO = umma_idesc_f16(kFmt, 0, 1, D, kM);   // P (TMEM) . V (MN-major)
 
   extern __shared__ __align__(128) unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -498,16 +501,14 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
   uint64_t *full_bar = bars, *empty_bar = bars + NS, *q_ready = bars + 2 * NS;
   uint64_t *mma_done = q_ready + 1;
-  // per group g: s_full[g][2], s_free[g][2], p_full[g][2], pv_done[g][2]
-  auto s_full = [&](int g, int i) { return mma_done + 1 + g * 8 + i; };
-  auto s_free = [&](int g, int i) { return mma_done + 1 + g * 8 + 2 + i; };
-  auto p_full = [&](int g, int i) { return mma_done + 1 + g * 8 + 4 + i; };
-  auto pv_done = [&](int g, int i) { return mma_done + 1 + g * 8 + 6 + i; };
+  // per group g: s_full[g][2], p_full[g][2], pv_done[g][2]
+  auto s_full = [&](int g, int i) { return mma_done + 1 + g * 6 + i; };
+  auto p_full = [&](int g, int i) { return mma_done + 1 + g * 6 + 2 + i; };
+  auto pv_done = [&](int g, int i) { return mma_done + 1 + g * 6 + 4 + i; };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
   const uint32_t q_sm = smem_u32(smem);
   const uint32_t ring = smem_u32(smem + L::kRingOff);
-  const uint32_t p_sm = smem_u32(smem + L::kPOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.x;
@@ -558,7 +559,6 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     for (int g = 0; g < NG; ++g)
       for (int i = 0; i < 2; ++i) {
         mbar_init(s_full(g, i), 1);
-        mbar_init(s_free(g, i), 128);
         mbar_init(p_full(g, i), 128);
         mbar_init(pv_done(g, i), 1);
       }
@@ -612,9 +612,10 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   } else if (warp == 1) {
     // ====================================================================== MMA issuer
     // Issues whatever is ready, in any order: S_j of a group as soon as K_j has
-    // landed and the group has read S_{j-2} (double-buffered S), P_j V_j of a
-    // group as soon as its softmax wrote P_j; a tile's stage goes back to the
-    // producer once every group that reads it has issued its P V.
+    // landed and P_{j-2} V_{j-2}, which reads the same TMEM buffer, has been
+    // issued; P_j V_j of a group as soon as its softmax wrote P_j; a tile's
+    // stage goes back to the producer once every group that reads it has
+    // issued its P V.
     if (lane == 0) {
       bool go = wait_bounded(q_ready, 0, abort_flag);
       tc_fence_after();
@@ -629,8 +630,8 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         for (int g = 0; g < NG; ++g) {
           if (npv[g] < gtiles[g]) done = false;
           const int js = ns[g];
-          if (js < gtiles[g] && mbar_try_wait(&full_bar[js % NS], (js / NS) & 1) &&
-              (js < 2 || mbar_try_wait(s_free(g, js & 1), ((js - 2) / 2) & 1))) {
+          if (js < gtiles[g] && (js < 2 || npv[g] >= js - 1) &&
+              mbar_try_wait(&full_bar[js % NS], (js / NS) & 1)) {
             tc_fence_after();
             const uint32_t kaddr = ring + (js % NS) * L::kStageBytes;
 #pragma unroll
@@ -650,11 +651,9 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
             const uint32_t vaddr = ring + (jp % NS) * L::kStageBytes + L::kPanels * L::kKVPanel;
 #pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk)
-              umma_f16(tmem + g * 256 + 128,
-                       umma_desc_sw128(p_sm + (g * t5::kPBufs + jp % t5::kPBufs) * L::kPBytes + kk * 32,
-                                       16, 1024),
-                       umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
-                       kIdescO, jp > 0 || kk > 0);
+              umma_f16_ts(tmem + g * 256 + 128, tmem + g * 256 + (jp & 1) * kN + kk * 8,
+                          umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
+                          kIdescO, jp > 0 || kk > 0);
             umma_commit(pv_done(g, jp & 1));
             ++npv[g];
             progress = true;
@@ -723,25 +722,27 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       tmem_ld32(trow + sb * kN, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld32(trow + sb * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_free(grp, sb));
-      // max of the raw scores (the scale is positive); masked keys become -inf
-      float mx = -INFINITY;
-      // the mask only matters on tiles that reach past a row of this warp or
-      // start before a row's window (warp-uniform)
+      // max of the raw scores (the scale is positive); masked keys become -inf.
+      // The mask only matters on tiles that reach past a row of this warp or
+      // start before a row's window (warp-uniform).
       if (t0 + kN - 1 > wr0 || (p.window > 0 && t0 < first_key(wr1, p.window))) {
 #pragma unroll
         for (int c = 0; c < kN; ++c) {
           const int kp = t0 + c;
-          const float x = (kp <= pr && kp >= lo) ? __uint_as_float(sv[c]) : -INFINITY;
-          sv[c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          if (kp > pr || kp < lo) sv[c] = __float_as_uint(-INFINITY);
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < kN; ++c) mx = fmaxf(mx, __uint_as_float(sv[c]));
       }
-      mx *= p.scale_log2;  // log2 domain
+      // eight independent running maxima, then a tree: a short dependency chain
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sv[e]);
+#pragma unroll
+      for (int c = 8; c < kN; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], __uint_as_float(sv[c]));
+#pragma unroll
+      for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+        for (int e = 0; e < w; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + w]);
+      float mx = mx8[0] * p.scale_log2;  // log2 domain
       // move the reference max when it grew past the lazy bound (warp-uniform
       // TMEM traffic: lanes that keep theirs scale by 1)
       const bool grow = mx > m_ref + t5::kLazyRescale || (m_ref == -INFINITY && mx > -INFINITY);
@@ -763,28 +764,22 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       }
       if (grow) m_ref = mx;
       const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
-      // this tile's P row -> the group's P buffer; weight = 2^(s * scale_log2 - m_ref),
-      // one FMA and one exp2 per key
-      // (one buffer: free once P_{j-1} V_{j-1} is done; two: once P_{j-2} V_{j-2} is)
-      if (j >= t5::kPBufs) {
-        const int jr = j - t5::kPBufs;
-        wait_bounded(pv_done(grp, jr & 1), (jr / 2) & 1, abort_flag);
-      }
-      unsigned char *prow =
-          smem + L::kPOff + (grp * t5::kPBufs + j % t5::kPBufs) * L::kPBytes + r * 128;
+      // this tile's P row, weight = 2^(s * scale_log2 - m_ref) (one FMA and one
+      // exp2 per key), packed two per column over the first half of its S row;
+      // l sums the unrounded weights (|rounding| <= 2^-9 relative each), in four
+      // partial sums for a short dependency chain
+      uint32_t pw[32];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = ex2_approx(fmaf(__uint_as_float(sv[ch * 8 + 2 * e]), p.scale_log2, nbase));
-          const float c = ex2_approx(fmaf(__uint_as_float(sv[ch * 8 + 2 * e + 1]), p.scale_log2, nbase));
-          float ra, rc;
-          w[e] = Mma<T>::pack(a, c, ra, rc);
-          l += a + c;  // the sum of the unrounded weights (|rounding| <= 2^-9 relative each)
-        }
-        *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int c = 0; c < 32; ++c) {
+        const float a = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), p.scale_log2, nbase));
+        const float b2 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), p.scale_log2, nbase));
+        float ra, rb;
+        pw[c] = Mma<T>::pack(a, b2, ra, rb);
+        ls[c % 4] += a + b2;
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      tmem_st32(trow + sb * kN, pw);
       // rows of V outside every row's keys may hold anything: zero them (both
       // groups zero the same rows of a shared stage; the writes are identical)
       const int nvalid = min(kN, n - t0);
@@ -797,8 +792,10 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
           *reinterpret_cast<uint4 *>(vz + pn * L::kKVPanel + vr * 128 + (ch << 4)) =
               make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
       mbar_arrive(p_full(grp, sb));
     }
     // ---- O / l -> global memory
