@@ -53,6 +53,8 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_370_b200", "csrc", "pa_decode.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pa_decode_llama8b_traffic.md")
+PREFILL_SRC = os.path.join(ROOT, "paged_kv_cache_370_b200", "csrc", "pa_prefill.cu")
+PREFILL_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pa_prefill_llama8b_traffic.md")
 
 
 # ------------------------------------------------------------------------------------- setup
@@ -102,14 +104,14 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def recorded_traffic():
-    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
-    the current decode source; else None."""
+def recorded_traffic(summary=TRAFFIC_FILE, source=DECODE_SRC):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
     try:
-        text = open(TRAFFIC_FILE).read()
+        text = open(summary).read()
     except OSError:
         return None
-    src = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()
+    src = hashlib.sha256(open(source, "rb").read()).hexdigest()
     m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
     m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
     if not m_sha or not m_bytes or m_sha.group(1) != src:
@@ -799,7 +801,9 @@ def run_prefill(args):
             "roofline": {"bound": "tensor", "kernel": "pa_prefill", "achieved": round(tflops, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
                          "peak_kind": kind, "flops_per_launch": flops,
-                         "avg_launch_ms": round(att_ms, 5), "traffic": None},
+                         "avg_launch_ms": round(att_ms, 5),
+                         "traffic": (recorded_traffic(PREFILL_TRAFFIC_FILE, PREFILL_SRC)
+                                     if args.window == 0 else None)},
             "gpu_launches": 2 * rounds * len(steps), "clocks": clocks.summary(t0, t1),
             "device_error_word": code}
 
