@@ -14,7 +14,7 @@ _EXPORTS = (
     "pa_decode_default_partition", "pa_decode_launches", "pa_decode_static_workspace",
     "pa_decode_workspace_size", "pa_device_status", "pa_reshape_and_cache", "pa_slot_mapping",
     "SwapSpace", "pa_swap_out", "pa_swap_in", "pa_decode_window", "pa_decode_append_window",
-    "pa_decode_window_launches", "pa_prefill", "pa_decode_append_overlapped",
+    "pa_decode_window_launches", "pa_decode_append_window_launches", "pa_prefill", "pa_decode_append_overlapped",
 )
 
 __all__ = list(_EXPORTS)

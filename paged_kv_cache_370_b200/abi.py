@@ -64,7 +64,8 @@ def _load() -> ctypes.CDLL:
         "pa_decode_append_overlapped": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f,
                                             i, P, sz, i, P]),
         "pa_decode_window": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P, sz, i, P]),
-        "pa_decode_window_launches": (i, [i, i, i, i, i, i, i]),
+        "pa_decode_window_launches": (i, [i, i, i, i, i, i, i, i, i]),
+        "pa_decode_append_window_launches": (i, [i, i, i, i, i, i, i, i, i]),
         "pa_prefill": (i, [P, P, P, P, P, i, P, P, i, i, i, i, i, i, i, i, i, f, i, i, P]),
         "pa_decode_append_window": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i,
                                         P, sz, i, P]),
@@ -290,11 +291,21 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, q_start, ma
     _check(st, "pa_prefill")
 
 
-def pa_decode_window_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
-                              window, partition_tokens=0) -> int:
+def pa_decode_window_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                              num_blocks, max_context_len, window, partition_tokens=0) -> int:
     """Kernels one pa_decode_window call with these arguments launches."""
     return int(_lib.pa_decode_window_launches(num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                              max_context_len, window, partition_tokens))
+                                              block_size, num_blocks, max_context_len, window,
+                                              partition_tokens))
+
+
+def pa_decode_append_window_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                     num_blocks, max_context_len, window,
+                                     partition_tokens=0) -> int:
+    """Kernels one pa_decode_append_window call with these arguments launches."""
+    return int(_lib.pa_decode_append_window_launches(num_seqs, num_q_heads, num_kv_heads,
+                                                     head_dim, block_size, num_blocks,
+                                                     max_context_len, window, partition_tokens))
 
 
 def pa_decode_append_window(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,

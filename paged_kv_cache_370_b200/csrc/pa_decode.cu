@@ -136,9 +136,13 @@ struct DecodeParams {
   const int64_t *new_slots;  // nullptr: no fused write
   void *k_cache_w;
   void *v_cache_w;
-  // sliding window (partition kernel only): a sequence of length len attends
-  // to positions [len - window, len) (0: every position)
+  // sliding window: a sequence of length len attends to positions
+  // [len - window, len) (0: every position). The partition kernel applies it
+  // directly; the even-split kernel sees each sequence from the block holding
+  // its first attended position on (window_remap_kernel) and masks the
+  // win_skip[b] positions of that block before the window (nullptr: none)
   int window;
+  const int32_t *win_skip;
   // even-split kernel launched as a programmatic dependent of the preceding kernel
   int early_start;
 };
@@ -559,7 +563,7 @@ struct TileMeta {
   int seg_first_x;    // global index of the segment's first tile
   int flags;          // 1: first tile of this CTA's piece, 2: last tile of it,
                       // 4: holds the sequence's new token (fused write)
-  int pad;
+  int nskip;          // leading rows before a sliding window (the segment's first tile)
   long long new_slot;  // slot of the new token (flags & 4)
 };
 
@@ -613,7 +617,10 @@ __host__ __device__ constexpr int piece_stride() { return D + 4; }
 
 __device__ __forceinline__ int seg_tiles(int len) { return len > 0 ? (len + kTile - 1) / kTile : 1; }
 
-template <typename T, int D, int G>
+// kWindow: the sequences come from window_remap_kernel and the first tile of
+// each may start with positions before the window (a separate instantiation,
+// so that plain decode carries none of the masking)
+template <typename T, int D, int G, bool kWindow>
 __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     pa_decode_stream_kernel(const __grid_constant__ CUtensorMap tmap_k,
                             const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
@@ -794,6 +801,7 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         m.nvalid = nvalid;
         m.seg_first_x = (int)(x0 + i - j);
         m.flags = (seg_begin ? 1 : 0) | (seg_end ? 2 : 0) | (new_tok ? 4 : 0);
+        m.nskip = (kWindow && j == 0) ? min(max(__ldg(p.win_skip + b), 0), kTile - 1) : 0;
         m.new_slot = slot_b;
         mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes +
                                                 (seg_begin ? (uint32_t)C::kQBytes : 0u) +
@@ -905,6 +913,7 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       l0 = l1 = 0.f;
     }
     const int nvalid = mt.nvalid;
+    const int nskip = kWindow ? mt.nskip : 0;
     if ((mt.flags & 4) && (nvalid - 1) / 16 == warp) {
       // fused write: the new token (last valid row) replaces what the cache held
       // in this tile, and is stored at its slot for later steps
@@ -928,15 +937,18 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       }
       __syncwarp();
     }
-    if (nvalid < wrow + 16) {
-      // rows past the valid tokens may hold anything (0 * NaN would poison the
-      // product): zero this warp's own V rows there before reading them
+    if (nvalid < wrow + 16 || nskip > wrow) {
+      // rows past the valid tokens, or before a sliding window, may hold anything
+      // (0 * NaN would poison the product): zero this warp's own V rows there
+      // before reading them
       unsigned char *vz = smem + s * C::kStageBytes + C::kPanels * kPanelBytes;
-      for (int r = max(nvalid, wrow) + (lane >> 3); r < wrow + 16; r += 4)
+      for (int r = (kWindow ? wrow : max(nvalid, wrow)) + (lane >> 3); r < wrow + 16; r += 4) {
+        if (kWindow && r < nvalid && r >= nskip) continue;
 #pragma unroll
         for (int pn = 0; pn < C::kPanels; ++pn)
           *reinterpret_cast<uint4 *>(vz + pn * kPanelBytes + r * 128 + (lane & 7) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
+      }
       __syncwarp();
     }
 
@@ -951,7 +963,8 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       Mma<T>::run(sa, a, qb[kk][0], qb[kk][1]);
       Mma<T>::run(sb, a2, qb[kk + 1][0], qb[kk + 1][1]);
     }
-    const bool va = wrow + g < nvalid, vb = wrow + g + 8 < nvalid;
+    const bool va = wrow + g < nvalid && wrow + g >= nskip;
+    const bool vb = wrow + g + 8 < nvalid && wrow + g + 8 >= nskip;
     const float s0 = va ? (sa[0] + sb[0]) * p.scale_log2 : -INFINITY;
     const float s1 = va ? (sa[1] + sb[1]) * p.scale_log2 : -INFINITY;
     const float s2 = vb ? (sa[2] + sb[2]) * p.scale_log2 : -INFINITY;
@@ -1153,6 +1166,33 @@ __global__ void __launch_bounds__(D) pa_decode_merge_kernel(
   out[hq * D + d] = Elem<T>::from_f32(acc / Ls);
 }
 
+// ------------------------------------------------------------------- sliding-window remap
+// A sliding window on the even-split kernel: sequence b is handed over from
+// the block holding its first attended position on -- its table shifted by
+// that many blocks (vtab, vwidth entries per row) and its length shorter by as
+// many positions (vlen) -- with vskip[b] = the positions at the start of that
+// block that precede the window, which the kernel masks. With block_size <= 64
+// they all lie in the sequence's first tile. A length outside [0, max_len] or
+// beyond its table becomes -1, which the kernel reports as a bad length.
+__global__ void __launch_bounds__(128) window_remap_kernel(
+    const int32_t *__restrict__ tables, int width, const int32_t *__restrict__ lens, int bs,
+    int window, int max_len, int vwidth, int32_t *__restrict__ vtab,
+    int32_t *__restrict__ vlen, int32_t *__restrict__ vskip) {
+  const int b = blockIdx.x;
+  const int len = __ldg(lens + b);
+  const bool ok = len >= 0 && len <= max_len && (long long)len <= (long long)width * bs;
+  const int lo = ok ? window_lo(len, window) : 0;
+  const int shift = lo / bs;
+  if (threadIdx.x == 0) {
+    vlen[b] = ok ? len - shift * bs : -1;
+    vskip[b] = lo - shift * bs;
+  }
+  for (int i = threadIdx.x; i < vwidth; i += blockDim.x) {
+    const int src = i + shift;
+    vtab[(size_t)b * vwidth + i] = src < width ? __ldg(tables + (size_t)b * width + src) : 0;
+  }
+}
+
 }  // namespace
 
 // ================================================================================ host side
@@ -1262,7 +1302,7 @@ int stream_ctas_per_sm() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 1;
   if (!per_sm[dev]) {
-    auto kernel = tc::pa_decode_stream_kernel<__nv_bfloat16, D, G>;
+    auto kernel = tc::pa_decode_stream_kernel<__nv_bfloat16, D, G, false>;
     const size_t smem = tc::Cfg<D, G>::kBytes;
     int n = 0;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -1308,6 +1348,22 @@ bool uses_stream_kernel(int group, int block_size, int num_blocks, int num_kv_he
   return group > 1 && tensor_core_block_size(block_size) && rows <= INT32_MAX;
 }
 
+// A sliding window runs on the even-split kernel when the positions of a
+// block before the window fit in one 64-token tile; otherwise (and where the
+// even-split kernel does not run at all) in the partition kernel.
+bool window_on_stream(int group, int block_size, int num_blocks, int num_kv_heads) {
+  return uses_stream_kernel(group, block_size, num_blocks, num_kv_heads) &&
+         block_size <= tc::kTile;
+}
+
+// Workspace after the even-split kernel's pieces for the window remap: the
+// shifted lengths and skips (padded to 16 bytes), then the shifted tables.
+size_t window_remap_bytes(int num_seqs, int max_context_len, int block_size) {
+  const long long vwidth = std::max(1, (max_context_len + block_size - 1) / block_size);
+  const size_t heads = ((size_t)2 * num_seqs * sizeof(int32_t) + 15) / 16 * 16;
+  return heads + (size_t)num_seqs * vwidth * sizeof(int32_t);
+}
+
 size_t stream_workspace(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                         int max_context_len, int partition_tokens) {
   const int group = num_q_heads / num_kv_heads;
@@ -1328,7 +1384,12 @@ pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dty
     if (!pool_tensor_map(&tk, prm.k_cache, rows, D, box_rows, dtype) ||
         !pool_tensor_map(&tv, prm.v_cache, rows, D, box_rows, dtype))
       return PA_ERR_CUDA;
-    if (!ensure_smem(tc::pa_decode_stream_kernel<T, D, G>, (size_t)C::kBytes, configured))
+    const bool win = prm.win_skip != nullptr;
+    static size_t configured_w[kMaxDevices] = {};
+    if (!(win ? ensure_smem(tc::pa_decode_stream_kernel<T, D, G, true>, (size_t)C::kBytes,
+                            configured_w)
+              : ensure_smem(tc::pa_decode_stream_kernel<T, D, G, false>, (size_t)C::kBytes,
+                            configured)))
       return PA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)prm.grid_ctas);
@@ -1340,8 +1401,10 @@ pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dty
     attr[0].val.programmaticStreamSerializationAllowed = prm.early_start ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, tc::pa_decode_stream_kernel<T, D, G>, tk, tv, prm) != cudaSuccess)
-      return PA_ERR_CUDA;
+    const cudaError_t e =
+        win ? cudaLaunchKernelEx(&cfg, tc::pa_decode_stream_kernel<T, D, G, true>, tk, tv, prm)
+            : cudaLaunchKernelEx(&cfg, tc::pa_decode_stream_kernel<T, D, G, false>, tk, tv, prm);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
   }
   using L = Smem<T, D, G>;
@@ -1424,10 +1487,13 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int nu
   const size_t simt = simt_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                      max_context_len, partition_tokens);
   const int group = num_q_heads / num_kv_heads;
+  // (the even-split kernel's pieces, and room for a sliding window's remap at
+  // the smallest block size that kernel takes)
   const size_t stream = (group == 2 || group == 4 || group == 8) &&
                                 (head_dim == 64 || head_dim == 128)
                             ? stream_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                               max_context_len, partition_tokens)
+                                               max_context_len, partition_tokens) +
+                                  window_remap_bytes(num_seqs, max_context_len, 8)
                             : 0;
   const size_t body = simt > stream ? simt : stream;
   return body ? kCounterRegion + body : 0;
@@ -1483,14 +1549,21 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_UNSUPPORTED;
   const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
   const int max_parts = max_context_len > 0 ? (max_context_len + pt - 1) / pt : 1;
-  // a sliding window runs in the partition kernel
-  const bool streamk = window == 0 && uses_stream_kernel(group, block_size, num_blocks, num_kv_heads);
+  // a sliding window runs on the even-split kernel after a remap where the
+  // block size allows (window_on_stream), else in the partition kernel
+  const bool wstream =
+      window > 0 && window_on_stream(group, block_size, num_blocks, num_kv_heads);
+  const bool streamk = (window == 0 && uses_stream_kernel(group, block_size, num_blocks,
+                                                          num_kv_heads)) ||
+                       wstream;
   const int nctas = streamk ? stream_grid(num_seqs, num_kv_heads, group, head_dim,
                                           max_context_len, partition_tokens)
                             : 0;
+  const size_t pieces_bytes = (size_t)2 * nctas * group * (head_dim + 4) * sizeof(float);
   size_t need;
   if (streamk)
-    need = kCounterRegion + (size_t)2 * nctas * group * (head_dim + 4) * sizeof(float);
+    need = kCounterRegion + pieces_bytes +
+           (wstream ? window_remap_bytes(num_seqs, max_context_len, block_size) : 0);
   else
     need = max_parts > 1 ? kCounterRegion + (size_t)num_seqs * num_q_heads * max_parts *
                                                 (head_dim + 2) * sizeof(float)
@@ -1520,6 +1593,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   prm.k_cache_w = fw ? fw->k_cache : nullptr;
   prm.v_cache_w = fw ? fw->v_cache : nullptr;
   prm.window = window;
+  prm.win_skip = nullptr;
   prm.early_start = early_start ? 1 : 0;
   if (fw && !streamk) return PA_ERR_INVALID;  // only the even-split kernel writes
   prm.max_blocks_per_seq = max_blocks_per_seq;
@@ -1535,6 +1609,26 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   if ((size_t)prm.table_slice * 4 > 16384) return PA_ERR_UNSUPPORTED;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (wstream) {
+    // each sequence from the block of its first attended position on; the
+    // even-split kernel then runs with no window of its own
+    const int vwidth = std::max(1, (max_context_len + block_size - 1) / block_size);
+    char *base = reinterpret_cast<char *>(ws_body) + pieces_bytes;
+    int32_t *vlen = reinterpret_cast<int32_t *>(base);
+    int32_t *vskip = vlen + num_seqs;
+    int32_t *vtab = reinterpret_cast<int32_t *>(
+        base + ((size_t)2 * num_seqs * sizeof(int32_t) + 15) / 16 * 16);
+    window_remap_kernel<<<num_seqs, 128, 0, st>>>(block_tables, max_blocks_per_seq, context_lens,
+                                                  block_size, window, max_context_len, vwidth,
+                                                  vtab, vlen, vskip);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    prm.block_tables = vtab;
+    prm.context_lens = vlen;
+    prm.max_blocks_per_seq = vwidth;
+    prm.win_skip = vskip;
+    prm.window = 0;
+    prm.early_start = 0;  // the remap kernel just wrote the lengths and tables it reads
+  }
   if (dtype == PA_BF16)
     return dispatch_dim<__nv_bfloat16>(head_dim, group, prm, num_seqs, out, dtype, st);
   return dispatch_dim<__half>(head_dim, group, prm, num_seqs, out, dtype, st);
@@ -1570,15 +1664,33 @@ extern "C" pa_status pa_decode_window(void *out, const void *q, const void *k_ca
 }
 
 extern "C" int pa_decode_window_launches(int num_seqs, int num_q_heads, int num_kv_heads,
-                                         int head_dim, int max_context_len, int window,
+                                         int head_dim, int block_size, int num_blocks,
+                                         int max_context_len, int window,
                                          int partition_tokens) {
   if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
-      head_dim <= 0 || window <= 0)
+      head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || window <= 0)
     return 0;
+  // the remap kernel and the even-split kernel
+  if (window_on_stream(num_q_heads / num_kv_heads, block_size, num_blocks, num_kv_heads))
+    return 2;
   // the partition kernel, and the merge kernel when the longest context has
   // more than one partition (partitions are sized from max_context_len)
   const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
   return max_context_len > pt ? 2 : 1;
+}
+
+extern "C" int pa_decode_append_window_launches(int num_seqs, int num_q_heads, int num_kv_heads,
+                                                int head_dim, int block_size, int num_blocks,
+                                                int max_context_len, int window,
+                                                int partition_tokens) {
+  const int decode = pa_decode_window_launches(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                               block_size, num_blocks, max_context_len, window,
+                                               partition_tokens);
+  if (decode == 0) return 0;
+  // on the even-split kernel the write is fused; otherwise the write kernel runs first
+  return window_on_stream(num_q_heads / num_kv_heads, block_size, num_blocks, num_kv_heads)
+             ? decode
+             : 1 + decode;
 }
 
 extern "C" int pa_decode_append_launches(int num_seqs, int num_q_heads, int num_kv_heads,
@@ -1610,14 +1722,15 @@ pa_status decode_append_impl(void *out, const void *q, const void *k_new, const 
       !aligned(slot_mapping, 8))
     return PA_ERR_INVALID;
   const int group = num_q_heads / num_kv_heads;
-  if (window == 0 && uses_stream_kernel(group, block_size, num_blocks, num_kv_heads)) {
+  if ((window == 0 && uses_stream_kernel(group, block_size, num_blocks, num_kv_heads)) ||
+      (window > 0 && window_on_stream(group, block_size, num_blocks, num_kv_heads))) {
     const FusedWrite fw{k_new, v_new, slot_mapping, k_cache, v_cache};
     return decode_impl(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                        max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim,
                        block_size, num_blocks, scale, dtype, workspace, workspace_bytes,
-                       partition_tokens, stream, &fw, 0, early_start);
+                       partition_tokens, stream, &fw, window, early_start);
   }
-  // other shapes, and sliding windows: the write kernel, then the decode
+  // other shapes (and windows the partition kernel runs): the write kernel, then the decode
   const pa_status st = pa_reshape_and_cache(k_new, v_new, slot_mapping, num_seqs, k_cache,
                                             v_cache, num_blocks, num_kv_heads, block_size,
                                             head_dim, dtype, stream);

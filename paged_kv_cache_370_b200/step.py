@@ -59,12 +59,11 @@ class DecodeStep:
         self.append_launches = abi.pa_decode_append_launches(B, hq, hkv, d, bs, nb,
                                                              self.max_context_len,
                                                              self.partition_tokens)
-        if self.window > 0:  # the partition kernel (and merge), after a separate write
-            self.decode_launches = abi.pa_decode_window_launches(B, hq, hkv, d,
-                                                                 self.max_context_len,
-                                                                 self.window,
-                                                                 self.partition_tokens)
-            self.append_launches = 1 + self.decode_launches
+        if self.window > 0:
+            self.decode_launches = abi.pa_decode_window_launches(
+                B, hq, hkv, d, bs, nb, self.max_context_len, self.window, self.partition_tokens)
+            self.append_launches = abi.pa_decode_append_window_launches(
+                B, hq, hkv, d, bs, nb, self.max_context_len, self.window, self.partition_tokens)
         self.partition = self.partition_tokens or abi.pa_decode_default_partition(
             B, hkv, self.max_context_len)
 

@@ -100,7 +100,7 @@ def test_window_covering_everything_is_plain_decode():
         g = GpuBatch(batch, window=w)
         outs.append(g.run().clone())
         assert g.step.launches() == 1 + abi.pa_decode_window_launches(
-            4, 32, 8, 128, batch.max_context_len, w)
+            4, 32, 8, 128, 16, 200, batch.max_context_len, w)
     assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
     kp, vp = oracle_pools(batch)
     ref = oracle.decode(batch.q, kp, vp, batch.block_tables, batch.context_lens, batch.scale,
