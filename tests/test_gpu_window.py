@@ -131,3 +131,30 @@ def test_window_long_skew_full():
     batch = synth.long_skew()
     s = _window_case(batch, 4096, sample=np.arange(batch.num_seqs))
     print(f"\nlong_skew window 4096: {s}")
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_window_bad_inputs_are_reported_not_accessed(fused):
+    """Bad block ids and lengths under a window (the remap route of the even-split
+    kernel and its fused write): reported in the device error word, never used to
+    address memory, and the context stays usable."""
+    batch = synth.small_random(49, 3, [40, 70, 9], 8, 2, 128, 16, 20, "bf16")
+    g = GpuBatch(batch, window=32, fused=fused)
+    g.run()
+    assert abi.pa_device_status() == 0
+    bad = batch.block_tables.copy()
+    bad[1, 3] = batch.num_blocks + 1000      # inside sequence 1's window (positions 38..69)
+    g.step.block_tables.copy_(torch.from_numpy(bad).cuda())
+    g.run()
+    assert abi.pa_device_status() & abi.PA_DEVERR_BLOCK_ID
+    g.step.block_tables.copy_(torch.from_numpy(batch.block_tables).cuda())
+    g.step.context_lens[2] = 10_000          # beyond the table and max_context_len
+    g.run()
+    assert abi.pa_device_status() & abi.PA_DEVERR_CONTEXT_LEN
+    g.step.context_lens.copy_(torch.from_numpy(batch.context_lens).cuda())
+    out = widen_out(g.run())
+    assert abi.pa_device_status() == 0
+    kp, vp = oracle_pools(batch)
+    ref = oracle.decode_window(batch.q, kp, vp, batch.block_tables, batch.context_lens,
+                               batch.scale, batch.dtype, 32)
+    assert_close(out, ref, batch.dtype, "window after bad inputs")
