@@ -104,6 +104,26 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def read_stream_gbs(torch, device):
+    """A read-only streaming rate on this GPU, for context beside the copy peak:
+    torch's sum over 4 GiB of bf16 (a library reduction, read-bound), best of 5."""
+    x = torch.ones(2 << 30, dtype=torch.bfloat16, device=device)
+    best = float("inf")
+    for i in range(7):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        torch.sum(x, dtype=torch.float32)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            best = min(best, a.elapsed_time(b))
+    nbytes = x.numel() * x.element_size()
+    del x
+    torch.cuda.empty_cache()
+    return {"value": round(nbytes / (best * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "how": "torch.sum over 4 GiB of bf16, best of 5 after 2 warm-up runs"}
+
+
 def recorded_traffic(summary=TRAFFIC_FILE, source=DECODE_SRC):
     """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
     the current kernel source; else None."""
@@ -436,6 +456,17 @@ def run_ours(args, rank, world, local, dist):
     time.sleep(0.2)
     sampler.stop()
     total_ms = start_ev.elapsed_time(end_ev)
+    # ---- the spread over rounds: the same rounds again, an event after each
+    round_ms = []
+    if rounds:
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(rounds + 1)]
+        evs[0].record(stream)
+        for r in range(rounds):
+            g_round.replay()
+            evs[r + 1].record(stream)
+        torch.cuda.synchronize()
+        round_ms = [evs[r].elapsed_time(evs[r + 1]) / R for r in range(rounds)]
+    read_stream = read_stream_gbs(torch, device)
     # ---- per-kernel durations (same launches, separately timed with events)
     reps = max(1, min(50, K // R))
     ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -468,7 +499,8 @@ def run_ours(args, rank, world, local, dist):
     dec_bytes = float(np.mean([infos[i % V]["decode"]["total"] +
                                (infos[i % V]["write"] if fused else 0) for i in range(K)]))
     achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
-    traffic = recorded_traffic() if args.workload == "llama8b" else None
+    # recorded for the plain (no window) kernel on this workload only
+    traffic = recorded_traffic() if args.workload == "llama8b" and args.window == 0 else None
     launches = sum(s.launches() for s in (steps[i % V] for i in range(K)))
 
     e2e = None
@@ -488,6 +520,13 @@ def run_ours(args, rank, world, local, dist):
         "query_tokens_per_s": round(q_tok, 1),
         "pct_of_hbm_measured": round(100 * gbs / world / peak, 2),
         "pct_of_hbm_nominal_8tbs": round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
+        "ms_per_step_over_rounds": ({"median": round(float(np.median(round_ms)), 5),
+                                     "min": round(float(np.min(round_ms)), 5),
+                                     "max": round(float(np.max(round_ms)), 5),
+                                     "rounds": len(round_ms), "steps_per_round": R,
+                                     "how": "the timed rounds replayed again with an event "
+                                            "after each"} if round_ms else None),
+        "hbm_read_stream": read_stream,
         "roofline": {"bound": "hbm",
                      "kernel": ("pa_decode_append (KV write + decode, one kernel)" if fused
                                 else "pa_decode"),
@@ -598,11 +637,23 @@ def cpu_baseline(batch, target_s):
                                     batch.block_size)["total"]
         done += len(seqs)
         passes += 1
+    # one thread, on a smaller sample of the same sequences
+    n1, b1, t1 = 0, 0, 0.0
+    while t1 < max(1.0, target_s / 6) and n1 < batch.num_seqs:
+        seqs = order[n1: n1 + 2]
+        t = time.perf_counter()
+        _oracle_pass(batch, kp, vp, seqs, threads=1)
+        t1 += time.perf_counter() - t
+        b1 += decode_step_bytes(batch.context_lens[seqs], batch.num_q_heads,
+                                batch.num_kv_heads, batch.head_dim, batch.block_size)["total"]
+        n1 += len(seqs)
     return {"value": round(nbytes / t_used / 1e9, 4), "unit": "GB/s", "cores": cores,
             "kind": "oracle",
             "sample": f"{done} sequences of the batch (8 per call, {passes} calls, "
                       f"{t_used:.1f} s), fp64, OpenMP over (sequence, q head)",
-            "query_tokens_per_s": round(done / t_used, 2)}
+            "query_tokens_per_s": round(done / t_used, 2),
+            "single_thread": {"value": round(b1 / t1 / 1e9, 4), "unit": "GB/s",
+                              "sample": f"{n1} sequences (2 per call, {t1:.1f} s), one thread"}}
 
 
 def run_reference(args, rank, world):
