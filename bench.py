@@ -46,7 +46,7 @@ if ROOT not in sys.path:
 
 import synth  # noqa: E402
 from paged_kv_cache_370_b200.accounting import (decode_step_bytes, new_token_bytes,  # noqa: E402
-                                                split_scratch_bytes)
+                                                split_scratch_bytes, tail_overread_bytes)
 
 METRIC = "paged decode attention: KV GB/s and % of B200 HBM peak; query tokens/s"
 NOMINAL_HBM_GBS = 8000.0
@@ -298,6 +298,7 @@ def _byte_info(lens, hq, hkv, d, bs, pt, ntok, window=0):
         lens = np.minimum(np.asarray(lens), window)
     return {"decode": decode_step_bytes(lens, hq, hkv, d, bs),
             "scratch": split_scratch_bytes(lens, hq, d, pt),
+            "tail": tail_overread_bytes(lens, hkv, d, bs),
             "write": new_token_bytes(ntok, hkv, d), "lens": np.asarray(lens)}
 
 
@@ -540,7 +541,9 @@ def run_ours(args, rank, world, local, dist):
         "extra_bytes_per_step": {"split_scratch": int(np.mean([infos[i % V]["scratch"]
                                                                for i in range(K)])),
                                  "kv_write": int(infos[0]["write"]),
-                                 "copy_on_write": int(infos[0].get("copy", 0))},
+                                 "copy_on_write": int(infos[0].get("copy", 0)),
+                                 "tail_overread": int(np.mean([infos[i % V]["tail"]
+                                                               for i in range(K)]))},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }

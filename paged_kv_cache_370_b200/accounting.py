@@ -41,6 +41,15 @@ def decode_step_bytes(context_lens, num_q_heads: int, num_kv_heads: int, head_di
             "total": kv + q + out + tables + ctx}
 
 
+def tail_overread_bytes(context_lens, num_kv_heads: int, head_dim: int, block_size: int,
+                        elem_bytes: int = 2) -> int:
+    """K and V bytes of the unfilled tail rows of each sequence's last block, which a
+    kernel that copies whole blocks reads beyond the algorithmic bytes."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    tail = blocks_needed(lens, block_size) * block_size - lens
+    return int(2 * tail.sum() * num_kv_heads * head_dim * elem_bytes)
+
+
 def split_scratch_bytes(context_lens, num_q_heads: int, head_dim: int, partition_tokens: int) -> int:
     """Workspace bytes written and read back for sequences split into more than
     one partition: (head_dim + 2) fp32 per (sequence, q head, partition), twice."""

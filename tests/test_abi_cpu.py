@@ -442,6 +442,13 @@ def test_decode_step_bytes():
     assert b["total"] == b["kv"] + 2 * 3 * 32 * 128 * 2 + 20 + 12
 
 
+def test_tail_overread_bytes():
+    from paged_kv_cache_370_b200.accounting import tail_overread_bytes
+    # whole blocks read for lengths 1, 17, 32 at block size 16: 15 + 15 + 0 unfilled rows
+    assert tail_overread_bytes([1, 17, 32], 8, 128, 16) == 2 * 30 * 8 * 128 * 2
+    assert tail_overread_bytes([0, 16], 8, 128, 16) == 0
+
+
 def test_slide_window_releases_only_blocks_before_the_window():
     m = BlockManager(16, 4)
     m.add_seq(0, 10)                       # blocks for positions 0-3, 4-7, 8-9
