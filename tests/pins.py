@@ -201,6 +201,32 @@ def pin_bruteforce_fsum():
                 assert abs(got[b, h, d] - ref) <= 1e-13, "brute force disagrees"
 
 
+def pin_decode_one_bruteforce():
+    """The single-(sequence, q head) entry point used to check sampled outputs of
+    large batches, against the same pure-Python brute force: every head of every
+    sequence, each through its own table row, length and kv head."""
+    batch = synth.small_random(24, 3, [3, 9, 14], 4, 2, 8, 4, 12, "f16")
+    kp, vp = place_numpy(batch)
+    G = batch.num_q_heads // batch.num_kv_heads
+    q = lib_f64(batch.q, batch.dtype).tolist()
+    for b in range(batch.num_seqs):
+        K = lib_f64(batch.k[batch.rows(b)], batch.dtype).tolist()
+        V = lib_f64(batch.v[batch.rows(b)], batch.dtype).tolist()
+        n = len(K)
+        for h in range(batch.num_q_heads):
+            g = h // G
+            got = oracle.decode_one(batch.q[b, h], kp, vp, batch.block_tables[b],
+                                    int(batch.context_lens[b]), g, batch.scale, batch.dtype)
+            s = [float(batch.scale) * math.fsum(q[b][h][d] * K[t][g][d]
+                                                for d in range(batch.head_dim)) for t in range(n)]
+            m = max(s)
+            w = [math.exp(x - m) for x in s]
+            den = math.fsum(w)
+            for d in range(batch.head_dim):
+                ref = math.fsum(w[t] * V[t][g][d] for t in range(n)) / den
+                assert abs(got[d] - ref) <= 1e-13, "decode_one disagrees with brute force"
+
+
 def pin_relabel():
     batch = synth.small_random(24, 4, [13, 30, 2, 47], 4, 2, 16, 8, 40, "f16")
     kp, vp = place_numpy(batch)
@@ -774,7 +800,8 @@ def pin_allocator_prefix_cache_bruteforce():
 
 ALL_ORACLE_PINS = [
     pin_f16_decoder, pin_bf16_decoder, pin_worked_example_slots, pin_bs16_tables, pin_dense,
-    pin_len1_returns_v, pin_identical_keys_mean_v, pin_bruteforce_fsum, pin_relabel, pin_poison,
+    pin_len1_returns_v, pin_identical_keys_mean_v, pin_bruteforce_fsum, pin_decode_one_bruteforce,
+    pin_relabel, pin_poison,
     pin_partition_merge, pin_reshape_layout, pin_copy_blocks, pin_window_dense,
     pin_window_one_returns_last_v, pin_window_ignores_what_it_left, pin_window_bruteforce_fsum,
     pin_swap_blocks, pin_prefill_dense, pin_prefill_first_token_of_a_prompt,
