@@ -9,7 +9,11 @@
 // K/V already written to the pool), and the token at position p attends to
 // positions [lo, p] -- lo = p + 1 - window under a sliding window, else 0.
 //
-// Design:
+// Two kernels compute it. The default (pa_prefill_tc_kernel, further down)
+// runs both products on the 5th-generation tensor cores (tcgen05.mma, S, P
+// and O in tensor memory, 256 query rows per CTA). The first version
+// (pa_prefill_kernel, selected with -DPA_PREFILL_TCGEN05=0) uses mma.sync with
+// register accumulators; its design:
 //  * One CTA per (q head, 64 query tokens, sequence); the q heads of one kv
 //    head are neighbours in the grid, so the CTAs sharing a K/V tile run
 //    together and all but the first read it from L2. Tiles with the most keys
