@@ -560,6 +560,52 @@ def pin_swap_blocks():
     assert np.array_equal(dk2[untouched], dk[untouched]), "swap in wrote outside its pairs"
 
 
+# --------------------------------------------------------------------------- placement helpers
+def pin_place_history():
+    """The oracle's placement helper (the pools every GPU parity test compares
+    against) equals the independent numpy placement bit for bit, with and
+    without each sequence's last position: block sizes 4..32, lengths 0, 1,
+    block-aligned and ragged, both dtypes, GQA and MHA."""
+    extra = synth.small_random(26, 4, [0, 1, 4, 9], 4, 2, 16, 4, 16, "f16")
+    for batch in small_batches() + [extra]:
+        for include_new in (True, False):
+            want_k, want_v = place_numpy(batch, include_new=include_new, poison=True)
+            kp = np.full_like(want_k, NAN_BITS[batch.dtype])
+            vp = np.full_like(want_v, NAN_BITS[batch.dtype])
+            oracle.place_history(batch, kp, vp, include_new=include_new)
+            assert np.array_equal(kp, want_k), f"{batch.name}: K placement (new={include_new})"
+            assert np.array_equal(vp, want_v), f"{batch.name}: V placement (new={include_new})"
+
+
+def pin_new_token_slots():
+    """The slot where each sequence's step token is written, on the worked example
+    of page "大语言模型推理内存管理算法 paged attention", section 8 (block size 4,
+    logical blocks 0, 1, 2 in physical blocks 8, 3, 15) with the slot formula of
+    page "08. PagedAttention：把 KV Cache 分页管理", section "为什么叫
+    PagedAttention". A sequence of length n writes position n - 1: with 11 tokens
+    that is the 11th token, still in logical block 2, i.e. 15 * 4 + 2 = 62; with 12
+    tokens 15 * 4 + 3 = 63. Every length 0..12 is checked against the fixture's
+    block ranges; length 0 has no token (-1)."""
+    import types
+    g = read_golden("worked_example_bs4.txt")
+    bs = int(g["block_size"][0][0])
+    physical = [int(x) for x in g["physical"][0]]
+    ranges = [(int(v[0]), int(v[2]), int(v[3])) for v in g["logical_block"]]
+    lens = np.arange(0, 13, dtype=np.int32)
+    batch = types.SimpleNamespace(num_seqs=len(lens), block_size=bs, context_lens=lens,
+                                  block_tables=np.tile(np.array(physical, np.int32),
+                                                       (len(lens), 1)))
+    got = oracle.new_token_slots(batch)
+    assert got.dtype == np.int64 and got.shape == (len(lens),)
+    for n, s in zip(lens.tolist(), got.tolist()):
+        if n == 0:
+            assert s == -1, "an empty sequence writes nothing"
+            continue
+        lb, lo, _ = next(r for r in ranges if r[1] <= n - 1 <= r[2])
+        assert s == physical[lb] * bs + (n - 1 - lo), f"length {n}: slot {s}"
+    assert got[11] == 62 and got[12] == 63
+
+
 # --------------------------------------------------------------------------- block manager
 def pin_allocator_worked_example():
     g = read_golden("worked_example_bs4.txt")
@@ -805,7 +851,8 @@ ALL_ORACLE_PINS = [
     pin_partition_merge, pin_reshape_layout, pin_copy_blocks, pin_window_dense,
     pin_window_one_returns_last_v, pin_window_ignores_what_it_left, pin_window_bruteforce_fsum,
     pin_swap_blocks, pin_prefill_dense, pin_prefill_first_token_of_a_prompt,
-    pin_prefill_bruteforce_fsum, pin_prefill_relabel,
+    pin_prefill_bruteforce_fsum, pin_prefill_relabel, pin_place_history,
+    pin_new_token_slots,
 ]
 ALL_MODEL_PINS = [pin_allocator_worked_example, pin_allocator_capacity, pin_allocator_cow,
                   pin_allocator_sliding_window, pin_allocator_swap, pin_allocator_prefix_cache,

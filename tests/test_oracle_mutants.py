@@ -114,3 +114,38 @@ def test_model_pins_catch_mutant(name, tmp_path, monkeypatch):
             caught.append((pin.__name__, type(e).__name__))
             break
     assert caught, f"no model pin caught the planted mistake {name}"
+
+
+# Plausible mistakes in the oracle's Python placement helpers
+# (oracle/__init__.py: place_history, new_token_slots), which build the pools
+# every GPU parity test compares against; the oracle pins must catch each.
+HELPER_MUTANTS = {
+    "history_keeps_new_token": ("n = int(batch.context_lens[b]) - (0 if include_new else 1)",
+                                "n = int(batch.context_lens[b])"),
+    "history_drops_one_more": ("n = int(batch.context_lens[b]) - (0 if include_new else 1)",
+                               "n = int(batch.context_lens[b]) - 1"),
+    "new_token_at_len": ("slot(batch.block_tables[b], int(batch.context_lens[b]) - 1,",
+                         "slot(batch.block_tables[b], int(batch.context_lens[b]),"),
+    "new_token_first_position": ("slot(batch.block_tables[b], int(batch.context_lens[b]) - 1,",
+                                 "slot(batch.block_tables[b], 0 * int(batch.context_lens[b]),"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(HELPER_MUTANTS))
+def test_pins_catch_helper_mutant(name, monkeypatch):
+    old, new = HELPER_MUTANTS[name]
+    src = open(oracle.__file__).read()
+    assert src.count(old) == 1, f"anchor of mutant {name} not found once in oracle/__init__.py"
+    # the module re-executed from the mutated text; it loads the same compiled oracle
+    ns = {"__name__": "oracle_mutant", "__file__": oracle.__file__}
+    exec(compile(src.replace(old, new), oracle.__file__, "exec"), ns)
+    monkeypatch.setattr(oracle, "place_history", ns["place_history"])
+    monkeypatch.setattr(oracle, "new_token_slots", ns["new_token_slots"])
+    caught = []
+    for pin in pins.ALL_ORACLE_PINS:
+        try:
+            pin()
+        except Exception as e:  # noqa: BLE001 -- any failure of a pin counts
+            caught.append((pin.__name__, type(e).__name__))
+            break
+    assert caught, f"no pin caught the planted mistake {name}"
