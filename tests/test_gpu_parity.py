@@ -197,7 +197,9 @@ def _full_size(batch, partition_tokens=0, fused=False):
     _sampled_pool_check(g, batch)
     kp, vp = oracle_pools(batch, full=False)
     ref = oracle_decode(batch, kp, vp)
-    s = assert_close(out, ref, batch.dtype, batch.name)
+    # the long-context batch's keys scaled x8 collapse some softmaxes onto one V row:
+    # outputs of magnitude >= 4, where bf16 itself is spaced 2^-5 apart
+    s = assert_close(out, ref, batch.dtype, batch.name, ulp_branch=batch.name == "long_skew")
     print(f"\n{batch.name}: {s}")
     return g, out, s
 

@@ -82,7 +82,8 @@ def test_prefill_shapes(shape, window):
     g = GpuPrefill(batch)
     out = widen_out(g.run(window))
     _status_clean()
-    assert_close(out, _oracle(batch, window), dt, f"prefill {shape[:5]} window {window}")
+    assert_close(out, _oracle(batch, window), dt, f"prefill {shape[:5]} window {window}",
+                 ulp_branch=True)
 
 
 def test_prefill_single_tokens_match_decode():
@@ -132,8 +133,8 @@ def test_prefill_llama8b_full():
     rng = np.random.default_rng(4)
     qs = batch.meta["q_start"]
     T = int(qs[-1])
-    toks = rng.choice(T, size=500, replace=False)
-    heads = rng.integers(0, batch.num_q_heads, size=500)
+    toks = rng.choice(T, size=2000, replace=False)
+    heads = rng.integers(0, batch.num_q_heads, size=2000)
     G = batch.num_q_heads // batch.num_kv_heads
     got, ref = [], []
     for tok, h in zip(toks, heads):
@@ -143,5 +144,6 @@ def test_prefill_llama8b_full():
         ref.append(oracle.decode_one(batch.q[tok, h], kp, vp, batch.block_tables[b], pos + 1,
                                      int(h) // G, batch.scale, batch.dtype))
         got.append(out[tok, h])
-    s = assert_close(np.array(got)[None], np.array(ref)[None], batch.dtype, "llama8b prefill")
+    s = assert_close(np.array(got)[None], np.array(ref)[None], batch.dtype, "llama8b prefill",
+                     ulp_branch=True)
     print(f"\nllama8b prefill sample: {s}")

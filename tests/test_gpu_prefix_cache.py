@@ -98,7 +98,7 @@ def test_prefix_cached_prefill():
     # r0 again: its 4 full blocks (its last token's block is computed)
     assert cached == [0, 32, 32, 0, 64]
     assert abi.pa_device_status() == 0
-    assert_close(out, ref, DT, "prefix-cached prefill")
+    assert_close(out, ref, DT, "prefix-cached prefill", ulp_branch=True)
     for sid in range(len(prompts)):
         mgr.free_seq(sid)
         model.free_seq(sid)
@@ -108,4 +108,5 @@ def test_prefix_cached_prefill():
     out2, ref2, cached2 = _step(mgr, model, kc, vc, prompts2, 100)
     assert cached2 == [32, 64, 0]
     assert abi.pa_device_status() == 0
-    assert_close(out2, ref2, DT, "prefill from blocks cached after the requests ended")
+    assert_close(out2, ref2, DT, "prefill from blocks cached after the requests ended",
+                 ulp_branch=True)

@@ -60,10 +60,12 @@ def _window_case(batch, window, partition_tokens=0, fused=False, sample=None):
     if sample is None:
         ref = oracle.decode_window(batch.q, kp, vp, batch.block_tables, batch.context_lens,
                                    batch.scale, batch.dtype, window)
-        return assert_close(out, ref, batch.dtype, f"{batch.name} window {window}")
+        return assert_close(out, ref, batch.dtype, f"{batch.name} window {window}",
+                            ulp_branch=batch.name == "long_skew")
     ref = oracle.decode_window(batch.q[sample], kp, vp, batch.block_tables[sample],
                                batch.context_lens[sample], batch.scale, batch.dtype, window)
-    return assert_close(out[sample], ref, batch.dtype, f"{batch.name} window {window}")
+    return assert_close(out[sample], ref, batch.dtype, f"{batch.name} window {window}",
+                        ulp_branch=batch.name == "long_skew")
 
 
 SHAPES = [

@@ -1,11 +1,23 @@
 """Tolerance of attention outputs against the fp64 oracle.
 
 Bound: max abs error <= 1e-2 and mean abs error <= 1e-3 (bf16/fp16 output,
-fp32 accumulation). Where the output format itself cannot meet 1e-2 -- a bf16
-value of magnitude >= 4 is spaced 2^-5 apart, so even the correctly rounded
-result can be 0.0156 away -- an element may instead be within one unit in the
-last place of the output format at the reference value. The number of
-elements that needed that allowance is reported.
+fp32 accumulation), element by element.
+
+Where the output format itself cannot meet 1e-2 the bound is widened, and
+only where a caller allows it: a bf16 value of magnitude >= 4 is spaced 2^-5
+apart, so even the correctly rounded result can lie 2^-6 = 0.0156 from the
+exact one. The kernels round an fp32 result to the output type once (nearest
+even), so the output is at most half a unit in the last place from that fp32
+result; the fp32 result itself is held to the mean-error bound 1e-3 of the
+exact value. An allowed element therefore passes when it is within
+max(1e-2, ulp_out(ref) / 2 + 1e-3) of the reference: half a unit of the
+output format plus the arithmetic's 1e-3. For bf16 this is wider than 1e-2
+only at magnitudes >= 4 (fp16: >= 32), which the workloads reach only where
+the softmax collapses onto one large V row (the long-context batch's scaled
+keys) or averages a handful of rows (the first positions of a prompt in
+prefill, short sliding windows). Everywhere else callers leave the allowance
+off, so any element beyond 1e-2 fails. The number of elements that used the
+allowance is reported.
 """
 from __future__ import annotations
 
@@ -16,6 +28,7 @@ MEAN_TOL = 1e-3
 
 
 def out_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
+    """Spacing of the output format's representable values at |ref|."""
     a = np.abs(np.asarray(ref, dtype=np.float64))
     if dtype == "f16":
         e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
@@ -27,7 +40,7 @@ def out_ulp(ref: np.ndarray, dtype: str) -> np.ndarray:
 def compare(got: np.ndarray, ref: np.ndarray, dtype: str) -> dict:
     got = np.asarray(got, dtype=np.float64)
     err = np.abs(got - ref)
-    tol = np.maximum(ATOL, out_ulp(ref, dtype))
+    tol = np.maximum(ATOL, out_ulp(ref, dtype) / 2 + MEAN_TOL)
     finite = np.isfinite(got)
     bad = (err > tol) | ~finite
     floor = np.abs(_round_like(ref, dtype) - ref)
@@ -38,13 +51,19 @@ def compare(got: np.ndarray, ref: np.ndarray, dtype: str) -> dict:
         "n_bad": int(bad.sum()),
         "n_ulp_branch": int(((err > ATOL) & ~bad).sum()),
         "rounding_floor_mean": float(floor.mean()) if floor.size else 0.0,
+        "rounding_floor_max": float(floor.max()) if floor.size else 0.0,
     }
 
 
-def assert_close(got, ref, dtype, what=""):
+def assert_close(got, ref, dtype, what="", ulp_branch=False):
+    """Element-wise check against the oracle. ``ulp_branch``: allow, element by
+    element, half a unit of the output format plus 1e-3 where that exceeds 1e-2
+    (see the module docstring); otherwise every element must be within 1e-2."""
     s = compare(got, ref, dtype)
     assert s["n_bad"] == 0, f"{what}: {s['n_bad']} elements outside tolerance; {s}"
     assert s["mean_abs"] <= MEAN_TOL, f"{what}: mean abs error {s['mean_abs']}; {s}"
+    if not ulp_branch:
+        assert s["n_ulp_branch"] == 0, f"{what}: {s['n_ulp_branch']} elements beyond 1e-2; {s}"
     return s
 
 
