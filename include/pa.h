@@ -195,15 +195,23 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
  * inside the library, which every GPU that loads the library holds until the
  * process exits. The caller still passes q, the pools, the tables, the lengths
  * and the output.
- *  - Calls that would need more scratch than PA_STATIC_WORKSPACE_BYTES (see
- *    pa_decode_workspace_size) return PA_ERR_UNSUPPORTED and launch nothing.
+ *  - Calls whose kernel would need more scratch than PA_STATIC_WORKSPACE_BYTES
+ *    return PA_ERR_UNSUPPORTED and launch nothing. The need is that of the
+ *    kernel the call runs (for the given block_size), which is at most
+ *    pa_decode_workspace_size.
  *  - The first call on a device (made with that device current) looks up the
  *    array's device address; make that first call before any stream capture.
+ *    Only a successful lookup is kept (a failure returns PA_ERR_CUDA and the
+ *    next call tries again).
  *  - No device memory is allocated or freed, by this library or any other.
- *  - All calls share the one array and it keeps the last call's contents. It
- *    needs no clearing (each call writes every entry it later reads), but calls
- *    whose work overlaps on the GPU (other streams, other host threads) race on
- *    it: serialise them.
+ *  - All calls share the one array and it keeps the last call's contents. Its
+ *    first 64 KiB hold the even-split kernel's counters, which a call expects
+ *    at zero and which a call that gave up a wait (PA_DEVERR_TIMEOUT) may leave
+ *    non-zero; so every call first clears them on `stream` (a memset, not an
+ *    allocation) before its kernels. Calls whose work overlaps on the GPU
+ *    (other streams, other host threads) race on the array -- one may clear or
+ *    overwrite what the other is using, and both outputs are then undefined:
+ *    serialise them.
  * ------------------------------------------------------------------------------------------ */
 #define PA_STATIC_WORKSPACE_BYTES (16u << 20)
 
@@ -343,6 +351,13 @@ int pa_decode_append_launches(int num_seqs, int num_q_heads, int num_kv_heads, i
                               int block_size, int num_blocks, int max_context_len,
                               int partition_tokens);
 
+/* CTAs of the even-split kernel a pa_decode call with these arguments launches (one
+ * persistent wave on the current device by default), or 0 when the call runs the
+ * partition kernel instead. For accounting (e.g. the split-context scratch bytes). */
+int pa_decode_grid_ctas(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                        int block_size, int num_blocks, int max_context_len,
+                        int partition_tokens);
+
 /* Kernels one pa_decode call with these arguments launches (0 if none). */
 int pa_decode_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                        int block_size, int num_blocks, int max_context_len, int partition_tokens);
@@ -356,6 +371,23 @@ int pa_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_
  * `stream`; meant for tests and debugging, not the hot path.
  * ------------------------------------------------------------------------------------------ */
 pa_status pa_device_status(void *stream, int32_t *code);
+
+/* ------------------------------------------------------------------------------------------
+ * pa_debug_wait_test -- test hook for the bounded waits of the decode kernels (not for
+ * production use; the pages have no counterpart).
+ * Every wait of a decode kernel is bounded: a wait that runs out sets PA_DEVERR_TIMEOUT,
+ * and the kernel then runs to its end without waiting for data again (so every warp
+ * reaches every barrier), issues no further copy, skips the fused KV write, and
+ * returns; its outputs are undefined, everything it writes stays in bounds, and the
+ * context stays usable. With enable != 0, every later pa_decode* launch runs in a test
+ * mode that makes this happen on purpose and safely: its producer warps issue no copy
+ * and arrive on no data barrier, and its consumer warps give up each data wait after
+ * consumer_wait_ns nanoseconds (0 < consumer_wait_ns <= 2e9). No copy is then in flight
+ * when a CTA exits. enable == 0 restores normal launches (waits bounded at 2 s).
+ * Process-wide and not thread-safe: set it only while no other thread launches decode
+ * work. PA_ERR_INVALID for an out-of-range limit.
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_debug_wait_test(int enable, long long consumer_wait_ns);
 
 /* Human-readable name of a status code (static storage). */
 const char *pa_status_string(pa_status status);

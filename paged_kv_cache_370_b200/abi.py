@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "pa_decode": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, P, sz, i, P]),
         "pa_decode_default_partition": (i, [i, i, i]),
         "pa_decode_launches": (i, [i, i, i, i, i, i, i, i]),
+        "pa_decode_grid_ctas": (i, [i, i, i, i, i, i, i, i]),
+        "pa_debug_wait_test": (i, [i, ctypes.c_longlong]),
         "pa_decode_append": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, P, sz,
                                  i, P]),
         "pa_decode_append_launches": (i, [i, i, i, i, i, i, i, i]),
@@ -382,6 +384,22 @@ def pa_decode_static_workspace(out, q, k_cache, v_cache, block_tables, context_l
         B, hq, hkv, d, bs, nb, float(scale), _dtype_code(q), int(partition_tokens),
         _stream(stream))
     _check(st, "pa_decode_static_workspace")
+
+
+def pa_decode_grid_ctas(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                        max_context_len, partition_tokens=0) -> int:
+    """CTAs of the even-split kernel such a pa_decode call launches (0: the
+    partition kernel runs instead)."""
+    return int(_lib.pa_decode_grid_ctas(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                        block_size, num_blocks, max_context_len,
+                                        partition_tokens))
+
+
+def pa_debug_wait_test(enable: bool, consumer_wait_ns: int = 0):
+    """Test hook: later decode launches make their bounded data waits run out
+    (no copies issued); see include/pa.h. enable=False restores normal launches."""
+    _check(_lib.pa_debug_wait_test(1 if enable else 0, int(consumer_wait_ns)),
+           "pa_debug_wait_test")
 
 
 def pa_device_status(stream=None) -> int:

@@ -40,6 +40,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -57,17 +58,34 @@ constexpr int kStages = 4;
 constexpr int kTileBytes = 8192;                 // bytes of K (and of V) per stage
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
-// Wait for phase `parity` of `bar` to complete, at most kWaitLimitNs; also give
-// up when another thread of the CTA has raised *abort. Returns false on give-up.
+// Wait for phase `parity` of `bar` to complete, at most limit_ns; also give up
+// when another thread of the CTA has raised *abort. Returns false on give-up
+// (and then raises *abort and the device error bit).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  volatile int *abort) {
+                                                  volatile int *abort,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_ns() - t0 > kWaitLimitNs) {
+    if (global_ns() - t0 > limit_ns) {
       *abort = 1;
+      atomicOr(&g_decode_error, PA_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// The same wait without the early exit on *abort: for barriers whose arrivals
+// do not depend on any copy landing (they always come), so that a give-up
+// elsewhere in the CTA cannot let one warp run ahead of another.
+__device__ __forceinline__ bool mbar_wait_sure(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
       atomicOr(&g_decode_error, PA_DEVERR_TIMEOUT);
       return false;
     }
@@ -145,6 +163,11 @@ struct DecodeParams {
   const int32_t *win_skip;
   // even-split kernel launched as a programmatic dependent of the preceding kernel
   int early_start;
+  // limit of the consumers' waits for a stage's data (normally kWaitLimitNs)
+  unsigned long long wait_ns;
+  // test mode of the bounded waits: the producers issue no copy and arrive on no
+  // data barrier, so every data wait runs out (pa_debug_wait_test)
+  int starve;
 };
 
 // First position attended by a sequence of length len under a window of w
@@ -265,6 +288,10 @@ __global__ void __launch_bounds__(kThreads, 3)
           }
           bytes += 2u * (uint32_t)(r1 - r0) * D * sizeof(T);
         }
+        if (p.starve) {  // test mode: no copy, no arrival (the consumers' waits run out)
+          issued = i + 1;
+          continue;
+        }
         mbar_expect_tx_arrive(&full_bar[s], bytes);
         unsigned char *stage = smem + s * L::kStageBytes;
         for (int blk = t0 / p.block_size; blk <= (t1 - 1) / p.block_size; ++blk) {
@@ -281,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 3)
         issued = i + 1;
       }
       // do not leave while copies may still land in this CTA's shared memory
-      for (int i = max(0, issued - kStages); i < issued; ++i) {
+      for (int i = max(0, issued - kStages); i < issued && !p.starve; ++i) {
         const int s = i % kStages;
         const unsigned long long t_start = global_ns();
         while (!mbar_try_wait(&full_bar[s], (i / kStages) & 1)) {
@@ -339,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     const int s = i % kStages;
     // every lane waits; the warp then leaves together or not at all, so the
     // warp-wide shuffles below always see all 32 lanes
-    const bool landed = mbar_wait_bounded(&full_bar[s], (i / kStages) & 1, abort_flag);
+    const bool landed = mbar_wait_bounded(&full_bar[s], (i / kStages) & 1, abort_flag, p.wait_ns);
     if (!__all_sync(0xffffffffu, landed)) break;
     const unsigned char *stage = smem + s * L::kStageBytes;
     const uint4 *Ks = reinterpret_cast<const uint4 *>(stage);
@@ -543,6 +570,7 @@ __global__ void __launch_bounds__(kThreads, 3)
 #define PA_STREAM_STAGES_D64 4
 #endif
 
+
 namespace tc {
 
 constexpr int kTile = 64;            // tokens per stage
@@ -581,7 +609,7 @@ struct Cfg {
   static constexpr int kRedBytes = kWarps * G * D * 4;
   static constexpr int kMetaOffset = kRedOffset + kRedBytes;
   static constexpr int kBarOffset = kMetaOffset + kStages * (int)sizeof(TileMeta);
-  static constexpr int kMlOffset = kBarOffset + 2 * kStages * 8;
+  static constexpr int kMlOffset = kBarOffset + 3 * kStages * 8;  // full, empty, meta barriers
   static constexpr int kIdsOffset = kMlOffset + kWarps * 8 * 2 * 4;
   static constexpr int kCtrlOffset = kIdsOffset + 2 * kIdWindow * 8 * 4;  // one window per producer
   static constexpr int kBytes = 1024 + kCtrlOffset + 64;  // + slack to align the ring to 1 KB
@@ -634,6 +662,10 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
   uint64_t *empty_bar = full_bar + NS;
+  // meta_bar[s]: the tile's metadata is in meta[s] (one arrival per tile, even
+  // when the stage's data copies are not issued); the consumers take the metadata
+  // through it after a give-up, so they never read metadata not yet written.
+  uint64_t *meta_bar = empty_bar + NS;
   TileMeta *meta = reinterpret_cast<TileMeta *>(smem + C::kMetaOffset);
   float *mlbuf = reinterpret_cast<float *>(smem + C::kMlOffset);
   float *red = reinterpret_cast<float *>(smem + C::kRedOffset);
@@ -671,6 +703,7 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], kWarps);
+      mbar_init(&meta_bar[s], 1);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -771,10 +804,18 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     // otherwise), then let the next kernel start its own prologue.
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // the copies of the last NS tiles this warp issued (bit k: tile ntiles - NS + k)
+    uint32_t issued_mask = 0;
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % NS;
-      // stage free? (after a give-up the loop runs on without waiting: no early exits)
-      if (i >= NS) mbar_wait_bounded(&empty_bar[s], ((i / NS) & 1) ^ 1, abort_flag);
+      // stage free? The consumers arrive once per tile whatever happened, so this
+      // wait does not stop at a give-up: the producer never runs a full ring ahead
+      // and never rewrites metadata the consumers may still read
+      if (i >= NS) mbar_wait_sure(&empty_bar[s], ((i / NS) & 1) ^ 1);
+      // copies go out only while nothing has given up (and never in the test mode):
+      // a stage whose data never landed is not armed a second time
+      const bool issue = __shfl_sync(0xffffffffu, !p.starve && !*abort_flag, 0);
+      issued_mask = (issued_mask >> 1) | (issue ? 1u << (NS - 1) : 0u);
       __syncwarp();
       // this tile's ids have landed once at most kIdWindow - 1 newer groups are pending
       cp_async_wait<kIdWindow - 1>();
@@ -803,9 +844,11 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         m.flags = (seg_begin ? 1 : 0) | (seg_end ? 2 : 0) | (new_tok ? 4 : 0);
         m.nskip = (kWindow && j == 0) ? min(max(__ldg(p.win_skip + b), 0), kTile - 1) : 0;
         m.new_slot = slot_b;
-        mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes +
-                                                (seg_begin ? (uint32_t)C::kQBytes : 0u) +
-                                                (new_tok ? (uint32_t)C::kNewBytes : 0u));
+        if (issue)
+          mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes +
+                                                  (seg_begin ? (uint32_t)C::kQBytes : 0u) +
+                                                  (new_tok ? (uint32_t)C::kNewBytes : 0u));
+        mbar_arrive(&meta_bar[s]);
       }
       __syncwarp();
       const uint32_t stage = ring + s * C::kStageBytes;
@@ -816,7 +859,7 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         const int pn = lane % C::kPanels;
         const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
         const bool box_ok = box < 32 && ((okmask >> (box & 31)) & 1u);
-        if (box_ok) {
+        if (box_ok && issue) {
           // box of block t0/bs + box: whole block (bs <= 64) or a 64-row slice (bs > 64)
           const int r0 = bs > kTile ? t0 % bs : 0;
           const int row = bs > kTile ? 0 : box * bs;
@@ -825,11 +868,11 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
                       which ? &tmap_v : &tmap_k, pn * 64, y, &full_bar[s]);
         }
       }
-      if (lane == 0 && seg_begin && !v_producer)
+      if (lane == 0 && seg_begin && !v_producer && issue)
         bulk_g2s(smem + C::kQOffset + s * C::kQBytes,
                  static_cast<const T *>(p.q) + ((size_t)b * p.num_q_heads + (size_t)kvh * G) * D,
                  C::kQBytes, &full_bar[s]);
-      if (lane == 0 && new_tok && !v_producer) {
+      if (lane == 0 && new_tok && !v_producer && issue) {
         const size_t row = ((size_t)b * Hkv + kvh) * D;
         unsigned char *dst = smem + C::kNewOffset + s * C::kNewBytes;
         bulk_g2s(dst, static_cast<const T *>(p.k_new) + row, D * 2, &full_bar[s]);
@@ -861,6 +904,7 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     // do not leave while copies may still land in this CTA's shared memory
     if (lane == 0) {
       for (int i = max(0, ntiles - NS); i < ntiles; ++i) {
+        if (!((issued_mask >> (i - (ntiles - NS))) & 1u)) continue;  // nothing issued there
         const int s = i % NS;
         const unsigned long long t_start = global_ns();
         while (!mbar_try_wait(&full_bar[s], (i / NS) & 1)) {
@@ -888,12 +932,27 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
   uint32_t qb[KSTEPS][2];
   float o[KSTEPS][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  bool gave_up = false;  // a data wait of this warp has failed
 
   for (int i = 0; i < ntiles; ++i) {
     const int s = i % NS;
     // after a give-up the loop runs on (on whatever the stage holds) so every
-    // consumer warp reaches every barrier below
-    mbar_wait_bounded(&full_bar[s], (i / NS) & 1, abort_flag);
+    // consumer warp reaches every barrier below. A give-up leaves data barriers'
+    // phases behind: a stage that is not armed again never completes, and a parity
+    // wait on it then reports the older phase as done. Such a stale success can
+    // only come after this warp's own wait on that stage failed (every warp waits
+    // on every tile in order), so once this warp has seen a failed wait no data
+    // wait counts as landed, and the metadata comes through its own barrier, which
+    // completes once per tile whatever happened: all warps read the same, fully
+    // written metadata. Until then a landed stage carries its metadata (written
+    // before the producer's arrival).
+    const bool ok = __all_sync(
+        0xffffffffu, mbar_wait_bounded(&full_bar[s], (i / NS) & 1, abort_flag, p.wait_ns));
+    const bool landed = ok && !gave_up;
+    if (!landed) {
+      gave_up = true;
+      mbar_wait_sure(&meta_bar[s], (i / NS) & 1);
+    }
     __syncwarp();
     const TileMeta mt = meta[s];
     const uint32_t kst = ring + s * C::kStageBytes;
@@ -914,9 +973,10 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     }
     const int nvalid = mt.nvalid;
     const int nskip = kWindow ? mt.nskip : 0;
-    if ((mt.flags & 4) && (nvalid - 1) / 16 == warp) {
+    if ((mt.flags & 4) && landed && (nvalid - 1) / 16 == warp) {
       // fused write: the new token (last valid row) replaces what the cache held
-      // in this tile, and is stored at its slot for later steps
+      // in this tile, and is stored at its slot for later steps (not after a
+      // give-up: the copied rows may not have landed)
       constexpr int kChunks = D / 8;  // 16-byte chunks per row
       const int r = nvalid - 1;
       if (lane < 2 * kChunks) {
@@ -1285,7 +1345,7 @@ bool ensure_smem(Kernel kernel, size_t smem, size_t (&configured)[kMaxDevices]) 
 // Bytes at the start of every workspace that hold the even-split kernel's
 // counters; they must be zero before the first call and every call leaves them
 // zero. The split-partition scratch of the SIMT path starts after them.
-constexpr size_t kCounterRegion = 64 * 1024;
+constexpr size_t kCounterRegion = kPaCounterRegionBytes;
 constexpr int kMaxStreamCtas = (int)(kCounterRegion / sizeof(int));
 
 int sm_count() {
@@ -1454,7 +1514,19 @@ int resolve_partition(int num_seqs, int num_kv_heads, int max_context_len, int r
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Test mode of the bounded waits (pa_debug_wait_test): read at every launch.
+std::atomic<int> g_wait_test{0};
+std::atomic<long long> g_wait_test_ns{0};
+
 }  // namespace
+
+extern "C" pa_status pa_debug_wait_test(int enable, long long consumer_wait_ns) {
+  if (enable && (consumer_wait_ns <= 0 || consumer_wait_ns > (long long)kWaitLimitNs))
+    return PA_ERR_INVALID;
+  g_wait_test_ns.store(enable ? consumer_wait_ns : 0);
+  g_wait_test.store(enable ? 1 : 0);
+  return PA_OK;
+}
 
 extern "C" int pa_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_len) {
   // Long enough to amortise the merge, short enough that the grid covers the
@@ -1499,6 +1571,18 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int nu
   return body ? kCounterRegion + body : 0;
 }
 
+extern "C" int pa_decode_grid_ctas(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                   int block_size, int num_blocks, int max_context_len,
+                                   int partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+      block_size <= 0 || num_blocks <= 0 || (head_dim != 64 && head_dim != 128) ||
+      max_context_len < 0 || partition_tokens < 0 || partition_tokens % kPartitionQuantum)
+    return 0;
+  const int group = num_q_heads / num_kv_heads;
+  if (!uses_stream_kernel(group, block_size, num_blocks, num_kv_heads)) return 0;
+  return stream_grid(num_seqs, num_kv_heads, group, head_dim, max_context_len, partition_tokens);
+}
+
 extern "C" int pa_decode_launches(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                   int block_size, int num_blocks, int max_context_len,
                                   int partition_tokens) {
@@ -1512,6 +1596,30 @@ extern "C" int pa_decode_launches(int num_seqs, int num_q_heads, int num_kv_head
 }
 
 namespace {
+
+// Workspace one decode call needs (bytes, 0 for none), for the kernel that call
+// runs: the even-split kernel's counters and pieces (+ the window remap), or the
+// partition kernel's partial states when the longest context has more than one
+// partition. Arguments already validated.
+size_t decode_need(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                   int num_blocks, int max_context_len, int partition_tokens, int window) {
+  const int group = num_q_heads / num_kv_heads;
+  const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
+  const int max_parts = max_context_len > 0 ? (max_context_len + pt - 1) / pt : 1;
+  const bool wstream =
+      window > 0 && window_on_stream(group, block_size, num_blocks, num_kv_heads);
+  const bool streamk =
+      (window == 0 && uses_stream_kernel(group, block_size, num_blocks, num_kv_heads)) || wstream;
+  if (streamk) {
+    const int nctas = stream_grid(num_seqs, num_kv_heads, group, head_dim, max_context_len,
+                                  partition_tokens);
+    return kCounterRegion + (size_t)2 * nctas * group * (head_dim + 4) * sizeof(float) +
+           (wstream ? window_remap_bytes(num_seqs, max_context_len, block_size) : 0);
+  }
+  return max_parts > 1 ? kCounterRegion + (size_t)num_seqs * num_q_heads * max_parts *
+                                              (head_dim + 2) * sizeof(float)
+                       : 0;
+}
 
 // The new token of every sequence, written by the decode kernel itself.
 struct FusedWrite {
@@ -1560,14 +1668,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
                                           max_context_len, partition_tokens)
                             : 0;
   const size_t pieces_bytes = (size_t)2 * nctas * group * (head_dim + 4) * sizeof(float);
-  size_t need;
-  if (streamk)
-    need = kCounterRegion + pieces_bytes +
-           (wstream ? window_remap_bytes(num_seqs, max_context_len, block_size) : 0);
-  else
-    need = max_parts > 1 ? kCounterRegion + (size_t)num_seqs * num_q_heads * max_parts *
-                                                (head_dim + 2) * sizeof(float)
-                         : 0;
+  const size_t need = decode_need(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                  num_blocks, max_context_len, partition_tokens, window);
   if (need > workspace_bytes || (need && (!workspace || !aligned(workspace, 16))))
     return PA_ERR_INVALID;
   float *ws_body =
@@ -1595,6 +1697,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   prm.window = window;
   prm.win_skip = nullptr;
   prm.early_start = early_start ? 1 : 0;
+  prm.starve = g_wait_test.load();
+  prm.wait_ns = prm.starve ? (unsigned long long)g_wait_test_ns.load() : kWaitLimitNs;
   if (fw && !streamk) return PA_ERR_INVALID;  // only the even-split kernel writes
   prm.max_blocks_per_seq = max_blocks_per_seq;
   prm.max_context_len = max_context_len;
@@ -1786,6 +1890,18 @@ extern "C" pa_status pa_decode_append_window(
 bool pa_internal_pool_tensor_map(CUtensorMap *map, const void *base, long long rows, int head_dim,
                                  int box_rows, pa_dtype dtype) {
   return pool_tensor_map(map, base, rows, head_dim, box_rows, dtype);
+}
+
+size_t pa_internal_decode_need(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int num_blocks, int max_context_len,
+                               int partition_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
+      block_size <= 0 || num_blocks <= 0 || (head_dim != 64 && head_dim != 128) ||
+      max_context_len < 0 || partition_tokens < 0 || partition_tokens % kPartitionQuantum ||
+      partition_tokens > kMaxPartitionTokens)
+    return 0;
+  return decode_need(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                     max_context_len, partition_tokens, 0);
 }
 
 pa_status pa_internal_decode_status(cudaStream_t stream, int32_t *code) {

@@ -6,6 +6,14 @@
 // code the array's name only stands for the symbol -- it is not a device
 // address -- so the first call on each device looks the address up with
 // cudaGetSymbolAddress (with that device current) and passes the result on.
+// Only a successful lookup is kept; a failed one is retried by the next call.
+//
+// pa_decode requires the first bytes of its workspace (the even-split kernel's
+// per-CTA counters) to be zero when a call starts. A completed call leaves them
+// zero, but a call that gave up a wait (PA_DEVERR_TIMEOUT) may not, and the
+// caller of this entry point has no pointer to the array to clear them. So
+// every call first clears that region on its own stream (cudaMemsetAsync:
+// stream-ordered, no allocation) and then runs pa_decode.
 
 #include <cuda_runtime.h>
 
@@ -13,6 +21,7 @@
 #include <mutex>
 
 #include "pa.h"
+#include "pa_internal.h"
 
 namespace {
 
@@ -20,9 +29,24 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_static_workspace[PA_STATIC_WORKSPACE_BYTES];
 
-void *g_static_workspace_addr[kMaxDevices];
-cudaError_t g_static_workspace_err[kMaxDevices];
-std::once_flag g_static_workspace_once[kMaxDevices];
+std::mutex g_static_workspace_mu;
+void *g_static_workspace_addr[kMaxDevices];  // nullptr until a lookup succeeded
+
+static_assert(kPaCounterRegionBytes <= PA_STATIC_WORKSPACE_BYTES, "counters fit the array");
+
+// The array's device address on the current device, looked up once per device.
+void *static_workspace_address(int dev) {
+  std::lock_guard<std::mutex> lock(g_static_workspace_mu);
+  if (!g_static_workspace_addr[dev]) {
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_static_workspace) != cudaSuccess || !addr) {
+      cudaGetLastError();  // do not leave the failure for the next CUDA call to report
+      return nullptr;
+    }
+    g_static_workspace_addr[dev] = addr;
+  }
+  return g_static_workspace_addr[dev];
+}
 
 }  // namespace
 
@@ -32,20 +56,25 @@ extern "C" pa_status pa_decode_static_workspace(
     int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
     int block_size, int num_blocks, float scale, pa_dtype dtype, int partition_tokens,
     void *stream) {
-  const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                               max_context_len, partition_tokens);
+  // the scratch of the kernel this call runs (pa_decode itself rejects bad arguments)
+  const size_t need = pa_internal_decode_need(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                              block_size, num_blocks, max_context_len,
+                                              partition_tokens);
   if (need > PA_STATIC_WORKSPACE_BYTES) return PA_ERR_UNSUPPORTED;  // beyond the fixed array
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
-  // once per device, with that device current: the array's device address
-  std::call_once(g_static_workspace_once[dev], [dev] {
-    g_static_workspace_err[dev] =
-        cudaGetSymbolAddress(&g_static_workspace_addr[dev], g_static_workspace);
-  });
-  if (g_static_workspace_err[dev] != cudaSuccess || !g_static_workspace_addr[dev])
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
     return PA_ERR_CUDA;
+  }
+  void *ws = static_workspace_address(dev);
+  if (!ws) return PA_ERR_CUDA;
+  if (need > 0 && cudaMemsetAsync(ws, 0, kPaCounterRegionBytes,
+                                  static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return PA_ERR_CUDA;
+  }
   return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                    max_context_len, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                   num_blocks, scale, dtype, g_static_workspace_addr[dev],
-                   PA_STATIC_WORKSPACE_BYTES, partition_tokens, stream);
+                   num_blocks, scale, dtype, ws, PA_STATIC_WORKSPACE_BYTES, partition_tokens,
+                   stream);
 }
