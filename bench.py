@@ -14,13 +14,22 @@ head_dim 128, bf16, 16-token blocks, lengths uniform in [128, 2048], a
 steps rotate through them, so each step reads KV that is not in L2 (1.1 GB of
 KV across the four versus a 126 MB L2).
 
-Timing: each step's write and decode are replayed as CUDA graphs; CUDA events
-on the launching stream bracket the K timed steps (after W warm-up steps, with
-a barrier and a device synchronise on both sides) and the decode of every step.
-With N > 1 (torchrun, one process per GPU) every rank runs its own batches --
-the sequences shard across GPUs with no exchange -- and the slowest rank's
-time is used. ``e2e`` repeats the measurement with the step's inputs in pinned
-host memory, copied in and the output copied out inside every step.
+Timing: the W warm-up steps and then exactly the K timed steps are each one
+CUDA graph of consecutive steps (K above 512: rounds of 16 steps and one graph
+of the rest), the batches in rotation; CUDA events on the launching stream
+bracket the timed steps, with a barrier and a device synchronise on both
+sides. The decode kernel's own duration comes from at least 50 replays of a
+graph of decode launches. With N > 1 (torchrun, one process per GPU) every
+rank runs its own batches -- the sequences shard across GPUs with no exchange
+-- and the slowest rank's time is used. ``e2e`` repeats the K steps with each
+step's inputs in pinned host memory, copied in, and its output copied out,
+inside the timed region.
+
+On one GPU the line also carries, under ``workloads``, the other decode
+workloads (long-context skew, the mixed batch at every block size, the
+shared-prompt batch with its unique and logical bytes, a sliding window) and
+chunked prefill, each timed the same way over a short run (``--no-extras``
+skips them).
 
 ``--impl reference`` times the fp64 CPU oracle on the same workload instead
 (a bounded sample of sequences per step), on the host's cores.
@@ -31,8 +40,8 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
-import re
 import subprocess
 import sys
 import threading
@@ -46,15 +55,17 @@ if ROOT not in sys.path:
 
 import synth  # noqa: E402
 from paged_kv_cache_370_b200.accounting import (decode_step_bytes, new_token_bytes,  # noqa: E402
-                                                split_scratch_bytes, tail_overread_bytes)
+                                                split_scratch_bytes, stream_split_scratch_bytes,
+                                                tail_overread_bytes, unique_kv_bytes)
 
 METRIC = "paged decode attention: KV GB/s and % of B200 HBM peak; query tokens/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_370_b200", "csrc", "pa_decode.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pa_decode_llama8b_traffic.md")
-PREFILL_SRC = os.path.join(ROOT, "paged_kv_cache_370_b200", "csrc", "pa_prefill.cu")
-PREFILL_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "pa_prefill_llama8b_traffic.md")
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
+MAX_GRAPH_STEPS = 512
+# DRAM-traffic records written by bench_traffic.py from ncu captures
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "pa_decode_llama8b_traffic.json")
+PREFILL_TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "pa_prefill_llama8b_traffic.json")
 
 
 # ------------------------------------------------------------------------------------- setup
@@ -82,6 +93,10 @@ def parse_args():
                     help="each captured round holds this many steps of every rotated batch "
                          "(device-resident and host-fed timing alike)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="only the headline workload (no per-workload sub-objects)")
+    ap.add_argument("--extra-steps", type=int, default=20,
+                    help="timed steps of each extra workload")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -95,6 +110,7 @@ def dist_env():
 
 
 def measured_peaks():
+    """(HBM GB/s, kind) from MEASURED_PEAKS.json, else the fallback figure."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
@@ -102,6 +118,16 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_sustained():
+    """(sustained dense bf16 TFLOP/s, kind) from MEASURED_PEAKS.json, else the fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return (float(json.load(f)["bf16_tflops_sustained"]),
+                    "measured sustained bf16 (cuBLAS, seconds-long loop)")
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback (sustained bf16 under the power cap)"
 
 
 def read_stream_gbs(torch, device):
@@ -124,19 +150,21 @@ def read_stream_gbs(torch, device):
             "how": "torch.sum over 4 GiB of bf16, best of 5 after 2 warm-up runs"}
 
 
-def recorded_traffic(summary=TRAFFIC_FILE, source=DECODE_SRC):
-    """Per-launch DRAM bytes from a committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+def recorded_traffic(algorithmic_now: float, record=TRAFFIC_RECORD):
+    """DRAM bytes per launch of the kernel, from the ncu record written by
+    bench_traffic.py, scaled from the captured case to this launch by algorithmic
+    bytes (or FLOPs); None when there is no record or the kernel's source changed
+    since the capture."""
     try:
-        text = open(summary).read()
-    except OSError:
+        with open(record) as f:
+            rec = json.load(f)
+        src = os.path.join(ROOT, rec["source"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["source_sha256"]:
+            return None
+        return int(round(rec["traffic_bytes_per_launch"] * algorithmic_now /
+                         rec["algorithmic_per_launch"]))
+    except (OSError, KeyError, ValueError, ZeroDivisionError):
         return None
-    src = hashlib.sha256(open(source, "rb").read()).hexdigest()
-    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
-    m_bytes = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_sha or not m_bytes or m_sha.group(1) != src:
-        return None
-    return int(m_bytes.group(1))
 
 
 # ---------------------------------------------------------------------------------- clocks
@@ -184,16 +212,23 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
-    def summary(self, t0: float, t1: float) -> dict:
+    def summary(self, t0: float, t1: float, t_end: float | None = None) -> dict:
+        """Clocks over the timed region [t0, t1]; when it is too short for a sample
+        (50 ms apart), over it and the kernel-timing loop that follows, up to t_end."""
         inside = [s for s in self.samples if t0 <= s[0] <= t1]
-        used = inside or [s for s in self.samples if t0 - 1.0 <= s[0] <= t1 + 1.0]
+        end = max(t1, t_end or t1)
+        used = inside or [s for s in self.samples if t0 - 0.1 <= s[0] <= end + 0.1]
         if not used:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "samples_in_timed_region": 0}
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for s in used for i, v in enumerate(s[3]) if v == "Active"})
         return {"sm_mhz": float(np.median([s[1] for s in used])),
                 "sm_max_mhz": float(max(s[2] for s in used)), "reasons": reasons,
-                "samples": len(used), "samples_in_timed_region": len(inside)}
+                "samples": len(used), "samples_in_timed_region": len(inside),
+                "window": ("the timed region" if inside else
+                           f"the timed region ({1e3 * (t1 - t0):.1f} ms) and the kernel-timing "
+                           f"loop after it ({1e3 * (end - t1):.0f} ms), sampled every 50 ms")}
 
 
 # ------------------------------------------------------------------------------- workloads
@@ -229,9 +264,12 @@ def _workload_config(args, batches, pt):
                 "batches_rotated": len(batches),
                 "l2": f"inputs larger than L2: {len(batches)} rotating batches, "
                       f"{sum(decode_step_bytes(x.context_lens, 32, 8, 128, 16)['kv'] for x in batches) / 1e9:.2f} GB of KV",
-                "timing": f"CUDA graphs of {len(batches) * max(1, args.round_reps)} steps "
-                          "(the batches in rotation) replayed back to back; CUDA events "
-                          "on the stream",
+                "timing": (f"one CUDA graph of the {args.steps} timed steps (the batches in "
+                           "rotation), after a graph of the warm-up steps; CUDA events on the "
+                           "stream" if args.steps <= MAX_GRAPH_STEPS else
+                           f"CUDA graphs of {len(batches) * max(1, args.round_reps)} steps "
+                           "(the batches in rotation) replayed back to back, then one graph "
+                           "of the rest; CUDA events on the stream"),
                 "launch": ("plain stream order" if args.no_overlap or args.no_fuse else
                            "programmatic early start: each decode kernel's start-up overlaps "
                            "the previous kernel's tail (pa_decode_append_overlapped)")}
@@ -287,19 +325,31 @@ def device_steps(args, batches, torch, device):
         del k_all, v_all
         steps.append(step)
         infos.append(_byte_info(b.context_lens, b.num_q_heads, b.num_kv_heads, b.head_dim,
-                                b.block_size, step.partition, b.num_seqs, args.window))
+                                b.block_size, step.partition, b.num_seqs, args.window,
+                                _grid_ctas(step)))
     torch.cuda.synchronize()
     return steps, infos
 
 
-def _byte_info(lens, hq, hkv, d, bs, pt, ntok, window=0):
+def _byte_info(lens, hq, hkv, d, bs, pt, ntok, window=0, nctas=0):
+    """Algorithmic bytes of one step and the bytes moved beyond them. ``nctas``: CTAs
+    of the even-split kernel (0: the partition kernel runs), whose split-segment
+    pieces are its scratch."""
+    lens = np.asarray(lens, dtype=np.int64)
+    seen = lens
     if window > 0:
-        # the positions a window reads: the last `window` of each sequence
-        lens = np.minimum(np.asarray(lens), window)
-    return {"decode": decode_step_bytes(lens, hq, hkv, d, bs),
-            "scratch": split_scratch_bytes(lens, hq, d, pt),
-            "tail": tail_overread_bytes(lens, hkv, d, bs),
-            "write": new_token_bytes(ntok, hkv, d), "lens": np.asarray(lens)}
+        # the positions a window reads: the last `window` of each sequence; the
+        # even-split kernel sees each from the block of its first attended position
+        seen = np.minimum(lens, window)
+        lo = np.maximum(lens - window, 0)
+        kernel_lens = lens - (lo // bs) * bs
+    else:
+        kernel_lens = lens
+    scratch = (stream_split_scratch_bytes(kernel_lens, hkv, hq // hkv, d, nctas) if nctas
+               else split_scratch_bytes(seen, hq, d, pt))
+    return {"decode": decode_step_bytes(seen, hq, hkv, d, bs), "scratch": scratch,
+            "tail": tail_overread_bytes(seen, hkv, d, bs),
+            "write": new_token_bytes(ntok, hkv, d), "lens": seen}
 
 
 def shared_prompt_steps(args, torch, device):
@@ -351,8 +401,10 @@ def shared_prompt_steps(args, torch, device):
                       copy_pairs=torch.tensor(pairs, dtype=torch.int64, device=device),
                       fused=not args.no_fuse)
     torch.cuda.synchronize()
-    info = _byte_info(lens, 40, 40, 128, 16, step.partition, len(ids))
+    info = _byte_info(lens, 40, 40, 128, 16, step.partition, len(ids), 0, _grid_ctas(step))
     info["copy"] = 2 * 2 * len(pairs) * 40 * 16 * 128 * 2
+    # each physical block once, however many branches read it (the forked prompt)
+    info["unique_kv"] = unique_kv_bytes(tables, lens, 16, 40, 128)
     return [step], [info]
 
 
@@ -382,6 +434,66 @@ def capture(fn, torch):
     return g
 
 
+def _grid_ctas(step):
+    from paged_kv_cache_370_b200 import abi
+    B, hq, d = step.q.shape
+    nb, hkv, bs, _ = step.k_cache.shape
+    return abi.pa_decode_grid_ctas(B, hq, hkv, d, bs, nb, step.max_context_len,
+                                   step.partition_tokens)
+
+
+def _launches(step, fused):
+    return step.append_launches if fused else step.decode_launches
+
+
+def upload_graphs(plan, stream):
+    """Upload each graph's executable to the device ahead of its first replay
+    (cudaGraphUpload: no work runs), so that the timed region does not pay for
+    the upload a first launch would otherwise do."""
+    try:
+        from cuda.bindings import runtime as rt
+    except ImportError:  # older cuda-python layout
+        from cuda import cudart as rt
+    st = rt.cudaStream_t(init_value=int(stream.cuda_stream))
+    for g, _ in plan:
+        handle = g.raw_cuda_graph_exec()
+        err = rt.cudaGraphUpload(rt.cudaGraphExec_t(init_value=int(handle)), st)[0]
+        if int(err) != 0:
+            raise RuntimeError(f"cudaGraphUpload failed: {err}")
+
+
+def time_graphs(plan, stream, torch):
+    """Device milliseconds of replaying [(graph, times), ...] once, CUDA events on ``stream``."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for g, n in plan:
+        for _ in range(n):
+            g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def step_plan(n, start, fn, steps, R, torch):
+    """Graphs that run exactly n consecutive steps (batch (start + i) % V for step
+    i): one graph of n steps, or above MAX_GRAPH_STEPS rounds of R and one graph of
+    the rest (R a multiple of V, so the rotation carries on across rounds)."""
+    V = len(steps)
+
+    def graph(m):
+        return capture(lambda: [fn(steps[(start + i) % V]) for i in range(m)], torch)
+
+    if n <= 0:
+        return []
+    if n <= MAX_GRAPH_STEPS:
+        return [(graph(n), 1)]
+    rounds, rest = divmod(n, R)
+    plan = [(graph(R), rounds)]
+    if rest:
+        plan.append((graph(rest), 1))
+    return plan
+
+
 def run_ours(args, rank, world, local, dist):
     import torch
     device = torch.device("cuda", local)
@@ -389,9 +501,8 @@ def run_ours(args, rank, world, local, dist):
     batches = make_batches(args, rank)
     steps, infos = device_steps(args, batches, torch, device)
     pt = steps[0].partition
-    # graphs per batch: [copy-on-write copies (+ the KV write unless fused)] and
-    # [decode (with the fused KV write)]
     fused = steps[0].fused
+    V = len(steps)
 
     def pre(s):
         s.copy()
@@ -401,21 +512,20 @@ def run_ours(args, rank, world, local, dist):
     def has_pre(s):
         return (not s.fused) or (s.copy_pairs is not None and s.copy_pairs.numel() > 0)
 
-    g_write = [capture(lambda s=s: pre(s), torch) if has_pre(s) else None for s in steps]
-    g_dec = [capture(lambda s=s: s.append() if s.fused else s.attend(), torch) for s in steps]
-    V = len(steps)
-
     def one_step(s):
         pre(s) if has_pre(s) else None
         s.append() if s.fused else s.attend()
 
-    # one graph per round: round_reps steps of every batch in rotation, back to
-    # back (a serving loop launches whole decode steps as graphs); and the decode
-    # launches alone
+    def decode_only(s):
+        s.append() if s.fused else s.attend()
+
+    K, Wm = args.steps, args.warmup
     R = V * max(1, args.round_reps)
-    g_round = capture(lambda: [one_step(steps[i % V]) for i in range(R)], torch)
-    g_dec_only = capture(lambda: [s.append() if s.fused else s.attend()
-                                  for s in (steps[i % V] for i in range(R))], torch)
+    off = Wm % V  # the timed steps carry the batch rotation on from the warm-up
+    warm = step_plan(Wm, 0, one_step, steps, R, torch)
+    timed = step_plan(K, off, one_step, steps, R, torch)
+    g_dec = capture(lambda: [decode_only(steps[i % V]) for i in range(R)], torch)
+    g_pre = [capture(lambda s=s: pre(s), torch) if has_pre(s) else None for s in steps]
 
     def barrier():
         if dist is not None:
@@ -423,14 +533,6 @@ def run_ours(args, rank, world, local, dist):
         torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
-    for i in range(max(1, args.warmup // R)):
-        g_round.replay()
-    for i in range(args.warmup % R):
-        if g_write[i % V] is not None:
-            g_write[i % V].replay()
-        g_dec[i % V].replay()
-    K = args.steps
-    rounds, rest = divmod(K, R)
     props = torch.cuda.get_device_properties(device)
     bus = getattr(props, "pci_bus_id", None)
     bus_str = None
@@ -440,69 +542,53 @@ def run_ours(args, rank, world, local, dist):
     sampler = ClockSampler(bus_str)
     sampler.start()
     time.sleep(0.3)
+    # ---- warm-up: exactly W steps, untimed; the timed graphs uploaded to the device
+    time_graphs(warm, stream, torch)
+    upload_graphs(timed, stream)
     # ---- the timed region: exactly K steps
     start_ev, end_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     t0 = time.time()
     start_ev.record(stream)
-    for r in range(rounds):
-        g_round.replay()
-    for i in range(rest):
-        if g_write[i % V] is not None:
-            g_write[i % V].replay()
-        g_dec[i % V].replay()
+    for g, n in timed:
+        for _ in range(n):
+            g.replay()
     end_ev.record(stream)
     barrier()
     t1 = time.time()
+    total_ms = start_ev.elapsed_time(end_ev)
+    # ---- the decode kernel's own duration: >= 50 replays of a graph of R decode
+    # launches (about half a second), CUDA events on the same stream
+    est = max(total_ms / max(K, 1), 1e-3)
+    reps = max(50, int(math.ceil(500.0 / (est * R))))
+    tk0 = time.time()
+    dec_ms = time_graphs([(g_dec, reps)], stream, torch) / (reps * R)
+    tk1 = time.time()
+    pre_ms = 0.0
+    if any(g is not None for g in g_pre):
+        pre_ms = time_graphs([(g, 50) for g in g_pre if g is not None], stream, torch) / (50 * V)
+    # ---- the spread: the timed steps replayed again, an event after each replay
+    rep_ms = [time_graphs(timed, stream, torch) / K for _ in range(5)]
     time.sleep(0.2)
     sampler.stop()
-    total_ms = start_ev.elapsed_time(end_ev)
-    # ---- the spread over rounds: the same rounds again, an event after each
-    round_ms = []
-    if rounds:
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(rounds + 1)]
-        evs[0].record(stream)
-        for r in range(rounds):
-            g_round.replay()
-            evs[r + 1].record(stream)
-        torch.cuda.synchronize()
-        round_ms = [evs[r].elapsed_time(evs[r + 1]) / R for r in range(rounds)]
     read_stream = read_stream_gbs(torch, device)
-    # ---- per-kernel durations (same launches, separately timed with events)
-    reps = max(1, min(50, K // R))
-    ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ka.record(stream)
-    for _ in range(reps):
-        g_dec_only.replay()
-    kb.record(stream)
-    torch.cuda.synchronize()
-    dec_ms = [ka.elapsed_time(kb) / (reps * R)]
-    pa, pb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    wr_ms = [0.0]
-    if any(g is not None for g in g_write):
-        pa.record(stream)
-        for _ in range(reps):
-            for g in g_write:
-                if g is not None:
-                    g.replay()
-        pb.record(stream)
-        torch.cuda.synchronize()
-        wr_ms = [pa.elapsed_time(pb) / (reps * V)]
-    step_bytes = [infos[i % V]["decode"]["total"] for i in range(K)]
+    step_bytes = [infos[(off + i) % V]["decode"]["total"] for i in range(K)]
     total_ms_max, all_bytes = rank_aggregate(total_ms, float(sum(step_bytes)), dist, device)
     ms_per_step = total_ms_max / K
     gbs = all_bytes / (total_ms_max * 1e-3) / 1e9
-    q_tok = sum(len(infos[i % V]["lens"]) for i in range(K)) * world / (total_ms_max * 1e-3)
+    q_tok = sum(len(infos[(off + i) % V]["lens"]) for i in range(K)) * world / \
+        (total_ms_max * 1e-3)
 
     peak, peak_kind = measured_peaks()
-    dec_avg_ms = float(np.mean(dec_ms))
     # the fused kernel also reads each new token's K/V and stores it at its slot
     dec_bytes = float(np.mean([infos[i % V]["decode"]["total"] +
-                               (infos[i % V]["write"] if fused else 0) for i in range(K)]))
-    achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
+                               (infos[i % V]["write"] if fused else 0) for i in range(R)]))
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     # recorded for the plain (no window) kernel on this workload only
-    traffic = recorded_traffic() if args.workload == "llama8b" and args.window == 0 else None
-    launches = sum(s.launches() for s in (steps[i % V] for i in range(K)))
+    traffic = (recorded_traffic(dec_bytes) if args.workload == "llama8b" and args.window == 0
+               else None)
+    launches = sum(steps[(off + i) % V].launches() for i in range(K))
+    nctas = _grid_ctas(steps[0])
 
     e2e = None
     if not args.no_e2e:
@@ -510,10 +596,10 @@ def run_ours(args, rank, world, local, dist):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and batches is not None:
         cpu = cpu_baseline(batches[0], args.cpu_seconds)
-    clocks = sampler.summary(t0, t1)
+    clocks = sampler.summary(t0, t1, tk1)
     res = {
         "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "steps": K, "warmup": Wm, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype":
             "bf16" if (batches and batches[0].dtype == "bf16") else "f16",
         "data": "synthetic (seeded N(0,1) K/V/q, random block tables)",
@@ -521,12 +607,12 @@ def run_ours(args, rank, world, local, dist):
         "query_tokens_per_s": round(q_tok, 1),
         "pct_of_hbm_measured": round(100 * gbs / world / peak, 2),
         "pct_of_hbm_nominal_8tbs": round(100 * gbs / world / NOMINAL_HBM_GBS, 2),
-        "ms_per_step_over_rounds": ({"median": round(float(np.median(round_ms)), 5),
-                                     "min": round(float(np.min(round_ms)), 5),
-                                     "max": round(float(np.max(round_ms)), 5),
-                                     "rounds": len(round_ms), "steps_per_round": R,
-                                     "how": "the timed rounds replayed again with an event "
-                                            "after each"} if round_ms else None),
+        "ms_per_step_over_replays": {"median": round(float(np.median(rep_ms)), 5),
+                                     "min": round(float(np.min(rep_ms)), 5),
+                                     "max": round(float(np.max(rep_ms)), 5),
+                                     "replays": len(rep_ms),
+                                     "how": "the K timed steps replayed again 5 times, "
+                                            "CUDA events around each replay"},
         "hbm_read_stream": read_stream,
         "roofline": {"bound": "hbm",
                      "kernel": ("pa_decode_append (KV write + decode, one kernel)" if fused
@@ -534,16 +620,19 @@ def run_ours(args, rank, world, local, dist):
                      "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                      "traffic": traffic, "algorithmic_bytes_per_launch": int(dec_bytes),
-                     "avg_launch_ms": round(dec_avg_ms, 5),
+                     "avg_launch_ms": round(dec_ms, 5),
+                     "how": f"{reps} replays of a graph of {R} decode launches (the batches "
+                            "in rotation), CUDA events on the launching stream",
                      "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4)},
-        "kernel_ms": {"before_decode": round(float(np.mean(wr_ms)), 5),
-                      "decode": round(dec_avg_ms, 5)},
-        "extra_bytes_per_step": {"split_scratch": int(np.mean([infos[i % V]["scratch"]
-                                                               for i in range(K)])),
-                                 "kv_write": int(infos[0]["write"]),
-                                 "copy_on_write": int(infos[0].get("copy", 0)),
-                                 "tail_overread": int(np.mean([infos[i % V]["tail"]
-                                                               for i in range(K)]))},
+        "kernel_ms": {"before_decode": round(pre_ms, 5), "decode": round(dec_ms, 5)},
+        "extra_bytes_per_step": {
+            "split_scratch": int(np.mean([infos[i % V]["scratch"] for i in range(V)])),
+            "split_scratch_kernel": ("even-split: pieces of split segments, "
+                                     f"{nctas} CTAs" if nctas else
+                                     "partition kernel: partial states of split sequences"),
+            "kv_write": int(infos[0]["write"]),
+            "copy_on_write": int(infos[0].get("copy", 0)),
+            "tail_overread": int(np.mean([infos[i % V]["tail"] for i in range(V)]))},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
@@ -551,16 +640,23 @@ def run_ours(args, rank, world, local, dist):
         res["e2e"] = e2e
     if cpu is not None:
         res["cpu_baseline"] = cpu
+    del steps, g_dec, g_pre, timed, warm
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     return res
 
 
 def run_e2e(args, steps, infos, torch, device, dist, world):
-    """The same steps fed from pinned host buffers through the library's
-    HostStepPipeline: two rounds of R host-fed steps taking turns, each round's
-    uploads, kernels and downloads replayed as graphs on three streams."""
+    """The same K steps fed from pinned host buffers through the library's
+    HostStepPipeline: each round's uploads, kernels and downloads are graphs on
+    three streams, the next round's uploads and the previous round's downloads
+    running under a round's kernels. Up to 64 steps: rounds that grow from one
+    step and shrink back to one (only the first upload and the last download are
+    exposed); beyond: two sets of 16 steps taking turns, then the rest."""
     from paged_kv_cache_370_b200.step import HostDecodeStep, HostStepPipeline
     V = len(steps)
-    R = V * max(1, args.round_reps)
+    K = args.steps
+    off = args.warmup % V
 
     def host_step(s):
         return HostDecodeStep(k_cache=s.k_cache, v_cache=s.v_cache, q=s.q, k_new=s.k_new,
@@ -570,39 +666,49 @@ def run_e2e(args, steps, infos, torch, device, dist, world):
                               partition_tokens=s.partition_tokens, copy_pairs=s.copy_pairs,
                               fused=s.fused, window=s.window, overlapped=s.overlapped)
 
-    rounds = [[host_step(steps[i % V]) for i in range(R)] for _ in range(2)]
+    if K <= 64:
+        sizes = HostStepPipeline.ramp_sizes(K)
+        rounds, i = [], 0
+        for n in sizes:
+            rounds.append([host_step(steps[(off + i + j) % V]) for j in range(n)])
+            i += n
+        order = list(range(len(rounds)))
+        shape = f"rounds of {sizes} steps"
+    else:
+        R = V * max(1, args.round_reps)
+        n_rounds, rest = divmod(K, R)
+        rounds = [[host_step(steps[(off + j) % V]) for j in range(R)] for _ in range(2)]
+        order = [r % 2 for r in range(n_rounds)]
+        if rest:
+            rounds.append([host_step(steps[(off + j) % V]) for j in range(rest)])
+            order.append(2)
+        shape = f"two sets of {R} steps taking turns, then {rest}"
     pipe = HostStepPipeline(rounds)
     pipe.capture()
-    # a step count that is not a whole number of rounds ends with serial host steps
-    tail = [capture(h.run, torch) for h in rounds[0][:V]]
-    pipe.run(max(2, args.warmup // R))
+    for _ in range(max(1, -(-max(args.warmup, 3) // K))):  # >= W (and >= 3) warm-up steps
+        pipe.run_order(order)
     torch.cuda.synchronize()
-    K = args.steps
-    n_rounds, rest = divmod(K, R)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    pipe.run(n_rounds)
-    for i in range(rest):
-        tail[i % V].replay()
+    pipe.run_order(order)
     b.record()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    my_bytes = sum(infos[i % V]["decode"]["total"] for i in range(K))
+    my_bytes = sum(infos[(off + i) % V]["decode"]["total"] for i in range(K))
     ms, total = rank_aggregate(a.elapsed_time(b), float(my_bytes), dist, device)
-    h0 = rounds[0]
+    h_all = [h for x in order for h in rounds[x]]
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms / K, 5),
-            "h2d_bytes_per_step": int(np.mean([h0[i % V].h2d_bytes for i in range(K)])),
-            "d2h_bytes_per_step": int(h0[0].d2h_bytes),
+            "h2d_bytes_per_step": int(np.mean([h.h2d_bytes for h in h_all])),
+            "d2h_bytes_per_step": int(np.mean([h.d2h_bytes for h in h_all])),
             "how": "pinned host inputs copied in and output copied out every step through the "
-                   f"library's HostStepPipeline: rounds of {R} steps, each round's uploads, "
-                   "kernels and downloads replayed as CUDA graphs on three streams, the next "
-                   "round's uploads and the previous round's downloads under this round's "
-                   "kernels"}
+                   f"library's HostStepPipeline ({shape}); each round's uploads, kernels and "
+                   "downloads replayed as CUDA graphs on three streams, the next round's "
+                   "uploads and the previous round's downloads under a round's kernels"}
 
 
 # --------------------------------------------------------------------------- CPU (oracle)
@@ -759,15 +865,17 @@ def prefill_flops(batch, window=0) -> float:
     return 4.0 * batch.head_dim * batch.num_q_heads * keys
 
 
-def run_prefill(args):
+def prefill_measure(pool_blocks, window, n_timed, n_warm):
     """Chunked prefill on the Llama-3.1-8B shapes (16 sequences x 512 new tokens
     after up to 1,536 history tokens): one step = the chunk's K/V write
-    (pa_reshape_and_cache) + pa_prefill, graph-replayed over 4 rotating batches."""
+    (pa_reshape_and_cache) + pa_prefill, over 4 rotating batches. n_warm steps,
+    then exactly n_timed steps, each a graph of consecutive steps; the prefill
+    kernel's own duration from >= 50 replays of a graph of its launches."""
     import torch
     from paged_kv_cache_370_b200 import abi
-    dev = torch.device("cuda", 0)
+    dev = torch.device("cuda", torch.cuda.current_device())
     # 4 batches, each drawing distinct ids from its own quarter of the pool
-    nv, per = 4, max(2048, args.pool_blocks // 4)
+    nv, per = 4, max(2048, pool_blocks // 4)
     batches = [synth.llama8b_prefill(seed=synth.SEED_BASE + 7 + 10 * v, num_blocks=per)
                for v in range(nv)]
     b0 = batches[0]
@@ -794,7 +902,7 @@ def run_prefill(args):
               "lens": torch.from_numpy(b.context_lens).to(dev),
               "q_start": torch.from_numpy(qs.astype(np.int32)).to(dev),
               "max_q": int(b.meta["q_lens"].max()), "max_len": b.max_context_len,
-              "scale": float(b.scale), "flops": prefill_flops(b, args.window)}
+              "scale": float(b.scale), "flops": prefill_flops(b, window)}
         st["out"] = torch.empty_like(st["q"])
         steps.append(st)
         del k_all, v_all
@@ -804,62 +912,186 @@ def run_prefill(args):
 
     def attend(st):
         abi.pa_prefill(st["out"], st["q"], kc, vc, st["tables"], st["lens"], st["q_start"],
-                       st["max_q"], st["max_len"], st["scale"], args.window)
+                       st["max_q"], st["max_len"], st["scale"], window)
 
-    g_round = capture(lambda: [f(st) for st in steps for f in (write, attend)], torch)
+    def one_step(st):
+        write(st)
+        attend(st)
+
+    V = len(steps)
+    stream = torch.cuda.current_stream()
+    warm = step_plan(n_warm, 0, one_step, steps, 4 * V, torch)
+    timed = step_plan(n_timed, n_warm % V, one_step, steps, 4 * V, torch)
     g_att = capture(lambda: [attend(st) for st in steps], torch)
-    for _ in range(max(3, args.warmup // 10)):
-        g_round.replay()
-    torch.cuda.synchronize()
-    rounds = max(1, args.steps // len(steps))
     clocks = ClockSampler(os.environ.get("PA_BUS_ID"))
     clocks.start()
     time.sleep(0.3)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    time_graphs(warm, stream, torch)
+    upload_graphs(timed, stream)
+    torch.cuda.synchronize()
     t0 = time.time()
-    e0.record()
-    for _ in range(rounds):
-        g_round.replay()
-    e1.record()
-    torch.cuda.synchronize()
+    step_ms = time_graphs(timed, stream, torch) / n_timed
     t1 = time.time()
-    step_ms = e0.elapsed_time(e1) / (rounds * len(steps))
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record()
-    for _ in range(rounds):
-        g_att.replay()
-    a1.record()
-    torch.cuda.synchronize()
+    reps = 50
+    att_ms = time_graphs([(g_att, reps)], stream, torch) / (reps * V)
+    t2 = time.time()
     clocks.stop()
-    att_ms = a0.elapsed_time(a1) / (rounds * len(steps))
     flops = float(np.mean([st["flops"] for st in steps]))
-    peak = 1394.0
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak = float(json.load(f)["bf16_tflops_sustained"])
-        kind = "measured sustained bf16 (cuBLAS, seconds-long loop)"
-    except (OSError, KeyError, ValueError):
-        kind = "fallback"
+    step_flops = float(np.mean([steps[(n_warm + i) % V]["flops"] for i in range(n_timed)]))
+    peak, kind = measured_bf16_sustained()
     tflops = flops / (att_ms * 1e-3) / 1e12
     tokens = float(np.mean([int(st["q"].shape[0]) for st in steps]))
     code = abi.pa_device_status()
-    return {"metric": "paged prefill attention TFLOP/s (causal, bf16 in, fp32 accumulate)",
-            "value": round(flops / (step_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "n_gpus": 1,
-            "steps": rounds * len(steps), "warmup": args.warmup, "ms_per_step": round(step_ms, 5),
-            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+    del steps, kc, vc, g_att, warm, timed
+    torch.cuda.empty_cache()
+    return {"value": round(step_flops / (step_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(step_ms, 5), "steps": n_timed, "warmup": n_warm,
+            "query_tokens_per_s": round(tokens / (step_ms * 1e-3), 1),
             "config": {"workload": "Llama-3.1-8B-shaped chunked prefill", "num_seqs": 16,
                        "chunk_tokens": 512, "history": "uniform [0, 1536]",
-                       "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128, "block_size": 16,
-                       "window": args.window, "batches_rotated": len(steps)},
-            "query_tokens_per_s": round(tokens / (step_ms * 1e-3), 1),
+                       "num_q_heads": 32, "num_kv_heads": 8, "head_dim": 128,
+                       "block_size": 16, "window": window, "batches_rotated": V,
+                       "step": "the chunk's KV write + pa_prefill"},
             "roofline": {"bound": "tensor", "kernel": "pa_prefill", "achieved": round(tflops, 2),
                          "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
                          "peak_kind": kind, "flops_per_launch": flops,
                          "avg_launch_ms": round(att_ms, 5),
-                         "traffic": (recorded_traffic(PREFILL_TRAFFIC_FILE, PREFILL_SRC)
-                                     if args.window == 0 else None)},
-            "gpu_launches": 2 * rounds * len(steps), "clocks": clocks.summary(t0, t1),
+                         "how": f"{reps} replays of a graph of {V} prefill launches",
+                         "traffic": (recorded_traffic(flops, PREFILL_TRAFFIC_RECORD)
+                                     if window == 0 else None)},
+            "gpu_launches": 2 * n_timed, "clocks": clocks.summary(t0, t1, t2),
             "device_error_word": code}
+
+
+def run_prefill(args):
+    r = prefill_measure(args.pool_blocks, args.window, args.steps, max(3, args.warmup))
+    r.update({"metric": "paged prefill attention TFLOP/s (causal, bf16 in, fp32 accumulate)",
+              "n_gpus": 1, "higher_is_better": True, "dtype": "bf16", "data": "synthetic"})
+    return r
+
+
+# ---------------------------------------------------------------------- the other workloads
+def _decode_measure(args, batches, torch, device, n_timed, n_warm, extra=None):
+    """One decode workload on its own: the step graphs and CUDA events as for the
+    headline, over n_timed steps after n_warm."""
+    steps, infos = device_steps(args, batches, torch, device)
+    fused = steps[0].fused
+    V = len(steps)
+
+    def one_step(s):
+        s.copy()
+        if not s.fused:
+            s.write()
+        s.append() if s.fused else s.attend()
+
+    stream = torch.cuda.current_stream()
+    warm = step_plan(n_warm, 0, one_step, steps, 4 * V, torch)
+    timed = step_plan(n_timed, n_warm % V, one_step, steps, 4 * V, torch)
+    g_dec = capture(lambda: [(s.append() if s.fused else s.attend()) for s in steps], torch)
+    time_graphs(warm, stream, torch)
+    upload_graphs(timed, stream)
+    torch.cuda.synchronize()
+    ms = time_graphs(timed, stream, torch) / n_timed
+    reps = 50
+    dec_ms = time_graphs([(g_dec, reps)], stream, torch) / (reps * V)
+    peak, kind = measured_peaks()
+    nbytes = float(np.mean([infos[(n_warm + i) % V]["decode"]["total"] for i in range(n_timed)]))
+    kbytes = float(np.mean([i["decode"]["total"] + (i["write"] if fused else 0) for i in infos]))
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    kgbs = kbytes / (dec_ms * 1e-3) / 1e9
+    from paged_kv_cache_370_b200 import abi
+    res = {"value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(ms, 5),
+           "steps": n_timed, "warmup": n_warm,
+           "pct_of_hbm_measured": round(100 * gbs / peak, 2),
+           "pct_of_hbm_nominal_8tbs": round(100 * gbs / NOMINAL_HBM_GBS, 2),
+           "bytes_per_step": int(nbytes),
+           "query_tokens_per_s": round(float(np.mean([len(i["lens"]) for i in infos])) /
+                                       (ms * 1e-3), 1),
+           "kernel": {"avg_launch_ms": round(dec_ms, 5), "achieved_gbs": round(kgbs, 2),
+                      "frac": round(kgbs / peak, 4), "peak": peak, "peak_kind": kind,
+                      "algorithmic_bytes_per_launch": int(kbytes)},
+           "extra_bytes_per_step": {"split_scratch": int(np.mean([i["scratch"] for i in infos])),
+                                    "tail_overread": int(np.mean([i["tail"] for i in infos])),
+                                    "kv_write": int(infos[0]["write"]),
+                                    "copy_on_write": int(infos[0].get("copy", 0))},
+           "gpu_launches": int(sum(steps[(n_warm + i) % V].launches() for i in range(n_timed))),
+           "device_error_word": abi.pa_device_status()}
+    if "unique_kv" in infos[0]:
+        u = infos[0]["unique_kv"] + (infos[0]["decode"]["total"] - infos[0]["decode"]["kv"])
+        res["unique_bytes_per_step"] = int(u)
+        res["logical_bytes_per_step"] = int(nbytes)
+        res["unique_gbs"] = round(u / (ms * 1e-3) / 1e9, 2)
+        res["pct_of_hbm_measured_unique"] = round(100 * u / (ms * 1e-3) / 1e9 / peak, 2)
+        res["note"] = ("logical bytes count every branch's read of the shared prompt blocks; "
+                       "unique bytes count each physical block once (the prompt blocks are "
+                       "read by four branches and hit in L2 after the first)")
+    if extra:
+        res.update(extra)
+    del steps, g_dec, warm, timed
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_extras(args, torch, device):
+    """The other workloads of the line, each measured on its own over a short run."""
+    n, w = max(1, args.extra_steps), 5
+    base = argparse.Namespace(**vars(args))
+    base.window, base.partition_tokens = 0, 0
+    out = {}
+
+    def ns(**kw):
+        a = argparse.Namespace(**vars(base))
+        for k, v in kw.items():
+            setattr(a, k, v)
+        return a
+
+    def guarded(name, fn):
+        try:
+            out[name] = fn()
+        except Exception as e:  # noqa: BLE001 -- reported in the line, the headline stands
+            out[name] = {"error": f"{type(e).__name__}: {e}"}
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+    guarded("long_skew", lambda: _decode_measure(
+        ns(workload="long_skew"), [synth.long_skew()], torch, device, n, w,
+        {"config": {"workload": "long-context skew decode", "num_seqs": 8,
+                    "context_lens": "uniform [8192, 32768]", "num_q_heads": 32,
+                    "num_kv_heads": 8, "head_dim": 128, "block_size": 16,
+                    "l2": "inputs larger than L2 (671 MB of KV per step)"}}))
+
+    def mixed():
+        rows = {}
+        mb = synth.mixed_sweep(16)
+        for bs in (8, 16, 32, 64, 256):
+            batch = mb if bs == 16 else synth.mixed_sweep(bs, base=mb)
+            r = _decode_measure(ns(workload="mixed", block_size=bs), [batch], torch, device, n, w)
+            rows[str(bs)] = {k: r[k] for k in ("value", "ms_per_step", "pct_of_hbm_measured",
+                                                "pct_of_hbm_nominal_8tbs", "kernel",
+                                                "gpu_launches", "device_error_word")}
+            del batch
+        return {"unit": "GB/s", "by_block_size": rows,
+                "config": {"workload": "mixed serving batch", "num_seqs": 256,
+                           "context_lens": "log-uniform [16, 4096]", "num_q_heads": 32,
+                           "num_kv_heads": 8, "head_dim": 128,
+                           "pool": "2^20 / block_size blocks (the same token capacity)",
+                           "l2": "inputs larger than L2 (~770 MB of KV per step)"}}
+
+    guarded("mixed", mixed)
+    guarded("shared_prompt", lambda: _decode_measure(
+        ns(workload="shared_prompt"), None, torch, device, n, w,
+        {"config": {"workload": "OPT-13B-shaped shared-prompt decode with copy-on-write",
+                    "num_seqs": 64, "num_q_heads": 40, "num_kv_heads": 40, "head_dim": 128,
+                    "block_size": 16, "prompts": 16, "prompt_len": 512, "fork": 4}}))
+    guarded("window_1024", lambda: _decode_measure(
+        ns(workload="llama8b", window=1024), make_batches(ns(workload="llama8b"), 0),
+        torch, device, n, w,
+        {"config": {"workload": "Llama-3.1-8B-shaped decode, sliding window of 1,024 "
+                                "positions (bytes: the window's positions)",
+                    "batches_rotated": args.variants}}))
+    guarded("prefill", lambda: prefill_measure(args.pool_blocks, 0, n, w))
+    return out
 
 
 # ------------------------------------------------------------------------------------- main
@@ -886,6 +1118,10 @@ def main():
         dist = tdist
     try:
         res = run_ours(args, rank, world, local, dist)
+        if world == 1 and not args.no_extras and args.window == 0 and \
+                args.workload == "llama8b":
+            import torch
+            res["workloads"] = run_extras(args, torch, torch.device("cuda", local))
     finally:
         if dist is not None:
             dist.barrier()

@@ -62,3 +62,46 @@ def split_scratch_bytes(context_lens, num_q_heads: int, head_dim: int, partition
 def new_token_bytes(num_tokens: int, num_kv_heads: int, head_dim: int, elem_bytes: int = 2) -> int:
     """The KV write of a step: each new token's K and V rows read once and written once."""
     return 2 * 2 * num_tokens * num_kv_heads * head_dim * elem_bytes
+
+
+def stream_split_scratch_bytes(context_lens, num_kv_heads: int, group: int, head_dim: int,
+                               num_ctas: int, tile: int = 64) -> int:
+    """Workspace bytes the even-split kernel moves for one call: the work is the
+    list of (sequence, kv head) segments in order, each cut into tiles of ``tile``
+    tokens (an empty sequence still has one tile), and CTA c takes tiles
+    [c*W/n, (c+1)*W/n). A segment whose tiles belong to more than one CTA leaves
+    one piece per such CTA -- (head_dim + 2) fp32 for each of its ``group`` q
+    heads -- written once and read back once by the merge, plus a 4-byte counter
+    read and written per piece."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    n = int(num_ctas)
+    if n <= 0 or lens.size == 0:
+        return 0
+    per_seg = np.maximum(1, (lens + tile - 1) // tile)
+    seg = np.repeat(per_seg, num_kv_heads)           # sequences in order, kv heads inner
+    first = np.concatenate([[0], np.cumsum(seg)[:-1]])
+    W = int(seg.sum())
+    owner = lambda x: ((x + 1) * n - 1) // W           # noqa: E731 -- CTA holding tile x
+    ca, cb = owner(first), owner(first + seg - 1)
+    starts = (np.arange(n + 1, dtype=np.int64) * W) // n
+    has = (starts[1:] > starts[:-1]).astype(np.int64)  # CTAs that own any tile
+    cum = np.concatenate([[0], np.cumsum(has)])
+    pieces = cum[cb + 1] - cum[ca]
+    pieces = np.where(pieces > 1, pieces, 0)
+    return int(pieces.sum() * (2 * group * (head_dim + 2) * 4 + 8))
+
+
+def unique_kv_bytes(block_tables, context_lens, block_size: int, num_kv_heads: int,
+                    head_dim: int, elem_bytes: int = 2) -> int:
+    """K and V bytes of every physical block a batch reads, each block counted once:
+    rows [0, r) of a block, r the most any sequence reads from it (blocks shared
+    by several sequences -- a forked prompt -- are counted once, not per reader)."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    rows = {}
+    for b, n in enumerate(lens):
+        nblk = int(-(-int(n) // block_size))
+        for i in range(nblk):
+            blk = int(block_tables[b][i])
+            r = min(block_size, int(n) - i * block_size)
+            rows[blk] = max(rows.get(blk, 0), r)
+    return int(2 * sum(rows.values()) * num_kv_heads * head_dim * elem_bytes)

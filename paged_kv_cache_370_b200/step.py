@@ -207,28 +207,49 @@ class HostDecodeStep:
 class HostStepPipeline:
     """Host-fed steps run back to back with every copy under some step's kernels.
 
-    The steps come in two sets (rounds) that take turns. Each round has three
-    CUDA graphs: the uploads of its steps' inputs, its steps' kernels, and the
-    downloads of its steps' outputs. ``run`` replays them on three streams so that
-    round r+1's uploads and round r-1's downloads run while round r's kernels do.
-    Because the graph of kernels has no copy nodes in it, each decode kernel keeps
-    its programmatic dependency on the one before it (the early start of an
+    The steps come in sets (rounds), each a list of HostDecodeStep with buffers of
+    its own. Each round has three CUDA graphs: the uploads of its steps' inputs,
+    its steps' kernels, and the downloads of its steps' outputs. ``run`` /
+    ``run_order`` replay rounds on three streams so that the next round's uploads
+    and the previous round's downloads run while a round's kernels do. Because the
+    graph of kernels has no copy nodes in it, each decode kernel keeps its
+    programmatic dependency on the one before it (the early start of an
     ``overlapped`` step). Rounds' kernels run in order on the caller's stream, so
     the steps see the pools in the order given.
 
-    A round's buffers are reused two rounds later: its uploads wait for its
+    Only the first round's uploads and the last round's downloads are not hidden,
+    so a short run is best served by rounds that grow from one step and shrink
+    back to one (``ramp_sizes``); a long one by two rounds taking turns.
+
+    A round's buffers are reused when it comes again: its uploads wait for its
     previous kernels to finish, and its kernels for its previous downloads."""
 
     def __init__(self, rounds):
-        if len(rounds) != 2 or not all(rounds):
-            raise ValueError("two non-empty rounds of HostDecodeStep are needed")
+        if len(rounds) < 1 or not all(rounds):
+            raise ValueError("non-empty rounds of HostDecodeStep are needed")
         self.rounds = [list(r) for r in rounds]
+        n = len(self.rounds)
         self.s_in = torch.cuda.Stream()
         self.s_out = torch.cuda.Stream()
         self._graphs = None
-        self._up = [torch.cuda.Event() for _ in range(2)]
-        self._comp = [torch.cuda.Event() for _ in range(2)]
-        self._down = [torch.cuda.Event() for _ in range(2)]
+        self._up = [torch.cuda.Event() for _ in range(n)]
+        self._comp = [torch.cuda.Event() for _ in range(n)]
+        self._down = [torch.cuda.Event() for _ in range(n)]
+
+    @staticmethod
+    def ramp_sizes(num_steps: int, cap: int = 16) -> list[int]:
+        """Round sizes for one pass of num_steps host-fed steps: 1, 2, 4, ... up to
+        cap, the middle in rounds of at most cap, then back down to 1. Each round's
+        uploads then fit under the kernels of the round before it, and its
+        downloads under the kernels of the round after it."""
+        up, s = [], 1
+        while s < cap and 2 * (sum(up) + s) <= num_steps:
+            up.append(s)
+            s *= 2
+        mid = num_steps - 2 * sum(up)
+        n_mid = -(-mid // cap) if mid > 0 else 0
+        mids = [mid // n_mid + (1 if i < mid % n_mid else 0) for i in range(n_mid)]
+        return up + mids + up[::-1]
 
     @property
     def steps_per_round(self):
@@ -270,16 +291,19 @@ class HostStepPipeline:
             e.record(cur)
 
     def run(self, n_rounds: int):
-        """Enqueue ``n_rounds`` rounds (alternating sets) on the current stream and
+        """Enqueue ``n_rounds`` rounds (the sets in turn) on the current stream and
         the two copy streams; on return the current stream is ordered after every
         copy. Results are in each step's ``h_out`` once the stream passes."""
+        self.run_order([i % len(self.rounds) for i in range(n_rounds)])
+
+    def run_order(self, order):
+        """Enqueue the rounds whose indices ``order`` lists, in that order (as ``run``)."""
         if self._graphs is None:
             self.capture()
         cs = torch.cuda.current_stream()
         self.s_in.wait_stream(cs)
         self.s_out.wait_stream(cs)
-        for i in range(n_rounds):
-            x = i % 2
+        for x in order:
             up, comp, down = self._graphs[x]
             self.s_in.wait_event(self._comp[x])
             with torch.cuda.stream(self.s_in):
