@@ -436,52 +436,53 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
 // Same computation, one CTA per (q head, 256 query tokens, sequence), with the
 // two products on tcgen05.mma and every operand of P V but V in tensor memory.
 // The 256 rows form two groups of 128 (one tcgen05 M each); the groups share
-// every K/V tile and take turns on the tensor core, so one group's softmax
-// overlaps the other group's products.
-//   warp 0      stages 64-key K/V tiles with TMA into a 4-stage ring;
-//   warp 1      allocates TMEM (512 columns: per group two S buffers and O); its
-//               lane 0 issues, per tile, S = Q K^T for each group and, one tile
-//               behind, O += P V for each group with P read from TMEM,
-//               committing each to an mbarrier;
+// every K/V tile of 128 keys and take turns on the tensor core, so one group's
+// softmax overlaps the other group's products.
+//   warp 0      stages 128-key K/V tiles with TMA into a ring (2 stages at
+//               head_dim 128, 4 at 64);
+//   warp 1      allocates TMEM (512 columns: per group one S/P buffer of 128
+//               columns and O); its lane 0 issues, per tile and group, S = Q K^T
+//               (M = 128, N = 128: the shape the tensor core runs at its full
+//               rate) once the K tile has landed and the group's previous P V has
+//               been issued, and O += P V with P read from TMEM once the group's
+//               softmax wrote P, committing each to an mbarrier;
 //   warps 2-9   one thread per query row (group = (warp - 2) / 4, TMEM lane =
 //               32 * (warp % 4) + lane): copy its Q row into shared memory, then
 //               per tile read its S row from TMEM, mask, online softmax in the
 //               log2 domain, and write its P row (16-bit, two per column) over
-//               the S row it came from. S being double-buffered, so is P: the
-//               softmax never waits for a P V to finish; the next S into a
-//               buffer is issued after the P V that reads it (the tensor core
-//               runs its operations in issue order).
+//               the first half of the S row it came from. The tensor core runs
+//               its operations in issue order, so the next S into the buffer
+//               cannot overwrite P before the P V that reads it; while one group
+//               runs its softmax the other group's products keep the tensor core
+//               busy.
 //               O is rescaled in TMEM only when the row max grows by more than
 //               2^8 (the weights against the stale max stay <= 2^8 and the final
 //               division by the matching sum keeps the result exact); l sums the
-//               weights before their rounding to 16 bits; at the end O / l goes
+//               same rounded weights the product uses; at the end O / l goes
 //               from TMEM to global memory.
 namespace t5 {
 
 constexpr int kM = 128;        // query rows per group (tcgen05 M)
 constexpr int kGroups = 2;
-constexpr int kN = 64;         // keys per tile
-// K/V ring depth (4 x 32 KB + 64 KB of Q at D = 128 fit the 227 KB limit)
-#ifndef PA_PREFILL_TC_STAGES
-#define PA_PREFILL_TC_STAGES 4
-#endif
-constexpr int kStages = PA_PREFILL_TC_STAGES;
+constexpr int kN = 128;        // keys per tile (tcgen05 N of S, K of P V)
 constexpr int kThreads = (2 + 4 * kGroups) * 32;
-// group g: S/P buffers at 256g + {0, 64} (P in the first 32 columns), O at 256g + 128
+// group g: S/P buffer at 256g (P in its first 64 columns), O at 256g + 128
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
 
 template <int D>
 struct Lay {
   static constexpr int kPanels = D / 64;
+  // K/V ring depth: 2 x 64 KB + 64 KB of Q at head_dim 128, 4 x 32 KB + 32 KB at 64
+  static constexpr int kStages = D == 128 ? 2 : 4;
   static constexpr int kQPanel = kGroups * kM * 128;          // 256 rows x 128 bytes
   static constexpr int kQBytes = kPanels * kQPanel;
-  static constexpr int kKVPanel = kN * 128;                   // 64 rows x 128 bytes
+  static constexpr int kKVPanel = kN * 128;                   // 128 rows x 128 bytes
   static constexpr int kStageBytes = 2 * kPanels * kKVPanel;  // K panels, then V panels
   static constexpr int kRingOff = kQBytes;
   static constexpr int kBarOff = kRingOff + kStages * kStageBytes;
-  // full[S] empty[S] q_ready mma_done, then per group s_full[2] p_full[2] pv_done[2]
-  static constexpr int kNumBars = 2 * kStages + 2 + 6 * kGroups;
+  // full[S] empty[S] q_ready mma_done, then per group s_full p_full pv_done
+  static constexpr int kNumBars = 2 * kStages + 2 + 3 * kGroups;
   static constexpr int kTmemOff = kBarOff + kNumBars * 8;
   static constexpr int kFlagOff = kTmemOff + 8;
   static constexpr int kBytes = 1024 + kFlagOff + 16;
@@ -494,7 +495,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const PrefillParams p) {
   using L = t5::Lay<D>;
-  constexpr int kM = t5::kM, kN = t5::kN, NS = t5::kStages, NG = t5::kGroups;
+  constexpr int kM = t5::kM, kN = t5::kN, NS = L::kStages, NG = t5::kGroups;
   constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t kIdescS = umma_idesc_f16(kFmt, 0, 0, kN, kM);  // Q (K-major) . K (K-major)
   constexpr uint32_t kIdescO = umma_idesc_f16(kFmt, 0, 1, D, kM);   // P (TMEM) . V (MN-major)
@@ -505,10 +506,10 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
   uint64_t *full_bar = bars, *empty_bar = bars + NS, *q_ready = bars + 2 * NS;
   uint64_t *mma_done = q_ready + 1;
-  // per group g: s_full[g][2], p_full[g][2], pv_done[g][2]
-  auto s_full = [&](int g, int i) { return mma_done + 1 + g * 6 + i; };
-  auto p_full = [&](int g, int i) { return mma_done + 1 + g * 6 + 2 + i; };
-  auto pv_done = [&](int g, int i) { return mma_done + 1 + g * 6 + 4 + i; };
+  // per group g: s_full, p_full, pv_done (each completes once per tile)
+  auto s_full = [&](int g) { return mma_done + 1 + g * 3; };
+  auto p_full = [&](int g) { return mma_done + 1 + g * 3 + 1; };
+  auto pv_done = [&](int g) { return mma_done + 1 + g * 3 + 2; };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
   const uint32_t q_sm = smem_u32(smem);
@@ -560,12 +561,11 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     }
     mbar_init(q_ready, 4 * 32 * NG);
     mbar_init(mma_done, 1);
-    for (int g = 0; g < NG; ++g)
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(s_full(g, i), 1);
-        mbar_init(p_full(g, i), 128);
-        mbar_init(pv_done(g, i), 1);
-      }
+    for (int g = 0; g < NG; ++g) {
+      mbar_init(s_full(g), 1);
+      mbar_init(p_full(g), 128);
+      mbar_init(pv_done(g), 1);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -589,6 +589,8 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       __syncwarp();
       const int t0 = k_base + i * kN;
       const int t_end = min(t0 + kN, n);
+      // boxes of this tile: whole blocks (block_size <= 128, at most 16 at block
+      // size 8) or one 128-row slice of a larger block
       const int nbox = t_end > t0 ? (bs <= kN ? (t_end - 1) / bs - t0 / bs + 1 : 1) : 0;
       int phys = -1;
       bool ok = false;
@@ -601,25 +603,31 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
       if (lane == 0) mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes);
       __syncwarp();
-      const int box = lane / (2 * L::kPanels);
-      const int which = (lane / L::kPanels) % 2;
-      const int pn = lane % L::kPanels;
-      const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
-      if (box < nbox && ((okmask >> box) & 1u)) {
-        const int r0 = bs > kN ? t0 % bs : 0;
-        const int srow = bs > kN ? 0 : box * bs;
-        const int y = (box_phys * p.num_kv_heads + kvh) * bs + r0;
-        tma_load_2d(ring + s * L::kStageBytes + (which * L::kPanels + pn) * L::kKVPanel + srow * 128,
-                    which ? &tmap_v : &tmap_k, pn * 64, y, &full_bar[s]);
+      // one copy per (box, K or V, panel), spread over the lanes in rounds of 32
+      // (every lane takes part in each round's shuffle of the box's block id)
+      for (int c0 = 0; c0 < nbox * 2 * L::kPanels; c0 += 32) {
+        const int c = c0 + lane;
+        const int box = c / (2 * L::kPanels);
+        const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
+        if (c < nbox * 2 * L::kPanels && ((okmask >> box) & 1u)) {
+          const int which = (c / L::kPanels) % 2;
+          const int pn = c % L::kPanels;
+          const int r0 = bs > kN ? t0 % bs : 0;
+          const int srow = bs > kN ? 0 : box * bs;
+          const int y = (box_phys * p.num_kv_heads + kvh) * bs + r0;
+          tma_load_2d(ring + s * L::kStageBytes + (which * L::kPanels + pn) * L::kKVPanel +
+                          srow * 128,
+                      which ? &tmap_v : &tmap_k, pn * 64, y, &full_bar[s]);
+        }
       }
     }
   } else if (warp == 1) {
     // ====================================================================== MMA issuer
     // Issues whatever is ready, in any order: S_j of a group as soon as K_j has
-    // landed and P_{j-2} V_{j-2}, which reads the same TMEM buffer, has been
-    // issued; P_j V_j of a group as soon as its softmax wrote P_j; a tile's
-    // stage goes back to the producer once every group that reads it has
-    // issued its P V.
+    // landed and P_{j-1} V_{j-1} of that group, which reads the same TMEM
+    // columns, has been issued; P_j V_j of a group as soon as its softmax wrote
+    // P_j; a tile's stage goes back to the producer once every group that reads
+    // it has issued its P V.
     if (lane == 0) {
       bool go = wait_bounded(q_ready, 0, abort_flag);
       tc_fence_after();
@@ -634,31 +642,30 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         for (int g = 0; g < NG; ++g) {
           if (npv[g] < gtiles[g]) done = false;
           const int js = ns[g];
-          if (js < gtiles[g] && (js < 2 || npv[g] >= js - 1) &&
-              mbar_try_wait(&full_bar[js % NS], (js / NS) & 1)) {
+          if (js < gtiles[g] && npv[g] >= js && mbar_try_wait(&full_bar[js % NS], (js / NS) & 1)) {
             tc_fence_after();
             const uint32_t kaddr = ring + (js % NS) * L::kStageBytes;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-              umma_f16(tmem + g * 256 + (js & 1) * kN,
+              umma_f16(tmem + g * 256,
                        umma_desc_sw128(q_sm + (kk / 4) * L::kQPanel + g * kM * 128 + (kk % 4) * 32,
                                        16, 1024),
                        umma_desc_sw128(kaddr + (kk / 4) * L::kKVPanel + (kk % 4) * 32, 16, 1024),
                        kIdescS, kk > 0);
-            umma_commit(s_full(g, js & 1));
+            umma_commit(s_full(g));
             ++ns[g];
             progress = true;
           }
           const int jp = npv[g];
-          if (jp < ns[g] && mbar_try_wait(p_full(g, jp & 1), (jp / 2) & 1)) {
+          if (jp < ns[g] && mbar_try_wait(p_full(g), jp & 1)) {
             tc_fence_after();
             const uint32_t vaddr = ring + (jp % NS) * L::kStageBytes + L::kPanels * L::kKVPanel;
 #pragma unroll
             for (int kk = 0; kk < kN / 16; ++kk)
-              umma_f16_ts(tmem + g * 256 + 128, tmem + g * 256 + (jp & 1) * kN + kk * 8,
+              umma_f16_ts(tmem + g * 256 + 128, tmem + g * 256 + kk * 8,
                           umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
                           kIdescO, jp > 0 || kk > 0);
-            umma_commit(pv_done(g, jp & 1));
+            umma_commit(pv_done(g));
             ++npv[g];
             progress = true;
           }
@@ -718,13 +725,14 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     const int wr1 = min(p_first + grp * kM + 32 * (warp % 4) + 31, n - 1);
     float m_ref = -INFINITY, l = 0.f;
     for (int j = 0; j < my_tiles; ++j) {
-      const int sb = j & 1, st = j % NS;
+      const int st = j % NS;
       const int t0 = k_base + j * kN;
-      wait_bounded(s_full(grp, sb), (j / 2) & 1, abort_flag);
+      wait_bounded(s_full(grp), j & 1, abort_flag);
       tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld32(trow + sb * kN, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(trow + sb * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      uint32_t sv[kN];
+#pragma unroll
+      for (int c4 = 0; c4 < kN / 32; ++c4)
+        tmem_ld32(trow + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c4 * 32]));
       tmem_wait_ld();
       // max of the raw scores (the scale is positive); masked keys become -inf.
       // The mask only matters on tiles that reach past a row of this warp or
@@ -747,13 +755,42 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
 #pragma unroll
         for (int e = 0; e < w; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + w]);
       float mx = mx8[0] * p.scale_log2;  // log2 domain
-      // move the reference max when it grew past the lazy bound (warp-uniform
-      // TMEM traffic: lanes that keep theirs scale by 1)
+      // move the reference max when it grew past the lazy bound; O and l are
+      // rescaled below, once this tile's scores are no longer held in registers
       const bool grow = mx > m_ref + t5::kLazyRescale || (m_ref == -INFINITY && mx > -INFINITY);
-      if (__any_sync(0xffffffffu, grow && m_ref > -INFINITY)) {
-        wait_bounded(pv_done(grp, (j - 1) & 1), ((j - 1) / 2) & 1, abort_flag);  // O has P_{j-1} V_{j-1}
+      const bool rescale = __any_sync(0xffffffffu, grow && m_ref > -INFINITY);
+      const float alpha = grow && m_ref > -INFINITY ? exp2f(m_ref - mx) : 1.f;
+      if (grow) m_ref = mx;
+      const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
+      // this tile's P row, weight = 2^(s * scale_log2 - m_ref) (one FMA and one
+      // exp2 per key), packed two per column over the first half of its S row;
+      // l sums the same rounded weights the product uses, so the output is an exact
+      // weighted average of V (each weight perturbed by at most one rounding), in
+      // four partial sums for a short dependency chain
+      // (in halves of 64 keys: each half's 32 packed columns are stored at once,
+      // which keeps fewer values live)
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c4 = 0; c4 < kN / 64; ++c4) {
+        uint32_t pw[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int k = c4 * 64 + 2 * c;
+          const float a = ex2_approx(fmaf(__uint_as_float(sv[k]), p.scale_log2, nbase));
+          const float b2 = ex2_approx(fmaf(__uint_as_float(sv[k + 1]), p.scale_log2, nbase));
+          float ra, rb;
+          pw[c] = Mma<T>::pack(a, b2, ra, rb);
+          ls[c % 4] += ra + rb;
+        }
+        tmem_st32(trow + c4 * 32, pw);
+      }
+      l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+      // O against the new reference max (warp-uniform TMEM traffic: lanes that keep
+      // theirs scale by 1), before this tile's P V is issued. S_j was issued after
+      // P_{j-1} V_{j-1} and the tensor core runs in order, so O already holds it.
+      if (rescale) {
+        wait_bounded(pv_done(grp), (j - 1) & 1, abort_flag);
         tc_fence_after();
-        const float alpha = grow && m_ref > -INFINITY ? exp2f(m_ref - mx) : 1.f;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t o[32];
@@ -763,27 +800,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           tmem_st32(trow + 128 + c4 * 32, o);
         }
-        tmem_wait_st();
-        l *= alpha;
       }
-      if (grow) m_ref = mx;
-      const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
-      // this tile's P row, weight = 2^(s * scale_log2 - m_ref) (one FMA and one
-      // exp2 per key), packed two per column over the first half of its S row;
-      // l sums the unrounded weights (|rounding| <= 2^-9 relative each), in four
-      // partial sums for a short dependency chain
-      uint32_t pw[32];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float a = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), p.scale_log2, nbase));
-        const float b2 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), p.scale_log2, nbase));
-        float ra, rb;
-        pw[c] = Mma<T>::pack(a, b2, ra, rb);
-        ls[c % 4] += a + b2;
-      }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      tmem_st32(trow + sb * kN, pw);
       // rows of V outside every row's keys may hold anything: zero them (both
       // groups zero the same rows of a shared stage; the writes are identical)
       const int nvalid = min(kN, n - t0);
@@ -800,11 +817,11 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full(grp, sb));
+      mbar_arrive(p_full(grp));
     }
     // ---- O / l -> global memory
     if (my_tiles > 0) {
-      wait_bounded(pv_done(grp, (my_tiles - 1) & 1), ((my_tiles - 1) / 2) & 1, abort_flag);
+      wait_bounded(pv_done(grp), (my_tiles - 1) & 1, abort_flag);
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       T *og = static_cast<T *>(p.out);
