@@ -95,6 +95,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="only the headline workload (no per-workload sub-objects)")
+    ap.add_argument("--kernel-seconds", type=float, default=0.5,
+                    help="length of the kernel-duration loop (at least 50 graph replays)")
     ap.add_argument("--extra-steps", type=int, default=20,
                     help="timed steps of each extra workload")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -560,7 +562,7 @@ def run_ours(args, rank, world, local, dist):
     # ---- the decode kernel's own duration: >= 50 replays of a graph of R decode
     # launches (about half a second), CUDA events on the same stream
     est = max(total_ms / max(K, 1), 1e-3)
-    reps = max(50, int(math.ceil(500.0 / (est * R))))
+    reps = max(50, int(math.ceil(1e3 * args.kernel_seconds / (est * R))))
     tk0 = time.time()
     dec_ms = time_graphs([(g_dec, reps)], stream, torch) / (reps * R)
     tk1 = time.time()
