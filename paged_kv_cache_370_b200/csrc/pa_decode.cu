@@ -609,9 +609,12 @@ struct Cfg {
   static constexpr int kRedBytes = kWarps * G * D * 4;
   static constexpr int kMetaOffset = kRedOffset + kRedBytes;
   static constexpr int kBarOffset = kMetaOffset + kStages * (int)sizeof(TileMeta);
-  static constexpr int kMlOffset = kBarOffset + 3 * kStages * 8;  // full, empty, meta barriers
+  static constexpr int kMlOffset = kBarOffset + 2 * kStages * 8;  // full, empty barriers
   static constexpr int kIdsOffset = kMlOffset + kWarps * 8 * 2 * 4;
   static constexpr int kCtrlOffset = kIdsOffset + 2 * kIdWindow * 8 * 4;  // one window per producer
+  // after the control words (W, x0, x1, abort, last): the metadata barriers
+  static constexpr int kMetaBarOffset = kCtrlOffset + 32;
+  static_assert(kStages * 8 <= 32, "metadata barriers fit the control area");
   static constexpr int kBytes = 1024 + kCtrlOffset + 64;  // + slack to align the ring to 1 KB
   // CTAs per SM the register budget is sized for
   static constexpr int kMinCtas = D == 64 ? 3 : (G <= 4 ? 2 : 1);
@@ -665,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
   // meta_bar[s]: the tile's metadata is in meta[s] (one arrival per tile, even
   // when the stage's data copies are not issued); the consumers take the metadata
   // through it after a give-up, so they never read metadata not yet written.
-  uint64_t *meta_bar = empty_bar + NS;
+  uint64_t *meta_bar = reinterpret_cast<uint64_t *>(smem + C::kMetaBarOffset);
   TileMeta *meta = reinterpret_cast<TileMeta *>(smem + C::kMetaOffset);
   float *mlbuf = reinterpret_cast<float *>(smem + C::kMlOffset);
   float *red = reinterpret_cast<float *>(smem + C::kRedOffset);
@@ -808,15 +811,15 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     uint32_t issued_mask = 0;
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % NS;
-      // stage free? The consumers arrive once per tile whatever happened, so this
-      // wait does not stop at a give-up: the producer never runs a full ring ahead
-      // and never rewrites metadata the consumers may still read
-      if (i >= NS) mbar_wait_sure(&empty_bar[s], ((i / NS) & 1) ^ 1);
-      // copies go out only while nothing has given up (and never in the test mode):
-      // a stage whose data never landed is not armed a second time
-      const bool issue = __shfl_sync(0xffffffffu, !p.starve && !*abort_flag, 0);
-      issued_mask = (issued_mask >> 1) | (issue ? 1u << (NS - 1) : 0u);
-      __syncwarp();
+      // stage free? The consumers arrive once per tile whatever happened; after a
+      // give-up this wait carries on without the early exit, so the producer never
+      // runs a full ring ahead and never rewrites metadata the consumers may still
+      // read
+      if (i >= NS && !mbar_wait_bounded(&empty_bar[s], ((i / NS) & 1) ^ 1, abort_flag))
+        mbar_wait_sure(&empty_bar[s], ((i / NS) & 1) ^ 1);
+      // has any wait given up? (read after the free-stage wait, which orders it after
+      // the consumers' give-up; used once the ids are in)
+      const int gave_up = *abort_flag;
       // this tile's ids have landed once at most kIdWindow - 1 newer groups are pending
       cp_async_wait<kIdWindow - 1>();
       __syncwarp();
@@ -833,6 +836,10 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       if (lane < tile_boxes(j, len_b) && !ok && !v_producer)
         atomicOr(&g_decode_error, PA_DEVERR_BLOCK_ID);
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+      // copies go out only while nothing has given up (and never in the test mode):
+      // a stage whose data never landed is not armed a second time
+      const bool issue = !p.starve && !__any_sync(0xffffffffu, gave_up);
+      issued_mask = (issued_mask >> 1) | (issue ? 1u << (NS - 1) : 0u);
       if (lane == 0 && !v_producer) {
         TileMeta &m = meta[s];
         m.b = b;
@@ -1112,11 +1119,27 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         }
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
     const bool whole = mt.seg_first_x >= x0 && (long long)mt.seg_first_x + mt.seg_tiles <= x1;
     const bool first_of_cta = mt.seg_first_x <= x0;
     const int slot = first_of_cta ? 2 * cta : 2 * cta + 1;
     const size_t hq_base = (size_t)mt.b * p.num_q_heads + (size_t)mt.kvh * G;
+    // a split segment's pieces belong to CTAs ca..cb (those of them that own tiles)
+    const long long sf = mt.seg_first_x;
+    const int ca = owner_cta(sf, W, nctas);
+    const int cb = owner_cta(sf + mt.seg_tiles - 1, W, nctas);
+    // The CTA holding the segment's first tiles reaches this point at the end of its
+    // range, when the other pieces (made at the start of theirs) are normally out
+    // already: if the counter says so, it merges at once from its own values and
+    // theirs, without writing its piece, fencing or counting (same order and
+    // arithmetic as the merge below, so the same bits)
+    if (!whole && ca == cta && tid == 0) {
+      int pieces = 0;
+      for (int cc = ca; cc <= cb; ++cc) pieces += cta_has_tiles(cc, W, nctas) ? 1 : 0;
+      *last_flag = ld_acquire_gpu(p.ws_counters + ca) == pieces - 1 ? 2 : 0;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
+    const bool merge_now = !whole && ca == cta && *last_flag == 2;
+    if (merge_now) __threadfence();
     for (int e0 = tid * 4; e0 < G * D; e0 += kWarps * 32 * 4) {
       const int h = e0 / D, d = e0 % D;
       float M = -INFINITY;
@@ -1138,6 +1161,39 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         const float inv = L > 0.f ? 1.f / L : 0.f;
         *reinterpret_cast<uint2 *>(static_cast<T *>(p.out) + (hq_base + h) * D + d) =
             Elem<T>::from_f32x4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
+      } else if (merge_now) {
+        // this CTA's piece (M, L, sum) first, then the others' in CTA order
+        float Mm = M;
+        for (int cc = ca + 1; cc <= cb; ++cc) {
+          if (!cta_has_tiles(cc, W, nctas)) continue;
+          Mm = fmaxf(Mm, __ldcg(p.ws_pieces + ((size_t)(2 * cc) * G + h) * kPieceStride + D));
+        }
+        float Lm = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (M != -INFINITY) {
+          const float w = exp2f(M - Mm);
+          Lm += w * L;
+          acc.x += w * sum.x;
+          acc.y += w * sum.y;
+          acc.z += w * sum.z;
+          acc.w += w * sum.w;
+        }
+        for (int cc = ca + 1; cc <= cb; ++cc) {
+          if (!cta_has_tiles(cc, W, nctas)) continue;
+          const float *pc = p.ws_pieces + ((size_t)(2 * cc) * G + h) * kPieceStride;
+          const float mc = __ldcg(pc + D);
+          if (mc == -INFINITY) continue;
+          const float w = exp2f(mc - Mm);
+          Lm += w * __ldcg(pc + D + 1);
+          const float4 v = __ldcg(reinterpret_cast<const float4 *>(pc + d));
+          acc.x += w * v.x;
+          acc.y += w * v.y;
+          acc.z += w * v.z;
+          acc.w += w * v.w;
+        }
+        const float inv = Lm > 0.f ? 1.f / Lm : 0.f;
+        *reinterpret_cast<uint2 *>(static_cast<T *>(p.out) + (hq_base + h) * D + d) =
+            Elem<T>::from_f32x4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
       } else {
         float *pc = p.ws_pieces + ((size_t)slot * G + h) * kPieceStride;
         *reinterpret_cast<float4 *>(pc + d) = sum;
@@ -1147,13 +1203,13 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         }
       }
     }
-    if (!whole) {
+    if (merge_now) {
+      // every other piece had arrived: nothing more counts on this segment
+      if (tid == 0) p.ws_counters[ca] = 0;
+    } else if (!whole) {
       // the piece is out; the CTA that completes the segment's last piece merges
       __threadfence();
       asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
-      const long long sf = mt.seg_first_x;
-      const int ca = owner_cta(sf, W, nctas);
-      const int cb = owner_cta(sf + mt.seg_tiles - 1, W, nctas);
       if (tid == 0) {
         int pieces = 0;  // one per CTA in [ca, cb] that owns tiles
         for (int cc = ca; cc <= cb; ++cc) pieces += cta_has_tiles(cc, W, nctas) ? 1 : 0;

@@ -473,19 +473,26 @@ constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O resc
 template <int D>
 struct Lay {
   static constexpr int kPanels = D / 64;
-  // K/V ring depth: 2 x 64 KB + 64 KB of Q at head_dim 128, 4 x 32 KB + 32 KB at 64
-  static constexpr int kStages = D == 128 ? 2 : 4;
+  // Separate K and V rings: a K slot is free again once both groups' S have read
+  // it, long before the tile's P V, so K tiles are fetched further ahead. At
+  // head_dim 128: 64 KB of Q + 3 K slots + 2 V slots of 32 KB (224 KB); at 64:
+  // 32 KB of Q + 6 + 4 slots of 16 KB.
+  static constexpr int kKStages = D == 128 ? 3 : 6;
+  static constexpr int kVStages = D == 128 ? 2 : 4;
   static constexpr int kQPanel = kGroups * kM * 128;          // 256 rows x 128 bytes
   static constexpr int kQBytes = kPanels * kQPanel;
   static constexpr int kKVPanel = kN * 128;                   // 128 rows x 128 bytes
-  static constexpr int kStageBytes = 2 * kPanels * kKVPanel;  // K panels, then V panels
-  static constexpr int kRingOff = kQBytes;
-  static constexpr int kBarOff = kRingOff + kStages * kStageBytes;
-  // full[S] empty[S] q_ready mma_done, then per group s_full p_full pv_done
-  static constexpr int kNumBars = 2 * kStages + 2 + 3 * kGroups;
+  static constexpr int kSlotBytes = kPanels * kKVPanel;       // one operand of one tile
+  static constexpr int kKRingOff = kQBytes;
+  static constexpr int kVRingOff = kKRingOff + kKStages * kSlotBytes;
+  static constexpr int kBarOff = kVRingOff + kVStages * kSlotBytes;
+  // k_full[K] k_empty[K] v_full[V] v_empty[V] q_ready mma_done, then per group
+  // s_full p_full pv_done
+  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 + 3 * kGroups;
   static constexpr int kTmemOff = kBarOff + kNumBars * 8;
   static constexpr int kFlagOff = kTmemOff + 8;
   static constexpr int kBytes = 1024 + kFlagOff + 16;
+  static_assert(kBytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 }  // namespace t5
@@ -495,7 +502,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const PrefillParams p) {
   using L = t5::Lay<D>;
-  constexpr int kM = t5::kM, kN = t5::kN, NS = L::kStages, NG = t5::kGroups;
+  constexpr int kM = t5::kM, kN = t5::kN, NK = L::kKStages, NV = L::kVStages, NG = t5::kGroups;
   constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t kIdescS = umma_idesc_f16(kFmt, 0, 0, kN, kM);  // Q (K-major) . K (K-major)
   constexpr uint32_t kIdescO = umma_idesc_f16(kFmt, 0, 1, D, kM);   // P (TMEM) . V (MN-major)
@@ -504,7 +511,8 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
-  uint64_t *full_bar = bars, *empty_bar = bars + NS, *q_ready = bars + 2 * NS;
+  uint64_t *k_full = bars, *k_empty = bars + NK, *v_full = bars + 2 * NK;
+  uint64_t *v_empty = v_full + NV, *q_ready = v_full + 2 * NV;
   uint64_t *mma_done = q_ready + 1;
   // per group g: s_full, p_full, pv_done (each completes once per tile)
   auto s_full = [&](int g) { return mma_done + 1 + g * 3; };
@@ -513,7 +521,8 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
   const uint32_t q_sm = smem_u32(smem);
-  const uint32_t ring = smem_u32(smem + L::kRingOff);
+  const uint32_t k_ring = smem_u32(smem + L::kKRingOff);
+  const uint32_t v_ring = smem_u32(smem + L::kVRingOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.x;
@@ -555,9 +564,13 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   const int ntiles = gtiles[NG - 1] > 0 ? gtiles[NG - 1] : gtiles[0];
 
   if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);  // one tcgen05.commit per use
+    for (int s = 0; s < NK; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);  // one tcgen05.commit per use
+    }
+    for (int s = 0; s < NV; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(q_ready, 4 * 32 * NG);
     mbar_init(mma_done, 1);
@@ -582,15 +595,13 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
     }
     const int32_t *row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
-    const uint32_t box_bytes = 2u * L::kPanels * align * 128u;  // K and V of one box
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i % NS;
-      if (i >= NS && !wait_bounded(&empty_bar[s], ((i / NS) & 1) ^ 1, abort_flag)) break;
-      __syncwarp();
+    const uint32_t box_bytes = (uint32_t)L::kPanels * align * 128u;  // one operand of one box
+    // one operand (K: which = 0, V: 1) of tile i into its ring slot: every box of
+    // the tile (whole blocks, at most 16 at block size 8, or one 128-row slice of a
+    // larger block), one copy per (box, panel) spread over the lanes
+    auto load = [&](int i, int which) {
       const int t0 = k_base + i * kN;
       const int t_end = min(t0 + kN, n);
-      // boxes of this tile: whole blocks (block_size <= 128, at most 16 at block
-      // size 8) or one 128-row slice of a larger block
       const int nbox = t_end > t0 ? (bs <= kN ? (t_end - 1) / bs - t0 / bs + 1 : 1) : 0;
       int phys = -1;
       bool ok = false;
@@ -598,53 +609,89 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         const int lb = t0 / bs + lane;
         phys = lb < p.max_blocks_per_seq ? __ldg(row + lb) : -1;
         ok = phys >= 0 && phys < p.num_blocks;
-        if (!ok) atomicOr(&g_prefill_error, PA_DEVERR_BLOCK_ID);
+        if (!ok && which == 0) atomicOr(&g_prefill_error, PA_DEVERR_BLOCK_ID);
       }
       const unsigned okmask = __ballot_sync(0xffffffffu, ok);
-      if (lane == 0) mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes);
+      uint64_t *bar = which ? &v_full[i % NV] : &k_full[i % NK];
+      if (lane == 0) mbar_expect_tx_arrive(bar, __popc(okmask) * box_bytes);
       __syncwarp();
-      // one copy per (box, K or V, panel), spread over the lanes in rounds of 32
-      // (every lane takes part in each round's shuffle of the box's block id)
-      for (int c0 = 0; c0 < nbox * 2 * L::kPanels; c0 += 32) {
+      const uint32_t slot = which ? v_ring + (i % NV) * L::kSlotBytes
+                                  : k_ring + (i % NK) * L::kSlotBytes;
+      for (int c0 = 0; c0 < nbox * L::kPanels; c0 += 32) {
         const int c = c0 + lane;
-        const int box = c / (2 * L::kPanels);
+        const int box = c / L::kPanels;
         const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
-        if (c < nbox * 2 * L::kPanels && ((okmask >> box) & 1u)) {
-          const int which = (c / L::kPanels) % 2;
+        if (c < nbox * L::kPanels && ((okmask >> box) & 1u)) {
           const int pn = c % L::kPanels;
           const int r0 = bs > kN ? t0 % bs : 0;
           const int srow = bs > kN ? 0 : box * bs;
           const int y = (box_phys * p.num_kv_heads + kvh) * bs + r0;
-          tma_load_2d(ring + s * L::kStageBytes + (which * L::kPanels + pn) * L::kKVPanel +
-                          srow * 128,
-                      which ? &tmap_v : &tmap_k, pn * 64, y, &full_bar[s]);
+          tma_load_2d(slot + pn * L::kKVPanel + srow * 128, which ? &tmap_v : &tmap_k, pn * 64, y,
+                      bar);
         }
+      }
+    };
+    // K tiles first (S needs them first) and as far ahead as the K ring allows;
+    // a V tile once its K tile is out and a V slot is free
+    int ik = 0, iv = 0;
+    unsigned long long idle_since = global_ns();
+    while (ik < ntiles || iv < ntiles) {
+      bool progress = false;
+      if (ik < ntiles && (ik < NK || mbar_try_wait(&k_empty[ik % NK], ((ik / NK) & 1) ^ 1))) {
+        load(ik++, 0);
+        progress = true;
+      }
+      if (iv < ik && (iv < NV || mbar_try_wait(&v_empty[iv % NV], ((iv / NV) & 1) ^ 1))) {
+        load(iv++, 1);
+        progress = true;
+      }
+      if (progress) {
+        idle_since = global_ns();
+      } else if (*abort_flag || global_ns() - idle_since > kWaitLimitNs) {
+        if (lane == 0 && !*abort_flag) atomicOr(&g_prefill_error, PA_DEVERR_TIMEOUT);
+        break;
       }
     }
   } else if (warp == 1) {
     // ====================================================================== MMA issuer
-    // Issues whatever is ready, in any order: S_j of a group as soon as K_j has
-    // landed and P_{j-1} V_{j-1} of that group, which reads the same TMEM
-    // columns, has been issued; P_j V_j of a group as soon as its softmax wrote
-    // P_j; a tile's stage goes back to the producer once every group that reads
-    // it has issued its P V.
+    // Issues whatever is ready: P_j V_j of a group as soon as its softmax wrote
+    // P_j and V_j has landed, then at once S_{j+1} of that group (K_{j+1} landed;
+    // it reads the TMEM columns P_j V_j reads, and the tensor core runs them in
+    // issue order); a K slot goes back to the producer once every group that
+    // reads it has issued its S, a V slot once they have issued their P V.
     if (lane == 0) {
       bool go = wait_bounded(q_ready, 0, abort_flag);
       tc_fence_after();
       int ns[NG], npv[NG];
 #pragma unroll
       for (int g = 0; g < NG; ++g) ns[g] = npv[g] = 0;
-      int released = 0;
+      int released = 0, released_k = 0;
       unsigned long long idle_since = global_ns();
       while (go) {
         bool done = true, progress = false;
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
           if (npv[g] < gtiles[g]) done = false;
-          const int js = ns[g];
-          if (js < gtiles[g] && npv[g] >= js && mbar_try_wait(&full_bar[js % NS], (js / NS) & 1)) {
+          // this group's P V first, then at once its next S: the tensor core runs
+          // them back to back and the group's softmax gets its next S soonest
+          const int jp = npv[g];
+          if (jp < ns[g] && mbar_try_wait(p_full(g), jp & 1) &&
+              mbar_try_wait(&v_full[jp % NV], (jp / NV) & 1)) {
             tc_fence_after();
-            const uint32_t kaddr = ring + (js % NS) * L::kStageBytes;
+            const uint32_t vaddr = v_ring + (jp % NV) * L::kSlotBytes;
+#pragma unroll
+            for (int kk = 0; kk < kN / 16; ++kk)
+              umma_f16_ts(tmem + g * 256 + 128, tmem + g * 256 + kk * 8,
+                          umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
+                          kIdescO, jp > 0 || kk > 0);
+            umma_commit(pv_done(g));
+            ++npv[g];
+            progress = true;
+          }
+          const int js = ns[g];
+          if (js < gtiles[g] && npv[g] >= js && mbar_try_wait(&k_full[js % NK], (js / NK) & 1)) {
+            tc_fence_after();
+            const uint32_t kaddr = k_ring + (js % NK) * L::kSlotBytes;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
               umma_f16(tmem + g * 256,
@@ -656,28 +703,26 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
             ++ns[g];
             progress = true;
           }
-          const int jp = npv[g];
-          if (jp < ns[g] && mbar_try_wait(p_full(g), jp & 1)) {
-            tc_fence_after();
-            const uint32_t vaddr = ring + (jp % NS) * L::kStageBytes + L::kPanels * L::kKVPanel;
-#pragma unroll
-            for (int kk = 0; kk < kN / 16; ++kk)
-              umma_f16_ts(tmem + g * 256 + 128, tmem + g * 256 + kk * 8,
-                          umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
-                          kIdescO, jp > 0 || kk > 0);
-            umma_commit(pv_done(g));
-            ++npv[g];
-            progress = true;
-          }
         }
-        // release, in order, every tile all of whose readers have issued P V
+        // release, in order, every K tile all of whose readers have issued S, and
+        // every V tile all of whose readers have issued P V (each commit arrives
+        // once the products issued before it have finished reading)
+        while (released_k < ntiles) {
+          bool all = true;
+#pragma unroll
+          for (int g = 0; g < NG; ++g)
+            if (released_k < gtiles[g] && ns[g] <= released_k) all = false;
+          if (!all) break;
+          umma_commit(&k_empty[released_k % NK]);
+          ++released_k;
+        }
         while (released < ntiles) {
           bool all = true;
 #pragma unroll
           for (int g = 0; g < NG; ++g)
             if (released < gtiles[g] && npv[g] <= released) all = false;
           if (!all) break;
-          umma_commit(&empty_bar[released % NS]);
+          umma_commit(&v_empty[released % NV]);
           ++released;
         }
         if (done) break;
@@ -725,7 +770,6 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     const int wr1 = min(p_first + grp * kM + 32 * (warp % 4) + 31, n - 1);
     float m_ref = -INFINITY, l = 0.f;
     for (int j = 0; j < my_tiles; ++j) {
-      const int st = j % NS;
       const int t0 = k_base + j * kN;
       wait_bounded(s_full(grp), j & 1, abort_flag);
       tc_fence_after();
@@ -806,7 +850,9 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       const int nvalid = min(kN, n - t0);
       const int nskip = max(0, lo_first - t0);
       if (nvalid < kN || nskip > 0) {
-        unsigned char *vz = smem + L::kRingOff + st * L::kStageBytes + L::kPanels * L::kKVPanel;
+        // (after the TMA copies into this V slot have landed)
+        wait_bounded(&v_full[j % NV], (j / NV) & 1, abort_flag);
+        unsigned char *vz = smem + L::kVRingOff + (j % NV) * L::kSlotBytes;
         for (int c = r; c < kN * 8 * L::kPanels; c += 128) {
           const int vr = c / (8 * L::kPanels), pn = (c / 8) % L::kPanels, ch = c % 8;
           if (vr >= nskip && vr < nvalid) continue;

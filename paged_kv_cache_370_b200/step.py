@@ -237,19 +237,46 @@ class HostStepPipeline:
         self._down = [torch.cuda.Event() for _ in range(n)]
 
     @staticmethod
-    def ramp_sizes(num_steps: int, cap: int = 16) -> list[int]:
-        """Round sizes for one pass of num_steps host-fed steps: 1, 2, 4, ... up to
-        cap, the middle in rounds of at most cap, then back down to 1. Each round's
-        uploads then fit under the kernels of the round before it, and its
-        downloads under the kernels of the round after it."""
-        up, s = [], 1
-        while s < cap and 2 * (sum(up) + s) <= num_steps:
-            up.append(s)
-            s *= 2
-        mid = num_steps - 2 * sum(up)
-        n_mid = -(-mid // cap) if mid > 0 else 0
-        mids = [mid // n_mid + (1 if i < mid % n_mid else 0) for i in range(n_mid)]
-        return up + mids + up[::-1]
+    def ramp_sizes(num_steps: int, cap: int = 16, kernel_us: float = 55.0,
+                   upload_us: float = 16.0, download_us: float = 10.0,
+                   boundary_us: float = 10.0) -> list[int]:
+        """Round sizes for one pass of num_steps host-fed steps. A round's uploads
+        run under the kernels of the round before it and its downloads under those
+        of the round after it, so consecutive sizes may grow at most by the ratio
+        of a step's kernel time to its upload time and shrink at most by the ratio
+        to its download time (defaults: the Llama-3.1-8B-shaped batch, ~55 us of
+        kernels, ~16 and ~10 us of PCIe per step). What stays exposed is the first
+        round's uploads, the last round's downloads and a gap at each round
+        boundary; the sizes (at most ``cap``) minimise that sum."""
+        grow, shrink = kernel_us / upload_us, kernel_us / download_us
+        if num_steps <= 0:
+            return []
+        sizes = range(1, min(cap, num_steps) + 1)
+        # best[(left, prev)]: (cost, rest) of finishing `left` steps after a round of `prev`
+        best = {}
+
+        def solve(left, prev):
+            key = (left, prev)
+            if key in best:
+                return best[key]
+            out = (download_us * prev, [])  # prev is the last round
+            if left > 0:
+                out = (float("inf"), None)
+                for s in sizes:
+                    if s > left or s > grow * prev or prev > shrink * s:
+                        continue
+                    c, rest = solve(left - s, s)
+                    if rest is not None and c + boundary_us < out[0]:
+                        out = (c + boundary_us, [s] + rest)
+            best[key] = out
+            return out
+
+        cands = []
+        for s0 in sizes:
+            c, rest = solve(num_steps - s0, s0)
+            if rest is not None:
+                cands.append((upload_us * s0 + c, [s0] + rest))
+        return min(cands)[1]
 
     @property
     def steps_per_round(self):
