@@ -594,7 +594,7 @@ def run_ours(args, rank, world, local, dist):
 
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, steps, infos, torch, device, dist, world)
+        e2e = run_e2e(args, steps, infos, torch, device, dist, world, dec_ms)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and batches is not None:
         cpu = cpu_baseline(batches[0], args.cpu_seconds)
@@ -648,7 +648,7 @@ def run_ours(args, rank, world, local, dist):
     return res
 
 
-def run_e2e(args, steps, infos, torch, device, dist, world):
+def run_e2e(args, steps, infos, torch, device, dist, world, step_ms):
     """The same K steps fed from pinned host buffers through the library's
     HostStepPipeline: each round's uploads, kernels and downloads are graphs on
     three streams, the next round's uploads and the previous round's downloads
@@ -668,14 +668,37 @@ def run_e2e(args, steps, infos, torch, device, dist, world):
                               partition_tokens=s.partition_tokens, copy_pairs=s.copy_pairs,
                               fused=s.fused, window=s.window, overlapped=s.overlapped)
 
+    # this box's copy times for one step's inputs and output (pinned host memory),
+    # to plan the rounds: a round's uploads must fit under the kernels before it
+    probe = host_step(steps[0])
+    probe.upload()
+    probe.download()
+    torch.cuda.synchronize()
+    st = torch.cuda.Stream()
+
+    def copy_us(fn, reps=20):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(st):
+            a0.record(st)
+            for _ in range(reps):
+                fn()
+            a1.record(st)
+        torch.cuda.synchronize()
+        return 1e3 * a0.elapsed_time(a1) / reps
+
+    up_us, down_us = copy_us(probe.upload), copy_us(probe.download)
+    kern_us = 1e3 * step_ms
+    del probe
     if K <= 64:
-        sizes = HostStepPipeline.ramp_sizes(K)
+        sizes = HostStepPipeline.ramp_sizes(K, kernel_us=kern_us, upload_us=up_us,
+                                            download_us=down_us)
         rounds, i = [], 0
         for n in sizes:
             rounds.append([host_step(steps[(off + i + j) % V]) for j in range(n)])
             i += n
         order = list(range(len(rounds)))
-        shape = f"rounds of {sizes} steps"
+        shape = (f"rounds of {sizes} steps, planned from {up_us:.1f} us per upload, "
+                 f"{down_us:.1f} us per download and {kern_us:.1f} us of kernels per step")
     else:
         R = V * max(1, args.round_reps)
         n_rounds, rest = divmod(K, R)
@@ -687,16 +710,20 @@ def run_e2e(args, steps, infos, torch, device, dist, world):
         shape = f"two sets of {R} steps taking turns, then {rest}"
     pipe = HostStepPipeline(rounds)
     pipe.capture()
+    # the whole pass (every round's uploads, kernels and downloads on their three
+    # streams) as one graph: one launch from the host
+    g = pipe.graph(order)
+    stream = torch.cuda.current_stream()
     for _ in range(max(1, -(-max(args.warmup, 3) // K))):  # >= W (and >= 3) warm-up steps
-        pipe.run_order(order)
+        g.replay()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    pipe.run_order(order)
-    b.record()
+    a.record(stream)
+    g.replay()
+    b.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -708,9 +735,10 @@ def run_e2e(args, steps, infos, torch, device, dist, world):
             "h2d_bytes_per_step": int(np.mean([h.h2d_bytes for h in h_all])),
             "d2h_bytes_per_step": int(np.mean([h.d2h_bytes for h in h_all])),
             "how": "pinned host inputs copied in and output copied out every step through the "
-                   f"library's HostStepPipeline ({shape}); each round's uploads, kernels and "
-                   "downloads replayed as CUDA graphs on three streams, the next round's "
-                   "uploads and the previous round's downloads under a round's kernels"}
+                   f"library's HostStepPipeline ({shape}): each round's uploads, kernels and "
+                   "downloads on three streams, the next round's uploads and the previous "
+                   "round's downloads under a round's kernels, the whole pass one CUDA graph "
+                   "(HostStepPipeline.graph)"}
 
 
 # --------------------------------------------------------------------------- CPU (oracle)

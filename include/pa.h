@@ -316,7 +316,10 @@ pa_status pa_decode_append_window(void *out, const void *q, const void *k_new, c
  * head_dim 64 or 128; block_size a power of two >= 8 (PA_ERR_UNSUPPORTED otherwise).
  * Allocates nothing. Lengths or q_start entries out of range are clamped and reported
  * (PA_DEVERR_CONTEXT_LEN); bad block ids are skipped and reported (PA_DEVERR_BLOCK_ID).
- * One kernel launch.
+ * Stream work: a 4-byte clear of the device's work counter, then one persistent kernel
+ * (one CTA per SM takes (q head, 256 query tokens, sequence) items from that counter).
+ * The counter is one per device and per library: two pa_prefill calls on one device must
+ * not run at the same time (issue them on one stream, or order their streams).
  * ------------------------------------------------------------------------------------------ */
 pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
                      const int32_t *block_tables, int max_blocks_per_seq,

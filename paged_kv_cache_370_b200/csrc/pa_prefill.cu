@@ -39,6 +39,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 #include <type_traits>
 
 #include "pa.h"
@@ -433,33 +434,37 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
 }
 
 // ============================================================ tcgen05 kernel (5th-gen tensor cores)
-// Same computation, one CTA per (q head, 256 query tokens, sequence), with the
-// two products on tcgen05.mma and every operand of P V but V in tensor memory.
+// Same computation on tcgen05.mma, with every operand of P V but V in tensor
+// memory, as a persistent kernel: one CTA per SM takes work items -- (q head, 256
+// query tokens, sequence) -- one after another from a counter, and fetches the next
+// item's Q and K/V tiles while the current one computes, so neither a CTA launch
+// nor the first fetches of an item leave the SM idle.
 // The 256 rows form two groups of 128 (one tcgen05 M each); the groups share
 // every K/V tile of 128 keys and take turns on the tensor core, so one group's
 // softmax overlaps the other group's products.
-//   warp 0      stages 128-key K/V tiles with TMA into a ring (2 stages at
-//               head_dim 128, 4 at 64);
+//   warp 0      takes items, publishes each item's extent, stages its Q rows (TMA,
+//               once the previous item's last S has read the Q buffer) and its
+//               128-key K and V tiles (TMA) into two rings (3 K slots and 2 V slots
+//               at head_dim 128; 6 and 4 at 64);
 //   warp 1      allocates TMEM (512 columns: per group one S/P buffer of 128
-//               columns and O); its lane 0 issues, per tile and group, S = Q K^T
-//               (M = 128, N = 128: the shape the tensor core runs at its full
-//               rate) once the K tile has landed and the group's previous P V has
-//               been issued, and O += P V with P read from TMEM once the group's
-//               softmax wrote P, committing each to an mbarrier;
+//               columns and O); its lane 0 issues, item after item, per group: O +=
+//               P V with P read from TMEM once the group's softmax wrote P and V
+//               landed (the item's first one once the previous item's O was read
+//               out), then at once the group's next S = Q K^T (M = 128, N = 128: the
+//               shape the tensor core runs at its full rate), committing each to an
+//               mbarrier; a K slot goes back once both groups' S read it, a V slot
+//               once both groups' P V did;
 //   warps 2-9   one thread per query row (group = (warp - 2) / 4, TMEM lane =
-//               32 * (warp % 4) + lane): copy its Q row into shared memory, then
-//               per tile read its S row from TMEM, mask, online softmax in the
-//               log2 domain, and write its P row (16-bit, two per column) over
-//               the first half of the S row it came from. The tensor core runs
-//               its operations in issue order, so the next S into the buffer
-//               cannot overwrite P before the P V that reads it; while one group
-//               runs its softmax the other group's products keep the tensor core
-//               busy.
+//               32 * (warp % 4) + lane): per tile read its S row from TMEM, mask,
+//               online softmax in the log2 domain, and write its P row (16-bit, two
+//               per column) over the first half of the S row it came from; at the
+//               end of an item O / l goes from TMEM to global memory. The tensor
+//               core runs its operations in issue order, so the next S cannot
+//               overwrite P before the P V that reads it.
 //               O is rescaled in TMEM only when the row max grows by more than
 //               2^8 (the weights against the stale max stay <= 2^8 and the final
 //               division by the matching sum keeps the result exact); l sums the
-//               same rounded weights the product uses; at the end O / l goes
-//               from TMEM to global memory.
+//               same rounded weights the product uses.
 namespace t5 {
 
 constexpr int kM = 128;        // query rows per group (tcgen05 M)
@@ -469,6 +474,19 @@ constexpr int kThreads = (2 + 4 * kGroups) * 32;
 // group g: S/P buffer at 256g (P in its first 64 columns), O at 256g + 128
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O rescale
+
+// One work item as the producer publishes it to the other warps.
+struct Item {
+  int valid;        // 0: no more items
+  int h, b;         // q head, sequence
+  int qs0, q0;      // first query row of the sequence in q / out, first row of the item in it
+  int rows;         // query rows of the item (<= 256)
+  int n;            // positions of the sequence
+  int p_first;      // position of the item's first query row
+  int k_base;       // first key of the item's first tile
+  int gtiles[kGroups];  // tiles each group needs
+  int ntiles;       // tiles of the item (the larger of the two)
+};
 
 template <int D>
 struct Lay {
@@ -486,10 +504,11 @@ struct Lay {
   static constexpr int kKRingOff = kQBytes;
   static constexpr int kVRingOff = kKRingOff + kKStages * kSlotBytes;
   static constexpr int kBarOff = kVRingOff + kVStages * kSlotBytes;
-  // k_full[K] k_empty[K] v_full[V] v_empty[V] q_ready mma_done, then per group
-  // s_full p_full pv_done
-  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 + 3 * kGroups;
-  static constexpr int kTmemOff = kBarOff + kNumBars * 8;
+  // k_full[K] k_empty[K] v_full[V] v_empty[V] q_full q_free item_full[2]
+  // item_free[2] mma_done, then per group s_full p_full pv_done o_free
+  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 7 + 4 * kGroups;
+  static constexpr int kItemOff = kBarOff + kNumBars * 8;
+  static constexpr int kTmemOff = kItemOff + 2 * (int)sizeof(Item);
   static constexpr int kFlagOff = kTmemOff + 8;
   static constexpr int kBytes = 1024 + kFlagOff + 16;
   static_assert(kBytes <= 227 * 1024, "shared memory of one CTA");
@@ -500,8 +519,9 @@ struct Lay {
 template <typename T, int D>
 __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-    const PrefillParams p) {
+    const __grid_constant__ CUtensorMap tmap_q, const PrefillParams p, unsigned *work) {
   using L = t5::Lay<D>;
+  using t5::Item;
   constexpr int kM = t5::kM, kN = t5::kN, NK = L::kKStages, NV = L::kVStages, NG = t5::kGroups;
   constexpr uint32_t kFmt = std::is_same<T, __nv_bfloat16>::value ? 1u : 0u;
   constexpr uint32_t kIdescS = umma_idesc_f16(kFmt, 0, 0, kN, kM);  // Q (K-major) . K (K-major)
@@ -512,12 +532,15 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
   uint64_t *k_full = bars, *k_empty = bars + NK, *v_full = bars + 2 * NK;
-  uint64_t *v_empty = v_full + NV, *q_ready = v_full + 2 * NV;
-  uint64_t *mma_done = q_ready + 1;
-  // per group g: s_full, p_full, pv_done (each completes once per tile)
-  auto s_full = [&](int g) { return mma_done + 1 + g * 3; };
-  auto p_full = [&](int g) { return mma_done + 1 + g * 3 + 1; };
-  auto pv_done = [&](int g) { return mma_done + 1 + g * 3 + 2; };
+  uint64_t *v_empty = v_full + NV, *q_full = v_full + 2 * NV, *q_free = q_full + 1;
+  uint64_t *item_full = q_free + 1, *item_free = item_full + 2, *mma_done = item_free + 2;
+  // per group g: s_full, p_full, pv_done (each completes once per tile of the group),
+  // o_free (once per item: the group's O has been read out)
+  auto s_full = [&](int g) { return mma_done + 1 + g * 4; };
+  auto p_full = [&](int g) { return mma_done + 1 + g * 4 + 1; };
+  auto pv_done = [&](int g) { return mma_done + 1 + g * 4 + 2; };
+  auto o_free = [&](int g) { return mma_done + 1 + g * 4 + 3; };
+  Item *items = reinterpret_cast<Item *>(smem + L::kItemOff);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::kTmemOff);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::kFlagOff);
   const uint32_t q_sm = smem_u32(smem);
@@ -525,43 +548,11 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   const uint32_t v_ring = smem_u32(smem + L::kVRingOff);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int h = blockIdx.x;
-  const int qt = p.q_tiles - 1 - (int)blockIdx.y;  // the longest tiles first
-  const int b = blockIdx.z;
-  const int G = p.num_q_heads / p.num_kv_heads;
-  const int kvh = h / G;
   const int bs = p.block_size;
   const int cap = p.max_blocks_per_seq * bs;
-
-  // ---- this CTA's query rows and key range (the same in every thread)
-  int n = __ldg(p.context_lens + b);
-  const int qs0 = __ldg(p.q_start + b), qs1 = __ldg(p.q_start + b + 1);
-  int m = qs1 - qs0;
-  bool bad = false;
-  if (n < 0 || n > cap || n > p.max_context_len) {
-    bad = true;
-    n = n < 0 ? 0 : min(min(n, cap), p.max_context_len);
-  }
-  if (m < 0 || m > n || qs0 < 0 || qs1 > p.num_tokens) {
-    bad = true;
-    m = 0;
-  }
-  if (bad && tid == 0 && h == 0 && blockIdx.y == 0)
-    atomicOr(&g_prefill_error, PA_DEVERR_CONTEXT_LEN);
-  const int q0 = qt * NG * kM;
-  if (q0 >= m) return;  // no query rows here (uniform; before any TMEM is taken)
-  const int rows = min(NG * kM, m - q0);
-  const int p_first = n - m + q0;
   const int align = bs < kN ? bs : kN;
-  const int k_base = first_key(p_first, p.window) & ~(align - 1);
-  // tiles each group needs (up to its last row); group 1 may have no rows
-  int gtiles[NG];
-#pragma unroll
-  for (int g = 0; g < NG; ++g) {
-    const int grows = min(kM, rows - g * kM);
-    gtiles[g] = grows > 0 ? (p_first + g * kM + grows - 1 + 1 - k_base + kN - 1) / kN : 0;
-  }
-  const int ntiles = gtiles[NG - 1] > 0 ? gtiles[NG - 1] : gtiles[0];
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const long long n_items = (long long)p.num_q_heads * p.q_tiles * p.num_seqs;
 
   if (tid == 0) {
     for (int s = 0; s < NK; ++s) {
@@ -572,12 +563,18 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    mbar_init(q_ready, 4 * 32 * NG);
+    mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&item_full[i], 1);
+      mbar_init(&item_free[i], 1 + 4 * NG);  // the issuing thread and every softmax warp
+    }
     mbar_init(mma_done, 1);
     for (int g = 0; g < NG; ++g) {
       mbar_init(s_full(g), 1);
       mbar_init(p_full(g), 128);
       mbar_init(pv_done(g), 1);
+      mbar_init(o_free(g), 128);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -593,147 +590,253 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_q)));
     }
-    const int32_t *row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
     const uint32_t box_bytes = (uint32_t)L::kPanels * align * 128u;  // one operand of one box
-    // one operand (K: which = 0, V: 1) of tile i into its ring slot: every box of
-    // the tile (whole blocks, at most 16 at block size 8, or one 128-row slice of a
-    // larger block), one copy per (box, panel) spread over the lanes
-    auto load = [&](int i, int which) {
-      const int t0 = k_base + i * kN;
-      const int t_end = min(t0 + kN, n);
-      const int nbox = t_end > t0 ? (bs <= kN ? (t_end - 1) / bs - t0 / bs + 1 : 1) : 0;
-      int phys = -1;
-      bool ok = false;
-      if (lane < nbox) {
-        const int lb = t0 / bs + lane;
-        phys = lb < p.max_blocks_per_seq ? __ldg(row + lb) : -1;
-        ok = phys >= 0 && phys < p.num_blocks;
-        if (!ok && which == 0) atomicOr(&g_prefill_error, PA_DEVERR_BLOCK_ID);
-      }
-      const unsigned okmask = __ballot_sync(0xffffffffu, ok);
-      uint64_t *bar = which ? &v_full[i % NV] : &k_full[i % NK];
-      if (lane == 0) mbar_expect_tx_arrive(bar, __popc(okmask) * box_bytes);
-      __syncwarp();
-      const uint32_t slot = which ? v_ring + (i % NV) * L::kSlotBytes
-                                  : k_ring + (i % NK) * L::kSlotBytes;
-      for (int c0 = 0; c0 < nbox * L::kPanels; c0 += 32) {
-        const int c = c0 + lane;
-        const int box = c / L::kPanels;
-        const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
-        if (c < nbox * L::kPanels && ((okmask >> box) & 1u)) {
-          const int pn = c % L::kPanels;
-          const int r0 = bs > kN ? t0 % bs : 0;
-          const int srow = bs > kN ? 0 : box * bs;
-          const int y = (box_phys * p.num_kv_heads + kvh) * bs + r0;
-          tma_load_2d(slot + pn * L::kKVPanel + srow * 128, which ? &tmap_v : &tmap_k, pn * 64, y,
-                      bar);
+    long long kt = 0, vt = 0;  // K / V tiles loaded so far (over all items)
+    int nq = 0;                // items whose Q rows were loaded (those with tiles)
+    for (int it = 0;; ++it) {
+      // ---- the next work item: (q head fastest, longest query tiles first, sequence)
+      long long k = 0;
+      if (lane == 0) k = atomicAdd(work, 1u);
+      k = __shfl_sync(0xffffffffu, k, 0);
+      Item I;
+      I.valid = k < n_items;
+      if (I.valid) {
+        I.h = (int)(k % p.num_q_heads);
+        const int qt = p.q_tiles - 1 - (int)((k / p.num_q_heads) % p.q_tiles);
+        I.b = (int)(k / ((long long)p.num_q_heads * p.q_tiles));
+        int n = __ldg(p.context_lens + I.b);
+        const int qs0 = __ldg(p.q_start + I.b), qs1 = __ldg(p.q_start + I.b + 1);
+        int m = qs1 - qs0;
+        bool bad = false;
+        if (n < 0 || n > cap || n > p.max_context_len) {
+          bad = true;
+          n = n < 0 ? 0 : min(min(n, cap), p.max_context_len);
         }
-      }
-    };
-    // K tiles first (S needs them first) and as far ahead as the K ring allows;
-    // a V tile once its K tile is out and a V slot is free
-    int ik = 0, iv = 0;
-    unsigned long long idle_since = global_ns();
-    while (ik < ntiles || iv < ntiles) {
-      bool progress = false;
-      if (ik < ntiles && (ik < NK || mbar_try_wait(&k_empty[ik % NK], ((ik / NK) & 1) ^ 1))) {
-        load(ik++, 0);
-        progress = true;
-      }
-      if (iv < ik && (iv < NV || mbar_try_wait(&v_empty[iv % NV], ((iv / NV) & 1) ^ 1))) {
-        load(iv++, 1);
-        progress = true;
-      }
-      if (progress) {
-        idle_since = global_ns();
-      } else if (*abort_flag || global_ns() - idle_since > kWaitLimitNs) {
-        if (lane == 0 && !*abort_flag) atomicOr(&g_prefill_error, PA_DEVERR_TIMEOUT);
-        break;
-      }
-    }
-  } else if (warp == 1) {
-    // ====================================================================== MMA issuer
-    // Issues whatever is ready: P_j V_j of a group as soon as its softmax wrote
-    // P_j and V_j has landed, then at once S_{j+1} of that group (K_{j+1} landed;
-    // it reads the TMEM columns P_j V_j reads, and the tensor core runs them in
-    // issue order); a K slot goes back to the producer once every group that
-    // reads it has issued its S, a V slot once they have issued their P V.
-    if (lane == 0) {
-      bool go = wait_bounded(q_ready, 0, abort_flag);
-      tc_fence_after();
-      int ns[NG], npv[NG];
-#pragma unroll
-      for (int g = 0; g < NG; ++g) ns[g] = npv[g] = 0;
-      int released = 0, released_k = 0;
-      unsigned long long idle_since = global_ns();
-      while (go) {
-        bool done = true, progress = false;
+        if (m < 0 || m > n || qs0 < 0 || qs1 > p.num_tokens) {
+          bad = true;
+          m = 0;
+        }
+        if (bad && lane == 0 && I.h == 0 && qt == p.q_tiles - 1)
+          atomicOr(&g_prefill_error, PA_DEVERR_CONTEXT_LEN);
+        I.n = n;
+        I.qs0 = qs0;
+        I.q0 = qt * NG * kM;
+        I.rows = m > I.q0 ? min(NG * kM, m - I.q0) : 0;
+        I.p_first = n - m + I.q0;
+        I.k_base = first_key(I.p_first, p.window) & ~(align - 1);
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-          if (npv[g] < gtiles[g]) done = false;
-          // this group's P V first, then at once its next S: the tensor core runs
-          // them back to back and the group's softmax gets its next S soonest
-          const int jp = npv[g];
-          if (jp < ns[g] && mbar_try_wait(p_full(g), jp & 1) &&
-              mbar_try_wait(&v_full[jp % NV], (jp / NV) & 1)) {
-            tc_fence_after();
-            const uint32_t vaddr = v_ring + (jp % NV) * L::kSlotBytes;
-#pragma unroll
-            for (int kk = 0; kk < kN / 16; ++kk)
-              umma_f16_ts(tmem + g * 256 + 128, tmem + g * 256 + kk * 8,
-                          umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
-                          kIdescO, jp > 0 || kk > 0);
-            umma_commit(pv_done(g));
-            ++npv[g];
-            progress = true;
+          const int grows = min(kM, I.rows - g * kM);
+          I.gtiles[g] =
+              grows > 0 ? (I.p_first + g * kM + grows - 1 + 1 - I.k_base + kN - 1) / kN : 0;
+        }
+        I.ntiles = max(I.gtiles[0], I.gtiles[1]);
+      }
+      // publish it (the slot's previous item has been read by every other warp)
+      const int slot = it & 1;
+      if (it >= 2) wait_bounded(&item_free[slot], ((it >> 1) - 1) & 1, abort_flag);
+      if (lane == 0) {
+        items[slot] = I;
+        mbar_arrive(&item_full[slot]);
+      }
+      __syncwarp();
+      if (!I.valid) break;
+      if (I.ntiles == 0) continue;  // no query rows in this tile of the sequence
+      // ---- its Q rows, once the previous item's last S has read the buffer
+      if (nq > 0 && !wait_bounded(q_free, (nq - 1) & 1, abort_flag)) break;
+      if (lane == 0) {
+        mbar_expect_tx_arrive(q_full, (uint32_t)L::kQBytes);
+        for (int pn = 0; pn < L::kPanels; ++pn)
+          tma_load_3d(q_sm + pn * L::kQPanel, &tmap_q, pn * 64, I.h, I.qs0 + I.q0, q_full);
+      }
+      __syncwarp();
+      ++nq;
+      // ---- its K and V tiles
+      const int32_t *row = p.block_tables + (size_t)I.b * p.max_blocks_per_seq;
+      const int kvh = I.h / G;
+      auto load = [&](int i, int which, long long gi) {
+        const int t0 = I.k_base + i * kN;
+        const int t_end = min(t0 + kN, I.n);
+        const int nbox = t_end > t0 ? (bs <= kN ? (t_end - 1) / bs - t0 / bs + 1 : 1) : 0;
+        int phys = -1;
+        bool ok = false;
+        if (lane < nbox) {
+          const int lb = t0 / bs + lane;
+          phys = lb < p.max_blocks_per_seq ? __ldg(row + lb) : -1;
+          ok = phys >= 0 && phys < p.num_blocks;
+          if (!ok && which == 0) atomicOr(&g_prefill_error, PA_DEVERR_BLOCK_ID);
+        }
+        const unsigned okmask = __ballot_sync(0xffffffffu, ok);
+        uint64_t *bar = which ? &v_full[gi % NV] : &k_full[gi % NK];
+        if (lane == 0) mbar_expect_tx_arrive(bar, __popc(okmask) * box_bytes);
+        __syncwarp();
+        const uint32_t slot_addr = which ? v_ring + (uint32_t)(gi % NV) * L::kSlotBytes
+                                         : k_ring + (uint32_t)(gi % NK) * L::kSlotBytes;
+        for (int c0 = 0; c0 < nbox * L::kPanels; c0 += 32) {
+          const int c = c0 + lane;
+          const int box = c / L::kPanels;
+          const int box_phys = __shfl_sync(0xffffffffu, phys, box & 31);
+          if (c < nbox * L::kPanels && ((okmask >> box) & 1u)) {
+            const int pn = c % L::kPanels;
+            const int r0 = bs > kN ? t0 % bs : 0;
+            const int srow = bs > kN ? 0 : box * bs;
+            const int y = (box_phys * p.num_kv_heads + kvh) * bs + r0;
+            tma_load_2d(slot_addr + pn * L::kKVPanel + srow * 128, which ? &tmap_v : &tmap_k,
+                        pn * 64, y, bar);
           }
-          const int js = ns[g];
-          if (js < gtiles[g] && npv[g] >= js && mbar_try_wait(&k_full[js % NK], (js / NK) & 1)) {
-            tc_fence_after();
-            const uint32_t kaddr = k_ring + (js % NK) * L::kSlotBytes;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              umma_f16(tmem + g * 256,
-                       umma_desc_sw128(q_sm + (kk / 4) * L::kQPanel + g * kM * 128 + (kk % 4) * 32,
-                                       16, 1024),
-                       umma_desc_sw128(kaddr + (kk / 4) * L::kKVPanel + (kk % 4) * 32, 16, 1024),
-                       kIdescS, kk > 0);
-            umma_commit(s_full(g));
-            ++ns[g];
-            progress = true;
-          }
         }
-        // release, in order, every K tile all of whose readers have issued S, and
-        // every V tile all of whose readers have issued P V (each commit arrives
-        // once the products issued before it have finished reading)
-        while (released_k < ntiles) {
-          bool all = true;
-#pragma unroll
-          for (int g = 0; g < NG; ++g)
-            if (released_k < gtiles[g] && ns[g] <= released_k) all = false;
-          if (!all) break;
-          umma_commit(&k_empty[released_k % NK]);
-          ++released_k;
+      };
+      // K tiles first (S needs them first) and as far ahead as the K ring allows;
+      // a V tile once its K tile is out and a V slot is free
+      int ik = 0, iv = 0;
+      unsigned long long idle_since = global_ns();
+      bool stop = false;
+      while (ik < I.ntiles || iv < I.ntiles) {
+        bool progress = false;
+        if (ik < I.ntiles && (kt < NK || mbar_try_wait(&k_empty[kt % NK], ((kt / NK) & 1) ^ 1))) {
+          load(ik++, 0, kt++);
+          progress = true;
         }
-        while (released < ntiles) {
-          bool all = true;
-#pragma unroll
-          for (int g = 0; g < NG; ++g)
-            if (released < gtiles[g] && npv[g] <= released) all = false;
-          if (!all) break;
-          umma_commit(&v_empty[released % NV]);
-          ++released;
+        if (iv < ik && (vt < NV || mbar_try_wait(&v_empty[vt % NV], ((vt / NV) & 1) ^ 1))) {
+          load(iv++, 1, vt++);
+          progress = true;
         }
-        if (done) break;
-        const unsigned long long now = global_ns();
         if (progress) {
-          idle_since = now;
-        } else if (now - idle_since > kWaitLimitNs || *abort_flag) {
+          idle_since = global_ns();
+        } else if (*abort_flag || global_ns() - idle_since > kWaitLimitNs) {
+          if (lane == 0 && !*abort_flag) atomicOr(&g_prefill_error, PA_DEVERR_TIMEOUT);
           *abort_flag = 1;
-          atomicOr(&g_prefill_error, PA_DEVERR_TIMEOUT);
+          stop = true;
           break;
         }
+      }
+      if (stop) break;
+    }
+    // after a give-up, let the copies already issued land (bounded) before the CTA
+    // exits: the last copy into each K / V slot and the last Q copy
+    if (*abort_flag && lane == 0) {
+      const unsigned long long t_start = global_ns();
+      auto settle = [&](uint64_t *bar, uint32_t parity) {
+        while (!mbar_try_wait(bar, parity) && global_ns() - t_start < kWaitLimitNs) {
+        }
+      };
+      for (long long i = kt > NK ? kt - NK : 0; i < kt; ++i) settle(&k_full[i % NK], (i / NK) & 1);
+      for (long long i = vt > NV ? vt - NV : 0; i < vt; ++i) settle(&v_full[i % NV], (i / NV) & 1);
+      if (nq > 0) settle(q_full, (nq - 1) & 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ====================================================================== MMA issuer
+    if (lane == 0) {
+      long long ts[NG], tp[NG];  // S / P V issued so far per group (over all items)
+      long long krel = 0, vrel = 0;  // K / V tiles released so far
+      long long kb = 0;              // K (and V) tiles of the items before this one
+#pragma unroll
+      for (int g = 0; g < NG; ++g) ts[g] = tp[g] = 0;
+      int nq = 0;  // items whose Q was loaded (those with tiles)
+      bool go = true;
+      for (int it = 0; go; ++it) {
+        const int slot = it & 1;
+        if (!wait_bounded(&item_full[slot], (it >> 1) & 1, abort_flag)) break;
+        const Item I = items[slot];
+        mbar_arrive(&item_free[slot]);
+        if (!I.valid) break;
+        if (I.ntiles == 0) continue;
+        if (!wait_bounded(q_full, nq & 1, abort_flag)) break;
+        tc_fence_after();
+        int ns[NG], npv[NG];
+#pragma unroll
+        for (int g = 0; g < NG; ++g) ns[g] = npv[g] = 0;
+        int released_k = 0, released_v = 0;
+        bool q_released = false;
+        unsigned long long idle_since = global_ns();
+        while (true) {
+          bool done = true, progress = false;
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+            if (npv[g] < I.gtiles[g]) done = false;
+            // this group's P V first (the item's first one once the group's O of the
+            // previous item was read out), then at once its next S
+            const int jp = npv[g];
+            const long long gv = kb + jp;  // global V tile
+            if (jp < ns[g] && mbar_try_wait(p_full(g), tp[g] & 1) &&
+                mbar_try_wait(&v_full[gv % NV], (gv / NV) & 1) &&
+                (jp > 0 || nq == 0 || mbar_try_wait(o_free(g), (nq - 1) & 1))) {
+              tc_fence_after();
+              const uint32_t vaddr = v_ring + (uint32_t)(gv % NV) * L::kSlotBytes;
+#pragma unroll
+              for (int kk = 0; kk < kN / 16; ++kk)
+                umma_f16_ts(tmem + g * 256 + 128, tmem + g * 256 + kk * 8,
+                            umma_desc_sw128(vaddr + kk * 16 * 128, L::kKVPanel, 1024),
+                            kIdescO, jp > 0 || kk > 0);
+              umma_commit(pv_done(g));
+              ++npv[g];
+              ++tp[g];
+              progress = true;
+            }
+            const int js = ns[g];
+            const long long gk = kb + js;  // global K tile
+            if (js < I.gtiles[g] && npv[g] >= js &&
+                mbar_try_wait(&k_full[gk % NK], (gk / NK) & 1)) {
+              tc_fence_after();
+              const uint32_t kaddr = k_ring + (uint32_t)(gk % NK) * L::kSlotBytes;
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk)
+                umma_f16(tmem + g * 256,
+                         umma_desc_sw128(q_sm + (kk / 4) * L::kQPanel + g * kM * 128 +
+                                             (kk % 4) * 32,
+                                         16, 1024),
+                         umma_desc_sw128(kaddr + (kk / 4) * L::kKVPanel + (kk % 4) * 32, 16, 1024),
+                         kIdescS, kk > 0);
+              umma_commit(s_full(g));
+              ++ns[g];
+              ++ts[g];
+              progress = true;
+            }
+          }
+          // once every S of the item is out, the Q buffer goes back to the producer
+          if (!q_released && ns[0] == I.gtiles[0] && ns[1] == I.gtiles[1]) {
+            umma_commit(q_free);
+            q_released = true;
+          }
+          // release, in order, every K tile all of whose readers have issued S, and
+          // every V tile all of whose readers have issued P V (each commit arrives
+          // once the products issued before it have finished reading)
+          while (released_k < I.ntiles) {
+            bool all = true;
+#pragma unroll
+            for (int g = 0; g < NG; ++g)
+              if (released_k < I.gtiles[g] && ns[g] <= released_k) all = false;
+            if (!all) break;
+            umma_commit(&k_empty[krel % NK]);
+            ++krel;
+            ++released_k;
+          }
+          while (released_v < I.ntiles) {
+            bool all = true;
+#pragma unroll
+            for (int g = 0; g < NG; ++g)
+              if (released_v < I.gtiles[g] && npv[g] <= released_v) all = false;
+            if (!all) break;
+            umma_commit(&v_empty[vrel % NV]);
+            ++vrel;
+            ++released_v;
+          }
+          if (done && released_v == I.ntiles) break;
+          const unsigned long long now = global_ns();
+          if (progress) {
+            idle_since = now;
+          } else if (now - idle_since > kWaitLimitNs || *abort_flag) {
+            *abort_flag = 1;
+            atomicOr(&g_prefill_error, PA_DEVERR_TIMEOUT);
+            go = false;
+            break;
+          }
+        }
+        kb += I.ntiles;
+        ++nq;
       }
       // every product issued so far has finished before TMEM is released
       umma_commit(mma_done);
@@ -744,153 +847,153 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     // ====================================================== softmax, one row per thread
     const int grp = (warp - 2) / 4;
     const int r = 32 * (warp % 4) + lane;          // row in the group == TMEM lane
-    const int R = grp * kM + r;                    // row in the CTA
+    const int R = grp * kM + r;                    // row in the item
     const uint32_t trow = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + grp * 256;
-    const int my_tiles = gtiles[grp];
-    // this row of Q -> shared memory (128-byte swizzled, K-major)
-    {
-      const T *qg = static_cast<const T *>(p.q);
-      constexpr int kChunks = D / 8;
-#pragma unroll 4
-      for (int ch = 0; ch < kChunks; ++ch) {
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (R < rows)
-          v = __ldg(reinterpret_cast<const uint4 *>(
-                        qg + ((size_t)(qs0 + q0 + R) * p.num_q_heads + h) * D) + ch);
-        *reinterpret_cast<uint4 *>(smem + (ch / 8) * L::kQPanel + R * 128 +
-                                   (((ch % 8) ^ (R & 7)) << 4)) = v;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(q_ready);
-    }
-    const int pr = min(p_first + R, n - 1);        // rows past the chunk: computed, not stored
-    const int lo = first_key(pr, p.window);
-    const int lo_first = first_key(p_first, p.window);
-    const int wr0 = min(p_first + grp * kM + 32 * (warp % 4), n - 1);
-    const int wr1 = min(p_first + grp * kM + 32 * (warp % 4) + 31, n - 1);
-    float m_ref = -INFINITY, l = 0.f;
-    for (int j = 0; j < my_tiles; ++j) {
-      const int t0 = k_base + j * kN;
-      wait_bounded(s_full(grp), j & 1, abort_flag);
-      tc_fence_after();
-      uint32_t sv[kN];
-#pragma unroll
-      for (int c4 = 0; c4 < kN / 32; ++c4)
-        tmem_ld32(trow + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c4 * 32]));
-      tmem_wait_ld();
-      // max of the raw scores (the scale is positive); masked keys become -inf.
-      // The mask only matters on tiles that reach past a row of this warp or
-      // start before a row's window (warp-uniform).
-      if (t0 + kN - 1 > wr0 || (p.window > 0 && t0 < first_key(wr1, p.window))) {
-#pragma unroll
-        for (int c = 0; c < kN; ++c) {
-          const int kp = t0 + c;
-          if (kp > pr || kp < lo) sv[c] = __float_as_uint(-INFINITY);
-        }
-      }
-      // eight independent running maxima, then a tree: a short dependency chain
-      float mx8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sv[e]);
-#pragma unroll
-      for (int c = 8; c < kN; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], __uint_as_float(sv[c]));
-#pragma unroll
-      for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-        for (int e = 0; e < w; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + w]);
-      float mx = mx8[0] * p.scale_log2;  // log2 domain
-      // move the reference max when it grew past the lazy bound; O and l are
-      // rescaled below, once this tile's scores are no longer held in registers
-      const bool grow = mx > m_ref + t5::kLazyRescale || (m_ref == -INFINITY && mx > -INFINITY);
-      const bool rescale = __any_sync(0xffffffffu, grow && m_ref > -INFINITY);
-      const float alpha = grow && m_ref > -INFINITY ? exp2f(m_ref - mx) : 1.f;
-      if (grow) m_ref = mx;
-      const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
-      // this tile's P row, weight = 2^(s * scale_log2 - m_ref) (one FMA and one
-      // exp2 per key), packed two per column over the first half of its S row;
-      // l sums the same rounded weights the product uses, so the output is an exact
-      // weighted average of V (each weight perturbed by at most one rounding), in
-      // four partial sums for a short dependency chain
-      // (in halves of 64 keys: each half's 32 packed columns are stored at once,
-      // which keeps fewer values live)
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c4 = 0; c4 < kN / 64; ++c4) {
-        uint32_t pw[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int k = c4 * 64 + 2 * c;
-          const float a = ex2_approx(fmaf(__uint_as_float(sv[k]), p.scale_log2, nbase));
-          const float b2 = ex2_approx(fmaf(__uint_as_float(sv[k + 1]), p.scale_log2, nbase));
-          float ra, rb;
-          pw[c] = Mma<T>::pack(a, b2, ra, rb);
-          ls[c % 4] += ra + rb;
-        }
-        tmem_st32(trow + c4 * 32, pw);
-      }
-      l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
-      // O against the new reference max (warp-uniform TMEM traffic: lanes that keep
-      // theirs scale by 1), before this tile's P V is issued. S_j was issued after
-      // P_{j-1} V_{j-1} and the tensor core runs in order, so O already holds it.
-      if (rescale) {
-        wait_bounded(pv_done(grp), (j - 1) & 1, abort_flag);
+    long long tg = 0;   // tiles of this group so far (over all items)
+    long long vg = 0;   // V tiles of the items before this one
+    for (int it = 0;; ++it) {
+      const int slot = it & 1;
+      if (!wait_bounded(&item_full[slot], (it >> 1) & 1, abort_flag)) break;
+      const Item I = items[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&item_free[slot]);
+      if (!I.valid) break;
+      if (I.ntiles == 0) continue;
+      const int my_tiles = I.gtiles[grp];
+      const int rows = I.rows, n = I.n, k_base = I.k_base, p_first = I.p_first;
+      const int pr = min(p_first + R, n - 1);       // rows past the chunk: computed, not stored
+      const int lo = first_key(pr, p.window);
+      const int lo_first = first_key(p_first, p.window);
+      const int wr0 = min(p_first + grp * kM + 32 * (warp % 4), n - 1);
+      const int wr1 = min(p_first + grp * kM + 32 * (warp % 4) + 31, n - 1);
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < my_tiles; ++j) {
+        const long long t = tg + j;
+        const int t0 = k_base + j * kN;
+        wait_bounded(s_full(grp), t & 1, abort_flag);
         tc_fence_after();
+        uint32_t sv[kN];
+#pragma unroll
+        for (int c4 = 0; c4 < kN / 32; ++c4)
+          tmem_ld32(trow + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[c4 * 32]));
+        tmem_wait_ld();
+        // max of the raw scores (the scale is positive); masked keys become -inf.
+        // The mask only matters on tiles that reach past a row of this warp or
+        // start before a row's window (warp-uniform).
+        if (t0 + kN - 1 > wr0 || (p.window > 0 && t0 < first_key(wr1, p.window))) {
+#pragma unroll
+          for (int c = 0; c < kN; ++c) {
+            const int kp = t0 + c;
+            if (kp > pr || kp < lo) sv[c] = __float_as_uint(-INFINITY);
+          }
+        }
+        // eight independent running maxima, then a tree: a short dependency chain
+        float mx8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sv[e]);
+#pragma unroll
+        for (int c = 8; c < kN; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], __uint_as_float(sv[c]));
+#pragma unroll
+        for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + w]);
+        const float mx = mx8[0] * p.scale_log2;  // log2 domain
+        // move the reference max when it grew past the lazy bound; O and l are
+        // rescaled below, once this tile's scores are no longer held in registers
+        const bool grow =
+            mx > m_ref + t5::kLazyRescale || (m_ref == -INFINITY && mx > -INFINITY);
+        const bool rescale = __any_sync(0xffffffffu, grow && m_ref > -INFINITY);
+        const float alpha = grow && m_ref > -INFINITY ? exp2f(m_ref - mx) : 1.f;
+        if (grow) m_ref = mx;
+        const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
+        // this tile's P row, weight = 2^(s * scale_log2 - m_ref) (one FMA and one
+        // exp2 per key), packed two per column over the first half of its S row, in
+        // halves of 64 keys (each half's 32 columns stored at once); l sums the same
+        // rounded weights the product uses, in four partial sums
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c4 = 0; c4 < kN / 64; ++c4) {
+          uint32_t pw[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int kx = c4 * 64 + 2 * c;
+            const float a = ex2_approx(fmaf(__uint_as_float(sv[kx]), p.scale_log2, nbase));
+            const float b2 = ex2_approx(fmaf(__uint_as_float(sv[kx + 1]), p.scale_log2, nbase));
+            float ra, rb;
+            pw[c] = Mma<T>::pack(a, b2, ra, rb);
+            ls[c % 4] += ra + rb;
+          }
+          tmem_st32(trow + c4 * 32, pw);
+        }
+        l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        // O against the new reference max (warp-uniform TMEM traffic: lanes that keep
+        // theirs scale by 1), before this tile's P V is issued. S was issued after
+        // the group's previous P V and the tensor core runs in order, so O holds it.
+        if (rescale) {
+          wait_bounded(pv_done(grp), (t - 1) & 1, abort_flag);
+          tc_fence_after();
+#pragma unroll
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t o[32];
+            tmem_ld32(trow + 128 + c4 * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(trow + 128 + c4 * 32, o);
+          }
+        }
+        // rows of V outside every row's keys may hold anything: zero them (both
+        // groups zero the same rows of a shared slot; the writes are identical)
+        const int nvalid = min(kN, n - t0);
+        const int nskip = max(0, lo_first - t0);
+        if (nvalid < kN || nskip > 0) {
+          const long long gv = vg + j;
+          // (after the TMA copies into this V slot have landed)
+          wait_bounded(&v_full[gv % NV], (gv / NV) & 1, abort_flag);
+          unsigned char *vz = smem + L::kVRingOff + (gv % NV) * L::kSlotBytes;
+          for (int c = r; c < kN * 8 * L::kPanels; c += 128) {
+            const int vr = c / (8 * L::kPanels), pn = (c / 8) % L::kPanels, ch = c % 8;
+            if (vr >= nskip && vr < nvalid) continue;
+            *reinterpret_cast<uint4 *>(vz + pn * L::kKVPanel + vr * 128 + (ch << 4)) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full(grp));
+      }
+      // ---- O / l -> global memory, then O goes back to the issuing thread
+      if (my_tiles > 0) {
+        wait_bounded(pv_done(grp), (tg + my_tiles - 1) & 1, abort_flag);
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        T *og = static_cast<T *>(p.out);
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t o[32];
           tmem_ld32(trow + 128 + c4 * 32, o);
           tmem_wait_ld();
+          if (R < rows) {
+            uint4 *dst = reinterpret_cast<uint4 *>(
+                og + ((size_t)(I.qs0 + I.q0 + R) * p.num_q_heads + I.h) * D + c4 * 32);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(trow + 128 + c4 * 32, o);
-        }
-      }
-      // rows of V outside every row's keys may hold anything: zero them (both
-      // groups zero the same rows of a shared stage; the writes are identical)
-      const int nvalid = min(kN, n - t0);
-      const int nskip = max(0, lo_first - t0);
-      if (nvalid < kN || nskip > 0) {
-        // (after the TMA copies into this V slot have landed)
-        wait_bounded(&v_full[j % NV], (j / NV) & 1, abort_flag);
-        unsigned char *vz = smem + L::kVRingOff + (j % NV) * L::kSlotBytes;
-        for (int c = r; c < kN * 8 * L::kPanels; c += 128) {
-          const int vr = c / (8 * L::kPanels), pn = (c / 8) % L::kPanels, ch = c % 8;
-          if (vr >= nskip && vr < nvalid) continue;
-          *reinterpret_cast<uint4 *>(vz + pn * L::kKVPanel + vr * 128 + (ch << 4)) =
-              make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full(grp));
-    }
-    // ---- O / l -> global memory
-    if (my_tiles > 0) {
-      wait_bounded(pv_done(grp), (my_tiles - 1) & 1, abort_flag);
-      tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      T *og = static_cast<T *>(p.out);
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t w[4];
+              float a, c;
 #pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        uint32_t o[32];
-        tmem_ld32(trow + 128 + c4 * 32, o);
-        tmem_wait_ld();
-        if (R < rows) {
-          uint4 *dst = reinterpret_cast<uint4 *>(
-              og + ((size_t)(qs0 + q0 + R) * p.num_q_heads + h) * D + c4 * 32);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t w[4];
-            float a, c;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = Mma<T>::pack(__uint_as_float(o[q4 * 8 + 2 * e]) * inv,
-                                  __uint_as_float(o[q4 * 8 + 2 * e + 1]) * inv, a, c);
-            dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int e = 0; e < 4; ++e)
+                w[e] = Mma<T>::pack(__uint_as_float(o[q4 * 8 + 2 * e]) * inv,
+                                    __uint_as_float(o[q4 * 8 + 2 * e + 1]) * inv, a, c);
+              dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(o_free(grp));
+      tg += my_tiles;
+      vg += I.ntiles;
     }
   }
   tc_fence_before();
@@ -924,17 +1027,97 @@ pa_status launch(const PrefillParams &prm, const void *k_cache, const void *v_ca
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+// The persistent kernel's work counter: one per device, cleared on the stream before
+// every launch (a 4-byte memset). Only a successful address lookup is kept.
+__device__ unsigned g_prefill_work;
+
+unsigned *prefill_work_counter() {
+  static std::mutex mu;
+  static unsigned *addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_prefill_work) != cudaSuccess || !a) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<unsigned *>(a);
+  }
+  return addr[dev];
+}
+
+// TMA tensor map over q viewed as [num_tokens][num_q_heads][head_dim]: boxes of 64
+// head_dim columns x 1 head x 256 tokens (one 128-row group pair of one head),
+// 128-byte swizzle; tokens past num_tokens read as zeros. Cached per (base, shape).
+bool q_tensor_map(CUtensorMap *map, const void *q, int num_tokens, int num_q_heads, int head_dim,
+                  pa_dtype dtype) {
+  struct Key {
+    const void *q;
+    int t, h, d, dt;
+  };
+  constexpr int kSlots = 16;
+  static std::mutex mu;
+  static Key keys[kSlots];
+  static CUtensorMap maps[kSlots];
+  static int used = 0, next = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (keys[i].q == q && keys[i].t == num_tokens && keys[i].h == num_q_heads &&
+        keys[i].d == head_dim && keys[i].dt == (int)dtype) {
+      *map = maps[i];
+      return true;
+    }
+  using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                     const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                     const cuuint32_t *, CUtensorMapInterleave,
+                                     CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                     CUtensorMapFloatOOBfill);
+  static EncodeTiledFn enc = [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &qr) != cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads,
+                              (cuuint64_t)num_tokens};
+  const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2,
+                                 (cuuint64_t)num_q_heads * head_dim * 2};
+  const cuuint32_t box[3] = {64u, 1u, (cuuint32_t)(t5::kGroups * t5::kM)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUtensorMap m;
+  if (enc(&m, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+          3, const_cast<void *>(q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int slot = used < kSlots ? used++ : (next++ % kSlots);
+  keys[slot] = Key{q, num_tokens, num_q_heads, head_dim, (int)dtype};
+  maps[slot] = m;
+  *map = m;
+  return true;
+}
+
 template <typename T, int D>
 pa_status launch_tc(const PrefillParams &prm_in, int max_q_len, const void *k_cache,
                     const void *v_cache, pa_dtype dtype, cudaStream_t stream) {
   using L = t5::Lay<D>;
   PrefillParams prm = prm_in;
   prm.q_tiles = (max_q_len + t5::kGroups * t5::kM - 1) / (t5::kGroups * t5::kM);
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tq;
   const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
   const int box_rows = prm.block_size < t5::kN ? prm.block_size : t5::kN;
   if (!pa_internal_pool_tensor_map(&tk, k_cache, rows, D, box_rows, dtype) ||
-      !pa_internal_pool_tensor_map(&tv, v_cache, rows, D, box_rows, dtype))
+      !pa_internal_pool_tensor_map(&tv, v_cache, rows, D, box_rows, dtype) ||
+      !q_tensor_map(&tq, prm.q, prm.num_tokens, prm.num_q_heads, D, dtype))
     return PA_ERR_CUDA;
   static bool configured[64] = {};
   int dev = 0;
@@ -945,8 +1128,16 @@ pa_status launch_tc(const PrefillParams &prm_in, int max_q_len, const void *k_ca
       return PA_ERR_CUDA;
     configured[dev] = true;
   }
-  dim3 grid((unsigned)prm.num_q_heads, (unsigned)prm.q_tiles, (unsigned)prm.num_seqs);
-  pa_prefill_tc_kernel<T, D><<<grid, t5::kThreads, L::kBytes, stream>>>(tk, tv, prm);
+  unsigned *work = prefill_work_counter();
+  if (!work) return PA_ERR_CUDA;
+  // one CTA per SM (a CTA fills an SM's shared and tensor memory), never more than items
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return PA_ERR_CUDA;
+  const long long n_items = (long long)prm.num_q_heads * prm.q_tiles * prm.num_seqs;
+  const unsigned grid = (unsigned)std::min<long long>(n_items, sms);
+  if (cudaMemsetAsync(work, 0, sizeof(unsigned), stream) != cudaSuccess) return PA_ERR_CUDA;
+  pa_prefill_tc_kernel<T, D><<<grid, t5::kThreads, L::kBytes, stream>>>(tk, tv, tq, prm, work);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

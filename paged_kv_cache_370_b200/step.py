@@ -248,7 +248,10 @@ class HostStepPipeline:
         kernels, ~16 and ~10 us of PCIe per step). What stays exposed is the first
         round's uploads, the last round's downloads and a gap at each round
         boundary; the sizes (at most ``cap``) minimise that sum."""
-        grow, shrink = kernel_us / upload_us, kernel_us / download_us
+        # (copies slower than the kernels cannot be hidden whatever the sizes: then
+        # rounds may still keep their size)
+        grow = max(1.0, kernel_us / max(upload_us, 1e-9))
+        shrink = max(1.0, kernel_us / max(download_us, 1e-9))
         if num_steps <= 0:
             return []
         sizes = range(1, min(cap, num_steps) + 1)
@@ -316,6 +319,50 @@ class HostStepPipeline:
         # nothing is in flight: every round's buffers are free
         for e in self._comp + self._down:
             e.record(cur)
+
+    def graph(self, order):
+        """One CUDA graph of the rounds ``order`` lists, enqueued as ``run_order``
+        enqueues them: uploads on one side stream, kernels on the capturing stream,
+        downloads on another, joined by events inside the graph. Replaying it costs
+        one launch from the host, however short the rounds (``run_order`` needs a few
+        host calls per round, which can take longer than a short round's kernels).
+        The rounds' per-phase graphs need not have been captured; run each step once
+        before (e.g. ``capture`` or ``run_order``) so that every launch path is warm."""
+        cur = torch.cuda.current_stream()
+        cs, s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        comp, down = {}, {}
+        cs.wait_stream(cur)
+        with torch.cuda.graph(g, stream=cs):
+            s_in.wait_stream(cs)
+            s_out.wait_stream(cs)
+            for x in order:
+                r = self.rounds[x]
+                if x in comp:  # this set's buffers: free once its previous kernels ran
+                    s_in.wait_event(comp[x])
+                with torch.cuda.stream(s_in):
+                    for h in r:
+                        h.upload()
+                up = torch.cuda.Event()
+                up.record(s_in)
+                cs.wait_event(up)
+                if x in down:  # and once its previous outputs were read back
+                    cs.wait_event(down[x])
+                for h in r:
+                    h.step.run()
+                comp[x] = torch.cuda.Event()
+                comp[x].record(cs)
+                s_out.wait_event(comp[x])
+                with torch.cuda.stream(s_out):
+                    for h in r:
+                        h.download()
+                down[x] = torch.cuda.Event()
+                down[x].record(s_out)
+            cs.wait_stream(s_in)
+            cs.wait_stream(s_out)
+        cur.wait_stream(cs)
+        torch.cuda.synchronize()
+        return g
 
     def run(self, n_rounds: int):
         """Enqueue ``n_rounds`` rounds (the sets in turn) on the current stream and

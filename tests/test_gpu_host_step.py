@@ -126,3 +126,36 @@ def test_host_step_pipeline(overlapped):
     assert abi.pa_device_status() == 0
     kp, vp = oracle_pools(b2)
     assert_close(widen_out(ref[1]), oracle_decode(b2, kp, vp), b2.dtype, "pipeline")
+
+
+@pytest.mark.parametrize("order", [[0, 1, 2], [0, 1, 0, 1, 2]])
+def test_host_step_pipeline_as_one_graph(order):
+    """Rounds of different sizes (1, 3 and 2 steps) captured as one graph with the
+    three streams inside it, sets reused within the pass: every step's output has
+    the bits of the device-resident step, after every replay."""
+    b1 = synth.small_random(65, 5, [1, 64, 300, 1000, 17], 32, 8, 128, 16, 400, "bf16")
+    b2 = synth.small_random(66, 5, [5, 129, 2, 700, 256], 32, 8, 128, 16, 400, "bf16")
+    g1 = GpuBatch(b1, fused=True)
+    g2 = GpuBatch(b2, fused=True)
+    ref = [g1.run().clone().cpu(), g2.run().clone().cpu()]
+    gs = [g1, g2]
+    sizes = [1, 3, 2]
+    rounds, k = [], 0
+    for n in sizes:
+        rounds.append([_host_step(gs[(k + i) % 2].step, True) for i in range(n)])
+        k += n
+    pipe = HostStepPipeline(rounds)
+    pipe.capture()
+    graph = pipe.graph(order)
+    for _ in range(3):
+        for r in rounds:
+            for h in r:
+                h.h_out.fill_(0)
+        graph.replay()
+        torch.cuda.synchronize()
+        k = 0
+        for r in rounds:
+            for i, h in enumerate(r):
+                assert torch.equal(h.h_out.view(torch.int16), ref[(k + i) % 2].view(torch.int16))
+            k += len(r)
+    assert abi.pa_device_status() == 0
