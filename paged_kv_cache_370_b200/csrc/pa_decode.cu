@@ -57,6 +57,10 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kStages = 4;
 constexpr int kTileBytes = 8192;                 // bytes of K (and of V) per stage
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+// how long the decode consumers wait for the producer's word on the piece it may
+// fetch before their final merge (it comes one counter read after the producer's
+// last copies are issued); then they go ahead without it
+constexpr unsigned long long kPreWaitNs = 20000ull;  // 20 us
 
 // Wait for phase `parity` of `bar` to complete, at most limit_ns; also give up
 // when another thread of the CTA has raised *abort. Returns false on give-up
@@ -611,24 +615,41 @@ struct Cfg {
   static constexpr int kBarOffset = kMetaOffset + kStages * (int)sizeof(TileMeta);
   static constexpr int kMlOffset = kBarOffset + 2 * kStages * 8;  // full, empty barriers
   static constexpr int kIdsOffset = kMlOffset + kWarps * 8 * 2 * 4;
-  static constexpr int kCtrlOffset = kIdsOffset + 2 * kIdWindow * 8 * 4;  // one window per producer
-  // after the control words (W, x0, x1, abort, last): the metadata barriers
-  static constexpr int kMetaBarOffset = kCtrlOffset + 32;
-  static_assert(kStages * 8 <= 32, "metadata barriers fit the control area");
-  static constexpr int kBytes = 1024 + kCtrlOffset + 64;  // + slack to align the ring to 1 KB
   // CTAs per SM the register budget is sized for
   static constexpr int kMinCtas = D == 64 ? 3 : (G <= 4 ? 2 : 1);
+  // one split piece of another CTA (G heads of acc[D], max, sum, pad), fetched ahead
+  // of this CTA's final merge -- where kMinCtas CTAs still fit the SM's 228 KB
+  static constexpr int kPreOffset = (kIdsOffset + 2 * kIdWindow * 8 * 4 + 15) & ~15;
+  static constexpr int kPieceBytes = G * (D + 4) * 4;
+  static constexpr int kCtrlBytes = 80;
+  static constexpr bool kPreFits =
+      (1024 + kPreOffset + kPieceBytes + kCtrlBytes + 1024) * kMinCtas <= 228 * 1024;
+  static constexpr int kPreBytes = kPreFits ? kPieceBytes : 0;
+  static constexpr int kCtrlOffset = kPreOffset + kPreBytes;
+  // after the control words (W, x0, x1, abort, last): the metadata barriers, then
+  // the hand-off word of the fetched piece
+  static constexpr int kMetaBarOffset = kCtrlOffset + 32;
+  static_assert(kStages * 8 <= 32, "metadata barriers fit the control area");
+  static constexpr int kPreStateOffset = kCtrlOffset + 64;
+  static constexpr int kBytes = 1024 + kCtrlOffset + kCtrlBytes;  // + slack to align the ring to 1 KB
 };
 
 // The CTA owning global tile x when W tiles are split evenly over n CTAs
-// (CTA c owns [c*W/n, (c+1)*W/n)).
+// (CTA c owns [c*W/n, (c+1)*W/n)): the c with c*W < (x+1)*n <= (c+1)*W. An fp32
+// quotient is within one of it and two 64-bit products settle it (a 64-bit integer
+// division costs hundreds of cycles, and the flushes run these for every thread).
 __device__ __forceinline__ int owner_cta(long long x, long long W, int n) {
-  return (int)(((x + 1) * n - 1) / W);
+  const long long v = (x + 1) * n;
+  int c = (int)((float)v / (float)W);
+  while (c > 0 && (long long)c * W >= v) --c;
+  while ((long long)(c + 1) * W < v) ++c;
+  return c;
 }
 
-// Whether CTA c owns any tile (with more CTAs than tiles some own none).
+// Whether CTA c owns any tile (with more CTAs than tiles some own none; with at
+// least as many tiles as CTAs every CTA owns floor(W/n) or more).
 __device__ __forceinline__ bool cta_has_tiles(int c, long long W, int n) {
-  return (long long)c * W / n < (long long)(c + 1) * W / n;
+  return W >= n || (long long)c * W / n < (long long)(c + 1) * W / n;
 }
 
 __device__ __forceinline__ int clamp_len(int len, int cap, int max_len, bool &bad) {
@@ -675,6 +696,12 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
   long long *ctrl = reinterpret_cast<long long *>(smem + C::kCtrlOffset);  // W, x0, x1
   volatile int *abort_flag = reinterpret_cast<volatile int *>(ctrl + 3);
   volatile int *last_flag = abort_flag + 1;
+  // the piece fetched ahead of the final merge: pre_state 0 = open, 1 = the producer
+  // has issued its copy into pre_piece (landing on pre_bar), 2 = the consumers went
+  // ahead without it (whichever sets it first from 0 wins)
+  int *pre_state = reinterpret_cast<int *>(smem + C::kPreStateOffset);
+  uint64_t *pre_bar = reinterpret_cast<uint64_t *>(smem + C::kPreStateOffset + 8);
+  const float *pre_piece = reinterpret_cast<const float *>(smem + C::kPreOffset);
   const uint32_t ring = smem_u32(smem);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -709,6 +736,8 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       mbar_init(&meta_bar[s], 1);
     }
     *abort_flag = 0;
+    *pre_state = 0;
+    mbar_init(pre_bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -809,6 +838,14 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // the copies of the last NS tiles this warp issued (bit k: tile ntiles - NS + k)
     uint32_t issued_mask = 0;
+    // The segment this CTA ends in may start here and go on in the next CTAs, which
+    // make its other pieces at the start of theirs. With exactly one other piece, the
+    // K producer, once its last copies are issued (the consumers still have the
+    // tiles in the ring to go), checks the segment's counter and, if that piece is
+    // out, copies it into shared memory: the final merge then reads no global
+    // memory. (pre_cta: the CTA of that piece)
+    int pre_cta = -1;
+    bool pre_issued = false;
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % NS;
       // stage free? The consumers arrive once per tile whatever happened; after a
@@ -832,6 +869,16 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       const bool seg_begin = (j == 0) || (i == 0);
       const bool seg_end = (j == tb - 1) || (i == ntiles - 1);
       const bool new_tok = fused && j == tb - 1 && len_b > 0;  // tile of position len - 1
+      if (C::kPreBytes > 0 && !v_producer && j == 0 && x0 + i + tb > x1 && !p.starve) {
+        const int cb = owner_cta(x0 + i + tb - 1, W, nctas);
+        int n_other = 0, c_other = -1;
+        for (int cc = cta + 1; cc <= cb && n_other < 2; ++cc)
+          if (cta_has_tiles(cc, W, nctas)) {
+            ++n_other;
+            c_other = cc;
+          }
+        if (n_other == 1) pre_cta = c_other;
+      }
       const bool ok = lane < tile_boxes(j, len_b) && phys >= 0 && phys < p.num_blocks;
       if (lane < tile_boxes(j, len_b) && !ok && !v_producer)
         atomicOr(&g_decode_error, PA_DEVERR_BLOCK_ID);
@@ -906,6 +953,27 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         if (i + kIdWindow + 1 < ntiles) advance_ahead();
       } else {
         cp_async_commit();
+      }
+    }
+    if (pre_cta >= 0) {
+      // the counter counts the other pieces out; only this CTA's merge resets it
+      const bool out = ld_acquire_gpu(p.ws_counters + cta) == 1;
+      if (lane == 0 && atomicCAS(pre_state, 0, out ? 1 : 3) == 0 && out) {
+        pre_issued = true;
+        asm volatile("fence.proxy.async.global;" ::: "memory");  // the copy reads what was acquired
+        mbar_expect_tx_arrive(pre_bar, (uint32_t)C::kPreBytes);
+        bulk_g2s(smem + C::kPreOffset, p.ws_pieces + (size_t)(2 * pre_cta) * G * kPieceStride,
+                 (uint32_t)C::kPreBytes, pre_bar);
+      }
+    }
+    // the piece's copy, like the tiles', lands before the CTA exits
+    if (pre_issued && lane == 0) {
+      const unsigned long long t_start = global_ns();
+      while (!mbar_try_wait(pre_bar, 0)) {
+        if (global_ns() - t_start > kWaitLimitNs) {
+          atomicOr(&g_decode_error, PA_DEVERR_TIMEOUT);
+          break;
+        }
       }
     }
     // do not leave while copies may still land in this CTA's shared memory
@@ -1132,14 +1200,28 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     // already: if the counter says so, it merges at once from its own values and
     // theirs, without writing its piece, fencing or counting (same order and
     // arithmetic as the merge below, so the same bits)
+    // (from shared memory when the producer has fetched the other piece already)
     if (!whole && ca == cta && tid == 0) {
       int pieces = 0;
       for (int cc = ca; cc <= cb; ++cc) pieces += cta_has_tiles(cc, W, nctas) ? 1 : 0;
-      *last_flag = ld_acquire_gpu(p.ws_counters + ca) == pieces - 1 ? 2 : 0;
+      int flag = 0;
+      if (C::kPreBytes > 0 && pieces == 2 && !p.starve) {
+        // the producer decides one counter read after its last issue: wait for
+        // that (briefly), then take the piece from shared memory if it copied it
+        const unsigned long long t_start = global_ns();
+        while (*reinterpret_cast<volatile int *>(pre_state) == 0 && !*abort_flag &&
+               global_ns() - t_start < kPreWaitNs) {
+        }
+        if (atomicCAS(pre_state, 0, 2) == 1 && mbar_wait_bounded(pre_bar, 0, abort_flag))
+          flag = 3;
+      }
+      if (flag == 0) flag = ld_acquire_gpu(p.ws_counters + ca) == pieces - 1 ? 2 : 0;
+      *last_flag = flag;
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kWarps * 32) : "memory");
-    const bool merge_now = !whole && ca == cta && *last_flag == 2;
-    if (merge_now) __threadfence();
+    const bool from_smem = !whole && ca == cta && *last_flag == 3;
+    const bool merge_now = !whole && ca == cta && (*last_flag == 2 || from_smem);
+    if (merge_now && !from_smem) __threadfence();
     for (int e0 = tid * 4; e0 < G * D; e0 += kWarps * 32 * 4) {
       const int h = e0 / D, d = e0 % D;
       float M = -INFINITY;
@@ -1163,10 +1245,19 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
             Elem<T>::from_f32x4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
       } else if (merge_now) {
         // this CTA's piece (M, L, sum) first, then the others' in CTA order
+        auto piece = [&](int cc) {
+          return from_smem ? pre_piece + h * kPieceStride
+                           : p.ws_pieces + ((size_t)(2 * cc) * G + h) * kPieceStride;
+        };
+        auto rd = [&](const float *a) { return from_smem ? *a : __ldcg(a); };
+        auto rd4 = [&](const float *a) {
+          return from_smem ? *reinterpret_cast<const float4 *>(a)
+                           : __ldcg(reinterpret_cast<const float4 *>(a));
+        };
         float Mm = M;
         for (int cc = ca + 1; cc <= cb; ++cc) {
           if (!cta_has_tiles(cc, W, nctas)) continue;
-          Mm = fmaxf(Mm, __ldcg(p.ws_pieces + ((size_t)(2 * cc) * G + h) * kPieceStride + D));
+          Mm = fmaxf(Mm, rd(piece(cc) + D));
         }
         float Lm = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1180,12 +1271,12 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         }
         for (int cc = ca + 1; cc <= cb; ++cc) {
           if (!cta_has_tiles(cc, W, nctas)) continue;
-          const float *pc = p.ws_pieces + ((size_t)(2 * cc) * G + h) * kPieceStride;
-          const float mc = __ldcg(pc + D);
+          const float *pc = piece(cc);
+          const float mc = rd(pc + D);
           if (mc == -INFINITY) continue;
           const float w = exp2f(mc - Mm);
-          Lm += w * __ldcg(pc + D + 1);
-          const float4 v = __ldcg(reinterpret_cast<const float4 *>(pc + d));
+          Lm += w * rd(pc + D + 1);
+          const float4 v = rd4(pc + d);
           acc.x += w * v.x;
           acc.y += w * v.y;
           acc.z += w * v.z;
