@@ -586,6 +586,7 @@ constexpr int kWarps = 4;            // consumer warps, 16 tokens each
 constexpr int kThreads = (kWarps + 2) * 32;
 constexpr int kPanelBytes = kTile * 128;  // 64 columns of 2 bytes x 64 rows
 constexpr int kIdWindow = 8;             // tiles of block ids fetched ahead of their copies
+constexpr int kScanLoads = 8;            // lengths per lane loaded at once when sizing the job
 
 // Per-tile schedule handed from the producer warp to the consumers with the tile.
 struct TileMeta {
@@ -709,15 +710,23 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
   const int Hkv = p.num_kv_heads, B = p.num_seqs, bs = p.block_size;
   const int cap = p.max_blocks_per_seq * bs;
 
-  // ---- size the whole job (every CTA does the same scan) and take an even share
+  // ---- size the whole job (every CTA does the same scan) and take an even share;
+  // the lengths of up to 32 * kScanLoads sequences are loaded per round trip
   if (warp == kWarps) {
     long long W = 0;
     bool bad = false;
-    for (int base = 0; base < B; base += 32) {
+    for (int base = 0; base < B; base += 32 * kScanLoads) {
+      int len[kScanLoads];
+#pragma unroll
+      for (int k = 0; k < kScanLoads; ++k) {
+        const int bb = base + 32 * k + lane;
+        len[k] = bb < B ? __ldg(p.context_lens + bb) : 0;
+      }
       int tiles = 0;
-      if (base + lane < B)
-        tiles = Hkv * seg_tiles(clamp_len(__ldg(p.context_lens + base + lane), cap,
-                                          p.max_context_len, bad));
+#pragma unroll
+      for (int k = 0; k < kScanLoads; ++k)
+        if (base + 32 * k + lane < B)
+          tiles += Hkv * seg_tiles(clamp_len(len[k], cap, p.max_context_len, bad));
       for (int off = 16; off >= 1; off >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, off);
       W += tiles;
     }
@@ -780,8 +789,8 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     long long slot_b = fused ? __ldg(p.new_slots + b) : -1;
     long long slot_next = fused && b + 1 < B ? __ldg(p.new_slots + b + 1) : -1;
     int tb = seg_tiles(len_b);
-    int kvh = (int)((x0 - pre) / tb);
-    int j = (int)((x0 - pre) % tb);
+    int kvh = (int)(x0 - pre) / tb;  // (x0 - pre < Hkv * tb: 32-bit division)
+    int j = (int)(x0 - pre) % tb;
     const int box_rows = bs < kTile ? bs : kTile;
     const uint32_t box_bytes = 2u * C::kPanels * box_rows * 128u;
     const int32_t *tables = p.block_tables;
