@@ -449,6 +449,40 @@ def test_tail_overread_bytes():
     assert tail_overread_bytes([0, 16], 8, 128, 16) == 0
 
 
+def _split_pieces_walk(lens, hkv, n, tile=64):
+    """Pieces of split segments, found by walking every tile in order with CTA c
+    owning tiles [floor(c W / n), floor((c + 1) W / n))."""
+    tiles = [max(1, -(-int(l) // tile)) for l in lens for _ in range(hkv)]
+    W = sum(tiles)
+    starts = [c * W // n for c in range(n + 1)]
+    c, x, pieces = 0, 0, 0
+    for t in tiles:
+        owners = set()
+        for _ in range(t):
+            while x >= starts[c + 1]:
+                c += 1
+            owners.add(c)
+            x += 1
+        pieces += len(owners) if len(owners) > 1 else 0
+    return pieces
+
+
+def test_split_scratch_bytes_counts_the_pieces():
+    from paged_kv_cache_370_b200.accounting import stream_split_scratch_bytes
+    per_piece = 2 * 4 * (128 + 2) * 4 + 8
+    # one 10-tile segment over 2 CTAs: 5 tiles each, two pieces
+    assert stream_split_scratch_bytes([640], 1, 4, 128, 2) == 2 * per_piece
+    # two 1-tile segments over 2 CTAs: nothing is split
+    assert stream_split_scratch_bytes([64, 64], 1, 4, 128, 2) == 0
+    rng = np.random.default_rng(7)
+    for _ in range(60):
+        b = int(rng.integers(1, 40))
+        lens = rng.integers(0, 3000, size=b)
+        hkv, n = int(rng.choice([1, 2, 8])), int(rng.choice([1, 3, 16, 148, 296, 1000]))
+        assert stream_split_scratch_bytes(lens, hkv, 4, 128, n) == \
+            _split_pieces_walk(lens, hkv, n) * per_piece
+
+
 def test_slide_window_releases_only_blocks_before_the_window():
     m = BlockManager(16, 4)
     m.add_seq(0, 10)                       # blocks for positions 0-3, 4-7, 8-9
