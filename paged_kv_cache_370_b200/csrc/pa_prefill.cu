@@ -887,17 +887,20 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
             if (kp > pr || kp < lo) sv[c] = __float_as_uint(-INFINITY);
           }
         }
-        // eight independent running maxima, then a tree: a short dependency chain
-        float mx8[8];
+        // four independent running maxima of three inputs each (two keys a step),
+        // then their maximum: 64 instructions for 128 keys, short chains
+        auto sf = [&](int c) { return __uint_as_float(sv[c]); };
+        float mxa = sf(0), mxb = sf(1), mxc = sf(2), mxd = sf(3);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sv[e]);
-#pragma unroll
-        for (int c = 8; c < kN; ++c) mx8[c % 8] = fmaxf(mx8[c % 8], __uint_as_float(sv[c]));
-#pragma unroll
-        for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-          for (int e = 0; e < w; ++e) mx8[e] = fmaxf(mx8[e], mx8[e + w]);
-        const float mx = mx8[0] * p.scale_log2;  // log2 domain
+        for (int c = 4; c + 8 <= kN - 4; c += 8) {
+          mxa = fmax3f(mxa, sf(c), sf(c + 1));
+          mxb = fmax3f(mxb, sf(c + 2), sf(c + 3));
+          mxc = fmax3f(mxc, sf(c + 4), sf(c + 5));
+          mxd = fmax3f(mxd, sf(c + 6), sf(c + 7));
+        }
+        mxa = fmax3f(mxa, sf(kN - 4), sf(kN - 3));
+        mxb = fmax3f(mxb, sf(kN - 2), sf(kN - 1));
+        const float mx = fmax3f(mxa, mxb, fmaxf(mxc, mxd)) * p.scale_log2;  // log2 domain
         // move the reference max when it grew past the lazy bound; O and l are
         // rescaled below, once this tile's scores are no longer held in registers
         const bool grow =
@@ -906,26 +909,28 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         const float alpha = grow && m_ref > -INFINITY ? exp2f(m_ref - mx) : 1.f;
         if (grow) m_ref = mx;
         const float nbase = m_ref == -INFINITY ? 0.f : -m_ref;
-        // this tile's P row, weight = 2^(s * scale_log2 - m_ref) (one FMA and one
-        // exp2 per key), packed two per column over the first half of its S row, in
-        // halves of 64 keys (each half's 32 columns stored at once); l sums the same
-        // rounded weights the product uses, in four partial sums
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+        // this tile's P row, weight = 2^(s * scale_log2 - m_ref) (one FMA per key, two
+        // keys per instruction, and one exp2 per key), packed two per column over the
+        // first half of its S row, in halves of 64 keys (each half's 32 columns stored
+        // at once); l sums the same rounded weights the product uses, in four partial
+        // sums (packed adds there cost more registers than they save instructions)
+        const uint64_t scale2 = f32x2(p.scale_log2, p.scale_log2), base2 = f32x2(nbase, nbase);
+        float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c4 = 0; c4 < kN / 64; ++c4) {
           uint32_t pw[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const int kx = c4 * 64 + 2 * c;
-            const float a = ex2_approx(fmaf(__uint_as_float(sv[kx]), p.scale_log2, nbase));
-            const float b2 = ex2_approx(fmaf(__uint_as_float(sv[kx + 1]), p.scale_log2, nbase));
+            float xa, xb;
+            f32x2_split(fma_f32x2(f32x2(sf(kx), sf(kx + 1)), scale2, base2), xa, xb);
             float ra, rb;
-            pw[c] = Mma<T>::pack(a, b2, ra, rb);
-            ls[c % 4] += ra + rb;
+            pw[c] = Mma<T>::pack(ex2_approx(xa), ex2_approx(xb), ra, rb);
+            ls4[c % 4] += ra + rb;
           }
           tmem_st32(trow + c4 * 32, pw);
         }
-        l = l * alpha + ((ls[0] + ls[1]) + (ls[2] + ls[3]));
+        l = l * alpha + ((ls4[0] + ls4[1]) + (ls4[2] + ls4[3]));
         // O against the new reference max (warp-uniform TMEM traffic: lanes that keep
         // theirs scale by 1), before this tile's P V is issued. S was issued after
         // the group's previous P V and the tensor core runs in order, so O holds it.
