@@ -913,7 +913,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         // keys per instruction, and one exp2 per key), packed two per column over the
         // first half of its S row, in halves of 64 keys (each half's 32 columns stored
         // at once); l sums the same rounded weights the product uses, in four partial
-        // sums (packed adds there cost more registers than they save instructions)
+        // sums, each 16-bit weight added as it is (mixed-precision add)
         const uint64_t scale2 = f32x2(p.scale_log2, p.scale_log2), base2 = f32x2(nbase, nbase);
         float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -926,7 +926,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
             f32x2_split(fma_f32x2(f32x2(sf(kx), sf(kx + 1)), scale2, base2), xa, xb);
             float ra, rb;
             pw[c] = Mma<T>::pack(ex2_approx(xa), ex2_approx(xb), ra, rb);
-            ls4[c % 4] += ra + rb;
+            Mma<T>::add_halves(ls4[c % 4], pw[c]);
           }
           tmem_st32(trow + c4 * 32, pw);
         }

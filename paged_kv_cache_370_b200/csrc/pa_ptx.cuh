@@ -203,6 +203,14 @@ struct Mma<__nv_bfloat16> {
     rhi = __high2float(v);
     return *reinterpret_cast<uint32_t *>(&v);
   }
+  // acc += low half, then += high half of a packed pair (each half widened exactly;
+  // sm_100's mixed-precision add, one instruction per half)
+  static __device__ __forceinline__ void add_halves(float &acc, uint32_t pair) {
+    unsigned short lo, hi;
+    asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(pair));
+    asm("add.rn.f32.bf16 %0, %1, %0;" : "+f"(acc) : "h"(lo));
+    asm("add.rn.f32.bf16 %0, %1, %0;" : "+f"(acc) : "h"(hi));
+  }
 };
 
 template <>
@@ -220,6 +228,12 @@ struct Mma<__half> {
     rlo = __low2float(v);
     rhi = __high2float(v);
     return *reinterpret_cast<uint32_t *>(&v);
+  }
+  static __device__ __forceinline__ void add_halves(float &acc, uint32_t pair) {
+    unsigned short lo, hi;
+    asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(pair));
+    asm("add.rn.f32.f16 %0, %1, %0;" : "+f"(acc) : "h"(lo));
+    asm("add.rn.f32.f16 %0, %1, %0;" : "+f"(acc) : "h"(hi));
   }
 };
 
