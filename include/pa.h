@@ -258,16 +258,17 @@ pa_status pa_decode_append(void *out, const void *q, const void *k_new, const vo
  * range are never read, so they may hold anything -- e.g. the -1 that
  * pa_alloc_slide_window leaves. Arguments as pa_decode / pa_decode_append plus
  * `window` (> 0; PA_ERR_INVALID otherwise); pa_decode_workspace_size covers it.
- * Where pa_decode runs its even-split kernel and block_size <= 64, a small
- * kernel first rewrites, into the workspace, each sequence as the part of it
- * from the block holding its first attended position on (table shifted by that
- * many blocks, length shorter by as many positions, and the count of that
- * block's positions before the window); the even-split kernel then runs on
- * those and masks the counted positions. pa_decode_append_window writes the
- * new tokens inside that kernel, as pa_decode_append does. Otherwise a window
- * runs in the partition kernel (partitions of the window's positions, then the
- * merge kernel when the longest context has more than one), and
- * pa_decode_append_window writes the new tokens with pa_reshape_and_cache
+ * Where pa_decode runs its even-split kernel and block_size <= 64, that kernel
+ * (one launch) sees each sequence as the part of it from the block holding its
+ * first attended position on -- its table read that many blocks further on, its
+ * length shorter by as many positions -- and masks that block's positions
+ * before the window. pa_decode_append_window writes the new tokens inside that
+ * kernel, as pa_decode_append does; pa_decode_append_window_overlapped is the
+ * same call with the programmatic early start and contract of
+ * pa_decode_append_overlapped (on any other shape it is pa_decode_append_window).
+ * Otherwise a window runs in the partition kernel (partitions of the window's
+ * positions, then the merge kernel when the longest context has more than one),
+ * and pa_decode_append_window writes the new tokens with pa_reshape_and_cache
  * first. pa_decode_window_launches and pa_decode_append_window_launches give
  * the kernels each call launches.
  * ------------------------------------------------------------------------------------------ */
@@ -292,6 +293,12 @@ pa_status pa_decode_append_window(void *out, const void *q, const void *k_new, c
                                   int num_blocks, float scale, int window, pa_dtype dtype,
                                   void *workspace, size_t workspace_bytes, int partition_tokens,
                                   void *stream);
+pa_status pa_decode_append_window_overlapped(
+    void *out, const void *q, const void *k_new, const void *v_new, const int64_t *slot_mapping,
+    void *k_cache, void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+    const int32_t *context_lens, int max_context_len, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale, int window,
+    pa_dtype dtype, void *workspace, size_t workspace_bytes, int partition_tokens, void *stream);
 
 /* ------------------------------------------------------------------------------------------
  * pa_prefill -- paged attention for several query tokens per sequence (a prompt, or one

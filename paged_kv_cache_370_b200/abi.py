@@ -71,6 +71,8 @@ def _load() -> ctypes.CDLL:
         "pa_prefill": (i, [P, P, P, P, P, i, P, P, i, i, i, i, i, i, i, i, i, f, i, i, P]),
         "pa_decode_append_window": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i,
                                         P, sz, i, P]),
+        "pa_decode_append_window_overlapped": (i, [P, P, P, P, P, P, P, P, i, P, i, i, i, i, i, i,
+                                                   i, f, i, i, P, sz, i, P]),
         "pa_decode_static_workspace": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P]),
         "pa_device_status": (i, [P, P]),
         "pa_status_string": (ctypes.c_char_p, [i]),
@@ -312,12 +314,15 @@ def pa_decode_append_window_launches(num_seqs, num_q_heads, num_kv_heads, head_d
 
 def pa_decode_append_window(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,
                             context_lens, max_context_len, scale, window, workspace=None,
-                            partition_tokens=0, stream=None):
-    """pa_decode_append over each sequence's last ``window`` positions only."""
+                            partition_tokens=0, stream=None, overlapped=False):
+    """pa_decode_append over each sequence's last ``window`` positions only
+    (``overlapped``: pa_decode_append_window_overlapped, the programmatic early
+    start of pa_decode_append_overlapped, under the same contract)."""
     B, hq, d = q.shape
     nb, hkv, bs, _ = k_cache.shape
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = _lib.pa_decode_append_window(
+    fn = _lib.pa_decode_append_window_overlapped if overlapped else _lib.pa_decode_append_window
+    st = fn(
         _dev_ptr(out, "out"), _dev_ptr(q, "q"), _dev_ptr(k_new, "k_new"), _dev_ptr(v_new, "v_new"),
         _dev_ptr(slot_mapping, "slot_mapping"), _dev_ptr(k_cache, "k_cache"),
         _dev_ptr(v_cache, "v_cache"), _dev_ptr(block_tables, "block_tables"),

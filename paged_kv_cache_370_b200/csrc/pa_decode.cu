@@ -160,11 +160,9 @@ struct DecodeParams {
   void *v_cache_w;
   // sliding window: a sequence of length len attends to positions
   // [len - window, len) (0: every position). The partition kernel applies it
-  // directly; the even-split kernel sees each sequence from the block holding
-  // its first attended position on (window_remap_kernel) and masks the
-  // win_skip[b] positions of that block before the window (nullptr: none)
+  // directly; the even-split kernel (its kWindow instantiation) sees each
+  // sequence from the block holding its first attended position on (seq_view)
   int window;
-  const int32_t *win_skip;
   // even-split kernel launched as a programmatic dependent of the preceding kernel
   int early_start;
   // limit of the consumers' waits for a stage's data (normally kWaitLimitNs)
@@ -661,6 +659,32 @@ __device__ __forceinline__ int clamp_len(int len, int cap, int max_len, bool &ba
   return len;
 }
 
+// How the even-split kernel sees sequence b. With kWindow (a sliding window of
+// `window` positions), from the block holding its first attended position on:
+// its length shorter by `shift` whole blocks, its table read `shift` entries
+// further on, and the `skip` positions of that first block that precede the
+// window masked (skip < block_size <= 64: they lie in the first tile). Every place
+// that counts tiles or reads the table takes lengths from here, so the CTA ranges,
+// the producers' walks and the merges' owner arithmetic agree.
+struct SeqView {
+  int len, shift, skip;
+};
+template <bool kWindow>
+__device__ __forceinline__ SeqView seq_view(int raw_len, int cap, int max_len, int window, int bs,
+                                            bool &bad) {
+  SeqView v;
+  v.len = clamp_len(raw_len, cap, max_len, bad);
+  v.shift = 0;
+  v.skip = 0;
+  if (kWindow) {
+    const int lo = window_lo(v.len, window);
+    v.shift = lo / bs;
+    v.skip = lo - v.shift * bs;
+    v.len -= v.shift * bs;
+  }
+  return v;
+}
+
 // tiles of one (sequence, kv head) segment; an empty sequence still gets one
 // (empty) tile so that its output is written (zeros)
 // floats per stored piece of one head: acc[D], max, sum and padding that keeps
@@ -670,9 +694,10 @@ __host__ __device__ constexpr int piece_stride() { return D + 4; }
 
 __device__ __forceinline__ int seg_tiles(int len) { return len > 0 ? (len + kTile - 1) / kTile : 1; }
 
-// kWindow: the sequences come from window_remap_kernel and the first tile of
-// each may start with positions before the window (a separate instantiation,
-// so that plain decode carries none of the masking)
+// kWindow: a sliding window of p.window positions; every sequence is seen from
+// the block holding its first attended position on (seq_view), and the first
+// tile of each may start with positions before the window, which are masked (a
+// separate instantiation, so that plain decode carries none of it)
 template <typename T, int D, int G, bool kWindow>
 __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     pa_decode_stream_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -726,7 +751,8 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
 #pragma unroll
       for (int k = 0; k < kScanLoads; ++k)
         if (base + 32 * k + lane < B)
-          tiles += Hkv * seg_tiles(clamp_len(len[k], cap, p.max_context_len, bad));
+          tiles += Hkv * seg_tiles(
+                             seq_view<kWindow>(len[k], cap, p.max_context_len, p.window, bs, bad).len);
       for (int off = 16; off >= 1; off >>= 1) tiles += __shfl_xor_sync(0xffffffffu, tiles, off);
       W += tiles;
     }
@@ -764,8 +790,9 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     for (int base = 0; base < B; base += 32) {
       int tiles = 0;
       if (base + lane < B)
-        tiles = Hkv * seg_tiles(clamp_len(__ldg(p.context_lens + base + lane), cap,
-                                          p.max_context_len, bad));
+        tiles = Hkv * seg_tiles(seq_view<kWindow>(__ldg(p.context_lens + base + lane), cap,
+                                                  p.max_context_len, p.window, bs, bad)
+                                    .len);
       int incl = tiles;
       for (int off = 1; off < 32; off <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, incl, off);
@@ -782,7 +809,9 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
       }
       pre += total;
     }
-    int len_b = clamp_len(__ldg(p.context_lens + b), cap, p.max_context_len, bad);
+    SeqView view_b =
+        seq_view<kWindow>(__ldg(p.context_lens + b), cap, p.max_context_len, p.window, bs, bad);
+    int len_b = view_b.len, skip_b = view_b.skip;
     // the next sequence's length, loaded ahead of need
     int len_next = b + 1 < B ? __ldg(p.context_lens + b + 1) : 0;
     const bool fused = p.new_slots != nullptr;
@@ -806,11 +835,12 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
     // out of L2 (the K/V stream evicts them), so each id load costs a full HBM
     // round trip that must overlap the copies of the tiles before it.
     const uint32_t ids = smem_u32(smem + C::kIdsOffset) + (v_producer ? kIdWindow * 8 * 4 : 0);
-    int ab = b, akvh = kvh, aj = j, alen = len_b, atb = tb;  // cursor of the tile being fetched
+    // cursor of the tile being fetched (ashift: its sequence's table shift)
+    int ab = b, akvh = kvh, aj = j, alen = len_b, atb = tb, ashift = view_b.shift;
     auto fetch_ids = [&](int slot) {
       if (lane < tile_boxes(aj, alen))
         cp_async_4(ids + (slot * 8 + lane) * 4,
-                   tables + (size_t)ab * p.max_blocks_per_seq + (aj * kTile) / bs + lane);
+                   tables + (size_t)ab * p.max_blocks_per_seq + ashift + (aj * kTile) / bs + lane);
       cp_async_commit();
     };
     auto advance_ahead = [&]() {
@@ -819,7 +849,10 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         if (++akvh == Hkv) {
           akvh = 0;
           if (++ab < B) {
-            alen = clamp_len(__ldg(p.context_lens + ab), cap, p.max_context_len, bad);
+            const SeqView v = seq_view<kWindow>(__ldg(p.context_lens + ab), cap,
+                                                p.max_context_len, p.window, bs, bad);
+            alen = v.len;
+            ashift = v.shift;
             atb = seg_tiles(alen);
           }
         }
@@ -905,7 +938,7 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
         m.nvalid = nvalid;
         m.seg_first_x = (int)(x0 + i - j);
         m.flags = (seg_begin ? 1 : 0) | (seg_end ? 2 : 0) | (new_tok ? 4 : 0);
-        m.nskip = (kWindow && j == 0) ? min(max(__ldg(p.win_skip + b), 0), kTile - 1) : 0;
+        m.nskip = (kWindow && j == 0) ? min(skip_b, kTile - 1) : 0;
         m.new_slot = slot_b;
         if (issue)
           mbar_expect_tx_arrive(&full_bar[s], __popc(okmask) * box_bytes +
@@ -948,7 +981,10 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
           if (++kvh == Hkv) {
             kvh = 0;
             ++b;
-            len_b = clamp_len(len_next, cap, p.max_context_len, bad);
+            const SeqView v =
+                seq_view<kWindow>(len_next, cap, p.max_context_len, p.window, bs, bad);
+            len_b = v.len;
+            skip_b = v.skip;
             tb = seg_tiles(len_b);
             len_next = b + 1 < B ? __ldg(p.context_lens + b + 1) : 0;
             slot_b = slot_next;
@@ -1382,33 +1418,6 @@ __global__ void __launch_bounds__(D) pa_decode_merge_kernel(
   out[hq * D + d] = Elem<T>::from_f32(acc / Ls);
 }
 
-// ------------------------------------------------------------------- sliding-window remap
-// A sliding window on the even-split kernel: sequence b is handed over from
-// the block holding its first attended position on -- its table shifted by
-// that many blocks (vtab, vwidth entries per row) and its length shorter by as
-// many positions (vlen) -- with vskip[b] = the positions at the start of that
-// block that precede the window, which the kernel masks. With block_size <= 64
-// they all lie in the sequence's first tile. A length outside [0, max_len] or
-// beyond its table becomes -1, which the kernel reports as a bad length.
-__global__ void __launch_bounds__(128) window_remap_kernel(
-    const int32_t *__restrict__ tables, int width, const int32_t *__restrict__ lens, int bs,
-    int window, int max_len, int vwidth, int32_t *__restrict__ vtab,
-    int32_t *__restrict__ vlen, int32_t *__restrict__ vskip) {
-  const int b = blockIdx.x;
-  const int len = __ldg(lens + b);
-  const bool ok = len >= 0 && len <= max_len && (long long)len <= (long long)width * bs;
-  const int lo = ok ? window_lo(len, window) : 0;
-  const int shift = lo / bs;
-  if (threadIdx.x == 0) {
-    vlen[b] = ok ? len - shift * bs : -1;
-    vskip[b] = lo - shift * bs;
-  }
-  for (int i = threadIdx.x; i < vwidth; i += blockDim.x) {
-    const int src = i + shift;
-    vtab[(size_t)b * vwidth + i] = src < width ? __ldg(tables + (size_t)b * width + src) : 0;
-  }
-}
-
 }  // namespace
 
 // ================================================================================ host side
@@ -1572,14 +1581,6 @@ bool window_on_stream(int group, int block_size, int num_blocks, int num_kv_head
          block_size <= tc::kTile;
 }
 
-// Workspace after the even-split kernel's pieces for the window remap: the
-// shifted lengths and skips (padded to 16 bytes), then the shifted tables.
-size_t window_remap_bytes(int num_seqs, int max_context_len, int block_size) {
-  const long long vwidth = std::max(1, (max_context_len + block_size - 1) / block_size);
-  const size_t heads = ((size_t)2 * num_seqs * sizeof(int32_t) + 15) / 16 * 16;
-  return heads + (size_t)num_seqs * vwidth * sizeof(int32_t);
-}
-
 size_t stream_workspace(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                         int max_context_len, int partition_tokens) {
   const int group = num_q_heads / num_kv_heads;
@@ -1591,7 +1592,9 @@ size_t stream_workspace(int num_seqs, int num_q_heads, int num_kv_heads, int hea
 template <typename T, int D, int G>
 pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dtype dtype,
                         cudaStream_t stream) {
-  if (prm.window == 0 && uses_stream_kernel(G, prm.block_size, prm.num_blocks, prm.num_kv_heads)) {
+  const bool win = prm.window > 0;
+  if (win ? window_on_stream(G, prm.block_size, prm.num_blocks, prm.num_kv_heads)
+          : uses_stream_kernel(G, prm.block_size, prm.num_blocks, prm.num_kv_heads)) {
     using C = tc::Cfg<D, G>;
     static size_t configured[kMaxDevices] = {};
     const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
@@ -1600,7 +1603,6 @@ pa_status launch_decode(const DecodeParams &prm, int num_seqs, void *out, pa_dty
     if (!pool_tensor_map(&tk, prm.k_cache, rows, D, box_rows, dtype) ||
         !pool_tensor_map(&tv, prm.v_cache, rows, D, box_rows, dtype))
       return PA_ERR_CUDA;
-    const bool win = prm.win_skip != nullptr;
     static size_t configured_w[kMaxDevices] = {};
     if (!(win ? ensure_smem(tc::pa_decode_stream_kernel<T, D, G, true>, (size_t)C::kBytes,
                             configured_w)
@@ -1715,13 +1717,11 @@ extern "C" size_t pa_decode_workspace_size(int num_seqs, int num_q_heads, int nu
   const size_t simt = simt_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                      max_context_len, partition_tokens);
   const int group = num_q_heads / num_kv_heads;
-  // (the even-split kernel's pieces, and room for a sliding window's remap at
-  // the smallest block size that kernel takes)
+  // (the even-split kernel's pieces)
   const size_t stream = (group == 2 || group == 4 || group == 8) &&
                                 (head_dim == 64 || head_dim == 128)
                             ? stream_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                               max_context_len, partition_tokens) +
-                                  window_remap_bytes(num_seqs, max_context_len, 8)
+                                               max_context_len, partition_tokens)
                             : 0;
   const size_t body = simt > stream ? simt : stream;
   return body ? kCounterRegion + body : 0;
@@ -1754,7 +1754,7 @@ extern "C" int pa_decode_launches(int num_seqs, int num_q_heads, int num_kv_head
 namespace {
 
 // Workspace one decode call needs (bytes, 0 for none), for the kernel that call
-// runs: the even-split kernel's counters and pieces (+ the window remap), or the
+// runs: the even-split kernel's counters and pieces, or the
 // partition kernel's partial states when the longest context has more than one
 // partition. Arguments already validated.
 size_t decode_need(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
@@ -1769,8 +1769,7 @@ size_t decode_need(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim
   if (streamk) {
     const int nctas = stream_grid(num_seqs, num_kv_heads, group, head_dim, max_context_len,
                                   partition_tokens);
-    return kCounterRegion + (size_t)2 * nctas * group * (head_dim + 4) * sizeof(float) +
-           (wstream ? window_remap_bytes(num_seqs, max_context_len, block_size) : 0);
+    return kCounterRegion + (size_t)2 * nctas * group * (head_dim + 4) * sizeof(float);
   }
   return max_parts > 1 ? kCounterRegion + (size_t)num_seqs * num_q_heads * max_parts *
                                               (head_dim + 2) * sizeof(float)
@@ -1813,8 +1812,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   if (group != 1 && group != 2 && group != 4 && group != 8) return PA_ERR_UNSUPPORTED;
   const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
   const int max_parts = max_context_len > 0 ? (max_context_len + pt - 1) / pt : 1;
-  // a sliding window runs on the even-split kernel after a remap where the
-  // block size allows (window_on_stream), else in the partition kernel
+  // a sliding window runs on the even-split kernel (its kWindow instantiation)
+  // where the block size allows (window_on_stream), else in the partition kernel
   const bool wstream =
       window > 0 && window_on_stream(group, block_size, num_blocks, num_kv_heads);
   const bool streamk = (window == 0 && uses_stream_kernel(group, block_size, num_blocks,
@@ -1823,7 +1822,6 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   const int nctas = streamk ? stream_grid(num_seqs, num_kv_heads, group, head_dim,
                                           max_context_len, partition_tokens)
                             : 0;
-  const size_t pieces_bytes = (size_t)2 * nctas * group * (head_dim + 4) * sizeof(float);
   const size_t need = decode_need(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                   num_blocks, max_context_len, partition_tokens, window);
   if (need > workspace_bytes || (need && (!workspace || !aligned(workspace, 16))))
@@ -1851,7 +1849,6 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   prm.k_cache_w = fw ? fw->k_cache : nullptr;
   prm.v_cache_w = fw ? fw->v_cache : nullptr;
   prm.window = window;
-  prm.win_skip = nullptr;
   prm.early_start = early_start ? 1 : 0;
   prm.starve = g_wait_test.load();
   prm.wait_ns = prm.starve ? (unsigned long long)g_wait_test_ns.load() : kWaitLimitNs;
@@ -1869,26 +1866,6 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
   if ((size_t)prm.table_slice * 4 > 16384) return PA_ERR_UNSUPPORTED;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (wstream) {
-    // each sequence from the block of its first attended position on; the
-    // even-split kernel then runs with no window of its own
-    const int vwidth = std::max(1, (max_context_len + block_size - 1) / block_size);
-    char *base = reinterpret_cast<char *>(ws_body) + pieces_bytes;
-    int32_t *vlen = reinterpret_cast<int32_t *>(base);
-    int32_t *vskip = vlen + num_seqs;
-    int32_t *vtab = reinterpret_cast<int32_t *>(
-        base + ((size_t)2 * num_seqs * sizeof(int32_t) + 15) / 16 * 16);
-    window_remap_kernel<<<num_seqs, 128, 0, st>>>(block_tables, max_blocks_per_seq, context_lens,
-                                                  block_size, window, max_context_len, vwidth,
-                                                  vtab, vlen, vskip);
-    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
-    prm.block_tables = vtab;
-    prm.context_lens = vlen;
-    prm.max_blocks_per_seq = vwidth;
-    prm.win_skip = vskip;
-    prm.window = 0;
-    prm.early_start = 0;  // the remap kernel just wrote the lengths and tables it reads
-  }
   if (dtype == PA_BF16)
     return dispatch_dim<__nv_bfloat16>(head_dim, group, prm, num_seqs, out, dtype, st);
   return dispatch_dim<__half>(head_dim, group, prm, num_seqs, out, dtype, st);
@@ -1930,9 +1907,9 @@ extern "C" int pa_decode_window_launches(int num_seqs, int num_q_heads, int num_
   if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads ||
       head_dim <= 0 || block_size <= 0 || num_blocks <= 0 || window <= 0)
     return 0;
-  // the remap kernel and the even-split kernel
+  // the even-split kernel
   if (window_on_stream(num_q_heads / num_kv_heads, block_size, num_blocks, num_kv_heads))
-    return 2;
+    return 1;
   // the partition kernel, and the merge kernel when the longest context has
   // more than one partition (partitions are sized from max_context_len)
   const int pt = resolve_partition(num_seqs, num_kv_heads, max_context_len, partition_tokens);
@@ -2041,6 +2018,20 @@ extern "C" pa_status pa_decode_append_window(
                             max_blocks_per_seq, context_lens, max_context_len, num_seqs,
                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
                             dtype, workspace, workspace_bytes, partition_tokens, stream, window);
+}
+
+extern "C" pa_status pa_decode_append_window_overlapped(
+    void *out, const void *q, const void *k_new, const void *v_new, const int64_t *slot_mapping,
+    void *k_cache, void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+    const int32_t *context_lens, int max_context_len, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, float scale, int window,
+    pa_dtype dtype, void *workspace, size_t workspace_bytes, int partition_tokens, void *stream) {
+  if (window <= 0) return PA_ERR_INVALID;
+  return decode_append_impl(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,
+                            max_blocks_per_seq, context_lens, max_context_len, num_seqs,
+                            num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                            dtype, workspace, workspace_bytes, partition_tokens, stream, window,
+                            true);
 }
 
 bool pa_internal_pool_tensor_map(CUtensorMap *map, const void *base, long long rows, int head_dim,

@@ -33,8 +33,8 @@ class DecodeStep:
         self.fused = fused
         self.window = int(window)
         # fused steps only: the kernel may start during the preceding kernel's tail
-        # (pa_decode_append_overlapped); the lengths, tables and slots must not be
-        # written by that kernel
+        # (pa_decode_append_overlapped, pa_decode_append_window_overlapped); the
+        # lengths, tables and slots must not be written by that kernel
         self.overlapped = overlapped
         self.k_cache, self.v_cache = k_cache, v_cache
         self.q, self.k_new, self.v_new = q, k_new, v_new
@@ -98,7 +98,8 @@ class DecodeStep:
                                         self.slot_mapping, self.k_cache, self.v_cache,
                                         self.block_tables, self.context_lens,
                                         self.max_context_len, self.scale, self.window,
-                                        self.workspace, self.partition_tokens, stream)
+                                        self.workspace, self.partition_tokens, stream,
+                                        overlapped=self.overlapped)
             return
         fn = abi.pa_decode_append_overlapped if self.overlapped else abi.pa_decode_append
         fn(self.out, self.q, self.k_new, self.v_new, self.slot_mapping, self.k_cache,

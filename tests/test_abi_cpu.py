@@ -402,13 +402,10 @@ def test_workspace_size():
     # a fixed 64 KiB counter region, then room for the larger of the two kernels' scratch
     region = 64 * 1024
     # fixed partitions (SIMT kernel): acc [D] + (max, sum) per (seq, q head, partition);
-    # even split with 512 tokens per CTA: 2 pieces per CTA of G heads x (D + 4), then a
-    # sliding window's remap at block size 8: lengths and skips (16-byte padded) and
-    # tables of ceil(max_context_len / 8) entries per sequence
+    # even split with 512 tokens per CTA: 2 pieces per CTA of G heads x (D + 4)
     simt = 4 * 8 * 3 * (128 + 2) * 4
     ctas = -(-(4 * 2 * -(-1100 // 64)) // (512 // 64))
-    remap = -(-(2 * 4 * 4) // 16) * 16 + 4 * -(-1100 // 8) * 4
-    stream = 2 * ctas * 4 * (128 + 4) * 4 + remap
+    stream = 2 * ctas * 4 * (128 + 4) * 4
     assert abi.pa_decode_workspace_size(4, 8, 2, 128, 1100, 512) == region + max(simt, stream)
     assert abi.pa_decode_workspace_size(4, 8, 2, 128, 1100, 0) >= region
     assert abi.pa_decode_workspace_size(4, 6, 4, 128, 1100, 0) == 0  # 6 / 4 heads: invalid

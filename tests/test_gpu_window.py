@@ -160,3 +160,38 @@ def test_window_bad_inputs_are_reported_not_accessed(fused):
     ref = oracle.decode_window(batch.q, kp, vp, batch.block_tables, batch.context_lens,
                                batch.scale, batch.dtype, 32)
     assert_close(out, ref, batch.dtype, "window after bad inputs")
+
+
+def test_window_overlapped_launch_gives_the_same_bits():
+    """pa_decode_append_window_overlapped (the windowed kernel may start during the
+    preceding kernel's tail) returns the bits of pa_decode_append_window, also when
+    its launches follow each other back to back and inside a CUDA graph; the
+    entries and rows before each window are still never read."""
+    batch = synth.llama8b()
+    window = 1024
+    ref = GpuBatch(batch, fused=True, window=window, step_tables=_forget(batch, window))
+    _poison_before_window(ref, batch, window)
+    want = ref.run().clone()
+    assert abi.pa_device_status() == 0
+    del ref
+    g = GpuBatch(batch, fused=True, window=window, step_tables=_forget(batch, window))
+    _poison_before_window(g, batch, window)
+    g.step.overlapped = True
+    for _ in range(3):  # each launch follows the previous one on the stream
+        g.step.append()
+    torch.cuda.synchronize()
+    assert abi.pa_device_status() == 0
+    assert torch.equal(g.step.out.view(torch.int16), want.view(torch.int16))
+    graph = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            g.step.append()
+            g.step.append()
+    torch.cuda.current_stream().wait_stream(s)
+    g.step.out.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert abi.pa_device_status() == 0
+    assert torch.equal(g.step.out.view(torch.int16), want.view(torch.int16))
