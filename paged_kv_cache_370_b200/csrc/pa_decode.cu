@@ -724,7 +724,8 @@ __global__ void __launch_bounds__(kThreads, (Cfg<D, G>::kMinCtas))
   volatile int *last_flag = abort_flag + 1;
   // the piece fetched ahead of the final merge: pre_state 0 = open, 1 = the producer
   // has issued its copy into pre_piece (landing on pre_bar), 2 = the consumers went
-  // ahead without it (whichever sets it first from 0 wins)
+  // ahead without it, 3 = the producer found it not out yet (whichever sets it first
+  // from 0 wins)
   int *pre_state = reinterpret_cast<int *>(smem + C::kPreStateOffset);
   uint64_t *pre_bar = reinterpret_cast<uint64_t *>(smem + C::kPreStateOffset + 8);
   const float *pre_piece = reinterpret_cast<const float *>(smem + C::kPreOffset);
