@@ -78,8 +78,9 @@ struct PrefillParams {
   int block_size;
   int num_blocks;
   int window;
-  int q_tiles;                // grid.y
+  int q_tiles;                // grid.y (tcgen05 kernel: query tiles of an item)
   float scale_log2;
+  int pair_heads;             // tcgen05 kernel: 1 = an item is two q heads of one kv head
 };
 
 template <int D>
@@ -435,13 +436,15 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
 
 // ============================================================ tcgen05 kernel (5th-gen tensor cores)
 // Same computation on tcgen05.mma, with every operand of P V but V in tensor
-// memory, as a persistent kernel: one CTA per SM takes work items -- (q head, 256
-// query tokens, sequence) -- one after another from a counter, and fetches the next
-// item's Q and K/V tiles while the current one computes, so neither a CTA launch
-// nor the first fetches of an item leave the SM idle.
-// The 256 rows form two groups of 128 (one tcgen05 M each); the groups share
-// every K/V tile of 128 keys and take turns on the tensor core, so one group's
-// softmax overlaps the other group's products.
+// memory, as a persistent kernel: one CTA per SM takes work items one after another
+// from a counter, and fetches the next item's Q and K/V tiles while the current one
+// computes, so neither a CTA launch nor the first fetches of an item leave the SM
+// idle. An item is two groups of 128 query rows (one tcgen05 M each) that read the
+// same keys: with an even number of q heads per kv head, the same 128 query tokens
+// of two q heads of one kv head (the groups then need the same tiles); otherwise
+// 256 query tokens of one q head, split in two (the second group then needs one
+// tile more). The groups share every K/V tile of 128 keys and take turns on the
+// tensor core, so one group's softmax overlaps the other group's products.
 //   warp 0      takes items, publishes each item's extent, stages its Q rows (TMA,
 //               once the previous item's last S has read the Q buffer) and its
 //               128-key K and V tiles (TMA) into two rings (3 K slots and 2 V slots
@@ -478,9 +481,10 @@ constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O resc
 // One work item as the producer publishes it to the other warps.
 struct Item {
   int valid;        // 0: no more items
-  int h, b;         // q head, sequence
+  int h, b;         // q head (of group 0), sequence
+  int g_head, g_row;  // group g: q head h + g * g_head, query rows from q0 + g * g_row
   int qs0, q0;      // first query row of the sequence in q / out, first row of the item in it
-  int rows;         // query rows of the item (<= 256)
+  int rows;         // query rows of the item (<= 128 with two heads, else <= 256)
   int n;            // positions of the sequence
   int p_first;      // position of the item's first query row
   int k_base;       // first key of the item's first tile
@@ -552,7 +556,9 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   const int cap = p.max_blocks_per_seq * bs;
   const int align = bs < kN ? bs : kN;
   const int G = p.num_q_heads / p.num_kv_heads;
-  const long long n_items = (long long)p.num_q_heads * p.q_tiles * p.num_seqs;
+  const bool pair = p.pair_heads != 0;
+  const int h_items = pair ? p.num_q_heads / 2 : p.num_q_heads;  // items per query tile
+  const long long n_items = (long long)h_items * p.q_tiles * p.num_seqs;
 
   if (tid == 0) {
     for (int s = 0; s < NK; ++s) {
@@ -596,16 +602,20 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     long long kt = 0, vt = 0;  // K / V tiles loaded so far (over all items)
     int nq = 0;                // items whose Q rows were loaded (those with tiles)
     for (int it = 0;; ++it) {
-      // ---- the next work item: (q head fastest, longest query tiles first, sequence)
+      // ---- the next work item: (q head or head pair fastest, longest query tiles
+      // first, sequence)
       long long k = 0;
       if (lane == 0) k = atomicAdd(work, 1u);
       k = __shfl_sync(0xffffffffu, k, 0);
       Item I;
       I.valid = k < n_items;
       if (I.valid) {
-        I.h = (int)(k % p.num_q_heads);
-        const int qt = p.q_tiles - 1 - (int)((k / p.num_q_heads) % p.q_tiles);
-        I.b = (int)(k / ((long long)p.num_q_heads * p.q_tiles));
+        const int hi = (int)(k % h_items);
+        I.h = pair ? 2 * hi : hi;
+        I.g_head = pair ? 1 : 0;
+        I.g_row = pair ? 0 : kM;
+        const int qt = p.q_tiles - 1 - (int)((k / h_items) % p.q_tiles);
+        I.b = (int)(k / ((long long)h_items * p.q_tiles));
         int n = __ldg(p.context_lens + I.b);
         const int qs0 = __ldg(p.q_start + I.b), qs1 = __ldg(p.q_start + I.b + 1);
         int m = qs1 - qs0;
@@ -622,15 +632,16 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
           atomicOr(&g_prefill_error, PA_DEVERR_CONTEXT_LEN);
         I.n = n;
         I.qs0 = qs0;
-        I.q0 = qt * NG * kM;
-        I.rows = m > I.q0 ? min(NG * kM, m - I.q0) : 0;
+        const int item_rows = pair ? kM : NG * kM;
+        I.q0 = qt * item_rows;
+        I.rows = m > I.q0 ? min(item_rows, m - I.q0) : 0;
         I.p_first = n - m + I.q0;
         I.k_base = first_key(I.p_first, p.window) & ~(align - 1);
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-          const int grows = min(kM, I.rows - g * kM);
+          const int grows = min(kM, I.rows - g * I.g_row);
           I.gtiles[g] =
-              grows > 0 ? (I.p_first + g * kM + grows - 1 + 1 - I.k_base + kN - 1) / kN : 0;
+              grows > 0 ? (I.p_first + g * I.g_row + grows - 1 + 1 - I.k_base + kN - 1) / kN : 0;
         }
         I.ntiles = max(I.gtiles[0], I.gtiles[1]);
       }
@@ -649,7 +660,10 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       if (lane == 0) {
         mbar_expect_tx_arrive(q_full, (uint32_t)L::kQBytes);
         for (int pn = 0; pn < L::kPanels; ++pn)
-          tma_load_3d(q_sm + pn * L::kQPanel, &tmap_q, pn * 64, I.h, I.qs0 + I.q0, q_full);
+#pragma unroll
+          for (int g = 0; g < NG; ++g)
+            tma_load_3d(q_sm + pn * L::kQPanel + g * kM * 128, &tmap_q, pn * 64,
+                        I.h + g * I.g_head, I.qs0 + I.q0 + g * I.g_row, q_full);
       }
       __syncwarp();
       ++nq;
@@ -847,7 +861,6 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     // ====================================================== softmax, one row per thread
     const int grp = (warp - 2) / 4;
     const int r = 32 * (warp % 4) + lane;          // row in the group == TMEM lane
-    const int R = grp * kM + r;                    // row in the item
     const uint32_t trow = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + grp * 256;
     long long tg = 0;   // tiles of this group so far (over all items)
     long long vg = 0;   // V tiles of the items before this one
@@ -860,12 +873,13 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       if (!I.valid) break;
       if (I.ntiles == 0) continue;
       const int my_tiles = I.gtiles[grp];
+      const int R = grp * I.g_row + r;  // row in the item
       const int rows = I.rows, n = I.n, k_base = I.k_base, p_first = I.p_first;
       const int pr = min(p_first + R, n - 1);       // rows past the chunk: computed, not stored
       const int lo = first_key(pr, p.window);
       const int lo_first = first_key(p_first, p.window);
-      const int wr0 = min(p_first + grp * kM + 32 * (warp % 4), n - 1);
-      const int wr1 = min(p_first + grp * kM + 32 * (warp % 4) + 31, n - 1);
+      const int wr0 = min(p_first + grp * I.g_row + 32 * (warp % 4), n - 1);
+      const int wr1 = min(p_first + grp * I.g_row + 32 * (warp % 4) + 31, n - 1);
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < my_tiles; ++j) {
         const long long t = tg + j;
@@ -981,7 +995,8 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
           tmem_wait_ld();
           if (R < rows) {
             uint4 *dst = reinterpret_cast<uint4 *>(
-                og + ((size_t)(I.qs0 + I.q0 + R) * p.num_q_heads + I.h) * D + c4 * 32);
+                og + ((size_t)(I.qs0 + I.q0 + R) * p.num_q_heads + I.h + grp * I.g_head) * D +
+                c4 * 32);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               uint32_t w[4];
@@ -1096,7 +1111,7 @@ bool q_tensor_map(CUtensorMap *map, const void *q, int num_tokens, int num_q_hea
                               (cuuint64_t)num_tokens};
   const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2,
                                  (cuuint64_t)num_q_heads * head_dim * 2};
-  const cuuint32_t box[3] = {64u, 1u, (cuuint32_t)(t5::kGroups * t5::kM)};
+  const cuuint32_t box[3] = {64u, 1u, (cuuint32_t)t5::kM};  // one group's rows
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   CUtensorMap m;
   if (enc(&m, dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
@@ -1116,7 +1131,10 @@ pa_status launch_tc(const PrefillParams &prm_in, int max_q_len, const void *k_ca
                     const void *v_cache, pa_dtype dtype, cudaStream_t stream) {
   using L = t5::Lay<D>;
   PrefillParams prm = prm_in;
-  prm.q_tiles = (max_q_len + t5::kGroups * t5::kM - 1) / (t5::kGroups * t5::kM);
+  // two q heads of one kv head per item where the heads pair up, else 256 rows of one
+  prm.pair_heads = (prm.num_q_heads / prm.num_kv_heads) % 2 == 0 ? 1 : 0;
+  const int item_rows = prm.pair_heads ? t5::kM : t5::kGroups * t5::kM;
+  prm.q_tiles = (max_q_len + item_rows - 1) / item_rows;
   CUtensorMap tk, tv, tq;
   const long long rows = (long long)prm.num_blocks * prm.num_kv_heads * prm.block_size;
   const int box_rows = prm.block_size < t5::kN ? prm.block_size : t5::kN;
@@ -1139,7 +1157,9 @@ pa_status launch_tc(const PrefillParams &prm_in, int max_q_len, const void *k_ca
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return PA_ERR_CUDA;
-  const long long n_items = (long long)prm.num_q_heads * prm.q_tiles * prm.num_seqs;
+  const long long n_items =
+      (long long)(prm.pair_heads ? prm.num_q_heads / 2 : prm.num_q_heads) * prm.q_tiles *
+      prm.num_seqs;
   const unsigned grid = (unsigned)std::min<long long>(n_items, sms);
   if (cudaMemsetAsync(work, 0, sizeof(unsigned), stream) != cudaSuccess) return PA_ERR_CUDA;
   pa_prefill_tc_kernel<T, D><<<grid, t5::kThreads, L::kBytes, stream>>>(tk, tv, tq, prm, work);
@@ -1190,6 +1210,7 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
   prm.num_blocks = num_blocks;
   prm.window = window;
   prm.q_tiles = q_tiles;
+  prm.pair_heads = 0;
   prm.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 #if PA_PREFILL_TCGEN05
