@@ -323,10 +323,15 @@ pa_status pa_decode_append_window_overlapped(
  * head_dim 64 or 128; block_size a power of two >= 8 (PA_ERR_UNSUPPORTED otherwise).
  * Allocates nothing. Lengths or q_start entries out of range are clamped and reported
  * (PA_DEVERR_CONTEXT_LEN); bad block ids are skipped and reported (PA_DEVERR_BLOCK_ID).
- * Stream work: a 4-byte clear of the device's work counter, then one persistent kernel
- * (one CTA per SM takes (q head, 256 query tokens, sequence) items from that counter).
- * The counter is one per device and per library: two pa_prefill calls on one device must
- * not run at the same time (issue them on one stream, or order their streams).
+ * Stream work: a one-CTA kernel that writes the device's item order -- the (sequence,
+ * query tile) pairs by the number of key tiles they read, most first -- and clears the
+ * device's work counter (past 16,384 pairs: a 4-byte clear of the counter only, and
+ * items in index order), then one persistent kernel: one CTA per SM takes items from
+ * that counter in that order. An item is 128 query tokens of two q heads of one kv head
+ * (an even number of q heads per kv head), else 256 query tokens of one q head. The
+ * order and the counter are one per device and per library: two pa_prefill calls on one
+ * device must not run at the same time (issue them on one stream, or order their
+ * streams). The order changes which CTA computes an item and when, never its result.
  * ------------------------------------------------------------------------------------------ */
 pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
                      const int32_t *block_tables, int max_blocks_per_seq,

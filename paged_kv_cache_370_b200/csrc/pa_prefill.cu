@@ -81,6 +81,8 @@ struct PrefillParams {
   int q_tiles;                // grid.y (tcgen05 kernel: query tiles of an item)
   float scale_log2;
   int pair_heads;             // tcgen05 kernel: 1 = an item is two q heads of one kv head
+  const int *order;           // tcgen05 kernel: (sequence, query tile) pairs in the order
+                              // items take them, or null for index order
 };
 
 template <int D>
@@ -437,7 +439,8 @@ __global__ void __launch_bounds__(kThreads, 2) pa_prefill_kernel(
 // ============================================================ tcgen05 kernel (5th-gen tensor cores)
 // Same computation on tcgen05.mma, with every operand of P V but V in tensor
 // memory, as a persistent kernel: one CTA per SM takes work items one after another
-// from a counter, and fetches the next item's Q and K/V tiles while the current one
+// from a counter (in the order prefill_order_kernel wrote: the items reading the most
+// key tiles first), and fetches the next item's Q and K/V tiles while the current one
 // computes, so neither a CTA launch nor the first fetches of an item leave the SM
 // idle. An item is two groups of 128 query rows (one tcgen05 M each) that read the
 // same keys: with an even number of q heads per kv head, the same 128 query tokens
@@ -482,7 +485,6 @@ constexpr float kLazyRescale = 8.f;  // log2 of the growth that forces an O resc
 struct Item {
   int valid;        // 0: no more items
   int h, b;         // q head (of group 0), sequence
-  int g_head, g_row;  // group g: q head h + g * g_head, query rows from q0 + g * g_row
   int qs0, q0;      // first query row of the sequence in q / out, first row of the item in it
   int rows;         // query rows of the item (<= 128 with two heads, else <= 256)
   int n;            // positions of the sequence
@@ -558,6 +560,8 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
   const int G = p.num_q_heads / p.num_kv_heads;
   const bool pair = p.pair_heads != 0;
   const int h_items = pair ? p.num_q_heads / 2 : p.num_q_heads;  // items per query tile
+  // group g of an item: q head h + g * g_head, query rows from q0 + g * g_row
+  const int g_head = pair ? 1 : 0, g_row = pair ? 0 : kM;
   const long long n_items = (long long)h_items * p.q_tiles * p.num_seqs;
 
   if (tid == 0) {
@@ -602,8 +606,8 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     long long kt = 0, vt = 0;  // K / V tiles loaded so far (over all items)
     int nq = 0;                // items whose Q rows were loaded (those with tiles)
     for (int it = 0;; ++it) {
-      // ---- the next work item: (q head or head pair fastest, longest query tiles
-      // first, sequence)
+      // ---- the next work item: q head (or head pair) fastest, then the (sequence,
+      // query tile) pairs in the given order
       long long k = 0;
       if (lane == 0) k = atomicAdd(work, 1u);
       k = __shfl_sync(0xffffffffu, k, 0);
@@ -612,10 +616,10 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       if (I.valid) {
         const int hi = (int)(k % h_items);
         I.h = pair ? 2 * hi : hi;
-        I.g_head = pair ? 1 : 0;
-        I.g_row = pair ? 0 : kM;
-        const int qt = p.q_tiles - 1 - (int)((k / h_items) % p.q_tiles);
-        I.b = (int)(k / ((long long)h_items * p.q_tiles));
+        const long long u = k / h_items;  // (sequence, query tile) pair of the item
+        const int pu = p.order ? __ldg(p.order + u) : (int)u;
+        const int qt = p.q_tiles - 1 - pu % p.q_tiles;
+        I.b = pu / p.q_tiles;
         int n = __ldg(p.context_lens + I.b);
         const int qs0 = __ldg(p.q_start + I.b), qs1 = __ldg(p.q_start + I.b + 1);
         int m = qs1 - qs0;
@@ -639,9 +643,9 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
         I.k_base = first_key(I.p_first, p.window) & ~(align - 1);
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-          const int grows = min(kM, I.rows - g * I.g_row);
+          const int grows = min(kM, I.rows - g * g_row);
           I.gtiles[g] =
-              grows > 0 ? (I.p_first + g * I.g_row + grows - 1 + 1 - I.k_base + kN - 1) / kN : 0;
+              grows > 0 ? (I.p_first + g * g_row + grows - 1 + 1 - I.k_base + kN - 1) / kN : 0;
         }
         I.ntiles = max(I.gtiles[0], I.gtiles[1]);
       }
@@ -663,7 +667,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
 #pragma unroll
           for (int g = 0; g < NG; ++g)
             tma_load_3d(q_sm + pn * L::kQPanel + g * kM * 128, &tmap_q, pn * 64,
-                        I.h + g * I.g_head, I.qs0 + I.q0 + g * I.g_row, q_full);
+                        I.h + g * g_head, I.qs0 + I.q0 + g * g_row, q_full);
       }
       __syncwarp();
       ++nq;
@@ -861,6 +865,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
     // ====================================================== softmax, one row per thread
     const int grp = (warp - 2) / 4;
     const int r = 32 * (warp % 4) + lane;          // row in the group == TMEM lane
+    const int R = grp * g_row + r;                 // row in the item
     const uint32_t trow = tmem + ((uint32_t)(32 * (warp % 4)) << 16) + grp * 256;
     long long tg = 0;   // tiles of this group so far (over all items)
     long long vg = 0;   // V tiles of the items before this one
@@ -873,13 +878,12 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
       if (!I.valid) break;
       if (I.ntiles == 0) continue;
       const int my_tiles = I.gtiles[grp];
-      const int R = grp * I.g_row + r;  // row in the item
       const int rows = I.rows, n = I.n, k_base = I.k_base, p_first = I.p_first;
       const int pr = min(p_first + R, n - 1);       // rows past the chunk: computed, not stored
       const int lo = first_key(pr, p.window);
       const int lo_first = first_key(p_first, p.window);
-      const int wr0 = min(p_first + grp * I.g_row + 32 * (warp % 4), n - 1);
-      const int wr1 = min(p_first + grp * I.g_row + 32 * (warp % 4) + 31, n - 1);
+      const int wr0 = min(p_first + grp * g_row + 32 * (warp % 4), n - 1);
+      const int wr1 = min(p_first + grp * g_row + 32 * (warp % 4) + 31, n - 1);
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < my_tiles; ++j) {
         const long long t = tg + j;
@@ -995,7 +999,7 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
           tmem_wait_ld();
           if (R < rows) {
             uint4 *dst = reinterpret_cast<uint4 *>(
-                og + ((size_t)(I.qs0 + I.q0 + R) * p.num_q_heads + I.h + grp * I.g_head) * D +
+                og + ((size_t)(I.qs0 + I.q0 + R) * p.num_q_heads + I.h + grp * g_head) * D +
                 c4 * 32);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
@@ -1047,32 +1051,119 @@ pa_status launch(const PrefillParams &prm, const void *k_cache, const void *v_ca
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-// The persistent kernel's work counter: one per device, cleared on the stream before
-// every launch (a 4-byte memset). Only a successful address lookup is kept.
+// The persistent kernel's work counter and item order: one of each per device,
+// written on the stream before every launch. Only a successful address lookup is
+// kept.
 __device__ unsigned g_prefill_work;
 
-unsigned *prefill_work_counter() {
+constexpr int kOrderThreads = 1024;
+constexpr int kOrderBuckets = 4096;  // tile counts from the last bucket on share it
+constexpr int kOrderCap = 16384;     // (sequence, query tile) pairs the order holds
+__device__ int g_prefill_order[kOrderCap];
+
+template <typename Sym>
+void *symbol_address(const Sym &sym, void **cache) {
   static std::mutex mu;
-  static unsigned *addr[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!cache[dev]) {
     void *a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_prefill_work) != cudaSuccess || !a) {
+    if (cudaGetSymbolAddress(&a, sym) != cudaSuccess || !a) {
       cudaGetLastError();
       return nullptr;
     }
-    addr[dev] = static_cast<unsigned *>(a);
+    cache[dev] = a;
   }
-  return addr[dev];
+  return cache[dev];
+}
+
+unsigned *prefill_work_counter() {
+  static void *addr[64] = {};
+  return static_cast<unsigned *>(symbol_address(g_prefill_work, addr));
+}
+
+int *prefill_order_buffer() {
+  static void *addr[64] = {};
+  return static_cast<int *>(symbol_address(g_prefill_order, addr));
+}
+
+// The order in which the persistent kernel's CTAs take the (sequence, query tile)
+// pairs: by the number of key tiles the pair's items read, most first, so that the
+// last items the CTAs take are short ones and the CTAs finish close together (the
+// longest-processing-time-first rule of list scheduling). One CTA: a counting sort
+// over the tile count (pairs with equal counts in any order; which CTA computes an
+// item, and when, does not change its result). It also clears the work counter.
+__global__ void __launch_bounds__(kOrderThreads) prefill_order_kernel(const PrefillParams p,
+                                                                     int *order, unsigned *work) {
+  __shared__ int hist[kOrderBuckets];
+  __shared__ int warp_base[kOrderThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) *work = 0u;
+  for (int i = tid; i < kOrderBuckets; i += kOrderThreads) hist[i] = 0;
+  __syncthreads();
+  const int pairs = p.num_seqs * p.q_tiles;
+  const int item_rows = p.pair_heads ? t5::kM : t5::kGroups * t5::kM;
+  const int align = p.block_size < t5::kN ? p.block_size : t5::kN;
+  const int cap = p.max_blocks_per_seq * p.block_size;
+  // the item's tiles as the persistent kernel counts them (lengths clamped the same
+  // way), as a bucket index that grows as the count falls
+  auto bucket_of = [&](int u) {
+    const int b = u / p.q_tiles;
+    const int qt = p.q_tiles - 1 - u % p.q_tiles;
+    const int n = max(0, min(min(__ldg(p.context_lens + b), cap), p.max_context_len));
+    const int qs0 = __ldg(p.q_start + b), qs1 = __ldg(p.q_start + b + 1);
+    int m = qs1 - qs0;
+    if (m < 0 || m > n || qs0 < 0 || qs1 > p.num_tokens) m = 0;
+    const int q0 = qt * item_rows;
+    const int rows = m > q0 ? min(item_rows, m - q0) : 0;
+    const int p_first = n - m + q0;
+    const int k_base = first_key(p_first, p.window) & ~(align - 1);
+    const int tiles = rows > 0 ? (p_first + rows - k_base + t5::kN - 1) / t5::kN : 0;
+    return kOrderBuckets - 1 - min(tiles, kOrderBuckets - 1);
+  };
+  for (int u = tid; u < pairs; u += kOrderThreads) atomicAdd(&hist[bucket_of(u)], 1);
+  __syncthreads();
+  // bucket starts: an exclusive prefix sum over the buckets, kPer per thread
+  constexpr int kPer = kOrderBuckets / kOrderThreads;
+  int cnt[kPer], sum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    cnt[i] = hist[tid * kPer + i];
+    sum += cnt[i];
+  }
+  int incl = sum;
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_base[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int w = warp_base[lane];
+    int wi = w;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += v;
+    }
+    warp_base[lane] = wi - w;
+  }
+  __syncthreads();
+  int start = warp_base[warp] + incl - sum;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    hist[tid * kPer + i] = start;
+    start += cnt[i];
+  }
+  __syncthreads();
+  for (int u = tid; u < pairs; u += kOrderThreads) order[atomicAdd(&hist[bucket_of(u)], 1)] = u;
 }
 
 // TMA tensor map over q viewed as [num_tokens][num_q_heads][head_dim]: boxes of 64
-// head_dim columns x 1 head x 256 tokens (one 128-row group pair of one head),
+// head_dim columns x 1 head x 128 tokens (the rows of one group),
 // 128-byte swizzle; tokens past num_tokens read as zeros. Cached per (base, shape).
 bool q_tensor_map(CUtensorMap *map, const void *q, int num_tokens, int num_q_heads, int head_dim,
                   pa_dtype dtype) {
@@ -1161,7 +1252,17 @@ pa_status launch_tc(const PrefillParams &prm_in, int max_q_len, const void *k_ca
       (long long)(prm.pair_heads ? prm.num_q_heads / 2 : prm.num_q_heads) * prm.q_tiles *
       prm.num_seqs;
   const unsigned grid = (unsigned)std::min<long long>(n_items, sms);
-  if (cudaMemsetAsync(work, 0, sizeof(unsigned), stream) != cudaSuccess) return PA_ERR_CUDA;
+  // the item order (which also clears the counter), or index order past its capacity
+  prm.order = nullptr;
+  if ((long long)prm.num_seqs * prm.q_tiles <= kOrderCap) {
+    int *order = prefill_order_buffer();
+    if (!order) return PA_ERR_CUDA;
+    prefill_order_kernel<<<1, kOrderThreads, 0, stream>>>(prm, order, work);
+    if (cudaGetLastError() != cudaSuccess) return PA_ERR_CUDA;
+    prm.order = order;
+  } else if (cudaMemsetAsync(work, 0, sizeof(unsigned), stream) != cudaSuccess) {
+    return PA_ERR_CUDA;
+  }
   pa_prefill_tc_kernel<T, D><<<grid, t5::kThreads, L::kBytes, stream>>>(tk, tv, tq, prm, work);
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -1211,6 +1312,7 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
   prm.window = window;
   prm.q_tiles = q_tiles;
   prm.pair_heads = 0;
+  prm.order = nullptr;
   prm.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 #if PA_PREFILL_TCGEN05
