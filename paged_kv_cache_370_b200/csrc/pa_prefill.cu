@@ -597,6 +597,11 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
 
   if (warp == 0) {
     // ======================================================================== producer
+    // Launched as a programmatic dependent of prefill_order_kernel, the CTA may have
+    // started before that kernel finished: wait for it before the first read of the
+    // item order or the work counter (a no-op otherwise). Nothing else the kernel
+    // reads is written by it.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k)));
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_v)));
@@ -1057,7 +1062,7 @@ pa_status launch(const PrefillParams &prm, const void *k_cache, const void *v_ca
 __device__ unsigned g_prefill_work;
 
 constexpr int kOrderThreads = 1024;
-constexpr int kOrderBuckets = 4096;  // tile counts from the last bucket on share it
+constexpr int kOrderBuckets = 1024;  // tile counts from the last bucket on share it
 constexpr int kOrderCap = 16384;     // (sequence, query tile) pairs the order holds
 __device__ int g_prefill_order[kOrderCap];
 
@@ -1101,6 +1106,9 @@ __global__ void __launch_bounds__(kOrderThreads) prefill_order_kernel(const Pref
                                                                      int *order, unsigned *work) {
   __shared__ int hist[kOrderBuckets];
   __shared__ int warp_base[kOrderThreads / 32];
+  // the persistent kernel behind this one may start its set-up now; it reads the
+  // order and the counter only once this kernel has completed (griddepcontrol.wait)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) *work = 0u;
   for (int i = tid; i < kOrderBuckets; i += kOrderThreads) hist[i] = 0;
@@ -1263,7 +1271,19 @@ pa_status launch_tc(const PrefillParams &prm_in, int max_q_len, const void *k_ca
   } else if (cudaMemsetAsync(work, 0, sizeof(unsigned), stream) != cudaSuccess) {
     return PA_ERR_CUDA;
   }
-  pa_prefill_tc_kernel<T, D><<<grid, t5::kThreads, L::kBytes, stream>>>(tk, tv, tq, prm, work);
+  // behind the order kernel: a programmatic dependent (its set-up overlaps that kernel)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(t5::kThreads);
+  cfg.dynamicSmemBytes = L::kBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = prm.order ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, pa_prefill_tc_kernel<T, D>, tk, tv, tq, prm, work) != cudaSuccess)
+    return PA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
