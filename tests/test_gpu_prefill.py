@@ -71,6 +71,8 @@ SHAPES = [
     (4, 4, 64, "f16", 64, [0, 5, 140], [0, 5, 70]),
     # three q heads per kv head: items of 256 rows of one head, not head pairs
     (6, 2, 64, "bf16", 16, [300, 45, 129], [260, 45, 129]),
+    # two q heads per kv head: each item is both heads of one kv head
+    (8, 4, 128, "f16", 16, [200, 129, 16], [150, 129, 16]),
 ]
 
 
