@@ -170,8 +170,24 @@ def recorded_traffic(algorithmic_now: float, record=TRAFFIC_RECORD):
 
 
 # ---------------------------------------------------------------------------------- clocks
+def bus_id_of(torch, device) -> str | None:
+    """The PCI bus id of a CUDA device as nvidia-smi and NVML print it."""
+    props = torch.cuda.get_device_properties(device)
+    bus = getattr(props, "pci_bus_id", None)
+    if not isinstance(bus, int):
+        return None
+    return (f"{getattr(props, 'pci_domain_id', 0):08x}:{bus:02x}:"
+            f"{getattr(props, 'pci_device_id', 0):02x}.0")
+
+
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons for one GPU."""
+    """nvidia-smi samples of SM clock and throttle reasons for one GPU (every 50 ms
+    over the whole run), and NVML samples every ~0.2 ms while ``fast_start`` /
+    ``fast_stop`` bracket a timed region shorter than that interval."""
+
+    # NVML's clock-event reason bits, in the order of FIELDS' four reasons
+    _NVML_REASONS = ("nvmlClocksEventReasonHwSlowdown", "nvmlClocksEventReasonHwThermalSlowdown",
+                     "nvmlClocksEventReasonSwThermalSlowdown", "nvmlClocksEventReasonSwPowerCap")
 
     FIELDS = ("timestamp,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -206,6 +222,41 @@ class ClockSampler:
             except ValueError:
                 continue
 
+    def fast_start(self):
+        """Poll NVML from a thread until fast_stop (needs the GPU's bus id)."""
+        self._fast = None
+        if not self.bus_id:
+            return
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(self.bus_id)
+            max_sm = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            bits = [getattr(pynvml, n) for n in self._NVML_REASONS]
+        except Exception:
+            return
+        stop = threading.Event()
+
+        def poll():
+            while not stop.is_set():
+                try:
+                    sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    return
+                self.samples.append((time.time(), sm, max_sm,
+                                     ["Active" if r & b else "Not Active" for b in bits]))
+                time.sleep(2e-4)
+
+        self._fast = (threading.Thread(target=poll, daemon=True), stop)
+        self._fast[0].start()
+
+    def fast_stop(self):
+        if getattr(self, "_fast", None):
+            self._fast[1].set()
+            self._fast[0].join(timeout=2)
+            self._fast = None
+
     def stop(self):
         if self.proc:
             self.proc.terminate()
@@ -228,7 +279,7 @@ class ClockSampler:
         return {"sm_mhz": float(np.median([s[1] for s in used])),
                 "sm_max_mhz": float(max(s[2] for s in used)), "reasons": reasons,
                 "samples": len(used), "samples_in_timed_region": len(inside),
-                "window": ("the timed region" if inside else
+                "window": ("the timed region (NVML, every ~0.2 ms)" if inside else
                            f"the timed region ({1e3 * (t1 - t0):.1f} ms) and the kernel-timing "
                            f"loop after it ({1e3 * (end - t1):.0f} ms), sampled every 50 ms")}
 
@@ -540,13 +591,7 @@ def run_ours(args, rank, world, local, dist):
         torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
-    props = torch.cuda.get_device_properties(device)
-    bus = getattr(props, "pci_bus_id", None)
-    bus_str = None
-    if isinstance(bus, int):
-        bus_str = f"{getattr(props, 'pci_domain_id', 0):08x}:{bus:02x}:" \
-                  f"{getattr(props, 'pci_device_id', 0):02x}.0"
-    sampler = ClockSampler(bus_str)
+    sampler = ClockSampler(bus_id_of(torch, device))
     sampler.start()
     time.sleep(0.3)
     # ---- warm-up: exactly W steps, untimed; the timed graphs uploaded to the device
@@ -555,6 +600,7 @@ def run_ours(args, rank, world, local, dist):
     # ---- the timed region: exactly K steps
     start_ev, end_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
+    sampler.fast_start()
     t0 = time.time()
     # the device idles ~0.1 ms on a spin kernel (torch's) while the host queues the
     # start event and the graph behind it: the events then bracket the K steps'
@@ -568,6 +614,7 @@ def run_ours(args, rank, world, local, dist):
     end_ev.record(stream)
     barrier()
     t1 = time.time()
+    sampler.fast_stop()
     total_ms = start_ev.elapsed_time(end_ev)
     # ---- the decode kernel's own duration: >= 50 replays of a graph of R decode
     # launches (about half a second), CUDA events on the same stream
@@ -963,15 +1010,17 @@ def prefill_measure(pool_blocks, window, n_timed, n_warm):
     warm = step_plan(n_warm, 0, one_step, steps, 4 * V, torch)
     timed = step_plan(n_timed, n_warm % V, one_step, steps, 4 * V, torch)
     g_att = capture(lambda: [attend(st) for st in steps], torch)
-    clocks = ClockSampler(os.environ.get("PA_BUS_ID"))
+    clocks = ClockSampler(bus_id_of(torch, dev))
     clocks.start()
     time.sleep(0.3)
     time_graphs(warm, stream, torch)
     upload_graphs(timed, stream)
     torch.cuda.synchronize()
+    clocks.fast_start()
     t0 = time.time()
     step_ms = time_graphs(timed, stream, torch) / n_timed
     t1 = time.time()
+    clocks.fast_stop()
     reps = 50
     att_ms = time_graphs([(g_att, reps)], stream, torch) / (reps * V)
     t2 = time.time()
