@@ -42,6 +42,10 @@ MUTANTS = {
     "prefill_not_causal": ("int p = n - m + (tok - q_start[b]);", "int p = n - 1;"),
     "prefill_position_shifted": ("int p = n - m + (tok - q_start[b]);",
                                  "int p = n - m + (tok - q_start[b]) - (tok > q_start[b]);"),
+    "prefill_window_one_short": ("int lo = (window > 0 && p + 1 > window) ? p + 1 - window : 0;",
+                                 "int lo = (window > 0 && p + 1 > window) ? p + 2 - window : 0;"),
+    "prefill_window_ignored": ("int lo = (window > 0 && p + 1 > window) ? p + 1 - window : 0;",
+                               "int lo = 0;"),
     "copy_k_only": ("v_cache[(size_t)dst * block_elems + i] = v_cache[(size_t)src * block_elems + i];",
                     ";"),
 }
