@@ -388,6 +388,23 @@ int pa_decode_default_partition(int num_seqs, int num_kv_heads, int max_context_
 pa_status pa_device_status(void *stream, int32_t *code);
 
 /* ------------------------------------------------------------------------------------------
+ * pa_hbm_read -- a measurement utility, not part of the method (the pages have no
+ * counterpart): reads `bytes` of device memory at `buf` once, as a read-only stream, so
+ * that a caller can time this GPU's read rate beside the kernels that are bound by it.
+ *
+ *   buf          device, `bytes` bytes, 16-byte aligned; only read
+ *   bytes        > 0, a multiple of 16; larger than L2 (126 MB) to measure HBM
+ *   sink         device, one uint32: cleared on `stream`, then the XOR of every 32-bit
+ *                word of the buffer (written so that the loads cannot be dropped)
+ *   ctas_per_sm  1..4: CTAs of 512 threads launched per SM
+ * Stream work: a 4-byte clear and one kernel (16-byte evict-first loads, four in flight
+ * per thread). Allocates nothing. PA_ERR_INVALID for a null or misaligned pointer, a size
+ * that is 0 or not a multiple of 16, or ctas_per_sm outside 1..4.
+ * ------------------------------------------------------------------------------------------ */
+pa_status pa_hbm_read(const void *buf, size_t bytes, uint32_t *sink, int ctas_per_sm,
+                      void *stream);
+
+/* ------------------------------------------------------------------------------------------
  * pa_debug_wait_test -- test hook for the bounded waits of the decode kernels (not for
  * production use; the pages have no counterpart).
  * Every wait of a decode kernel is bounded: a wait that runs out sets PA_DEVERR_TIMEOUT,

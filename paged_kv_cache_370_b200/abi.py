@@ -75,6 +75,7 @@ def _load() -> ctypes.CDLL:
                                                    i, f, i, i, P, sz, i, P]),
         "pa_decode_static_workspace": (i, [P, P, P, P, P, i, P, i, i, i, i, i, i, i, f, i, i, P]),
         "pa_device_status": (i, [P, P]),
+        "pa_hbm_read": (i, [P, sz, P, i, P]),
         "pa_status_string": (ctypes.c_char_p, [i]),
         "pa_slot_mapping": (i, [P, i, P, i, i, P]),
         "pa_alloc_create": (i, [i, i, P]),
@@ -405,6 +406,14 @@ def pa_debug_wait_test(enable: bool, consumer_wait_ns: int = 0):
     (no copies issued); see include/pa.h. enable=False restores normal launches."""
     _check(_lib.pa_debug_wait_test(1 if enable else 0, int(consumer_wait_ns)),
            "pa_debug_wait_test")
+
+
+def pa_hbm_read(buf, sink, ctas_per_sm=4, stream=None):
+    """Read the device buffer ``buf`` once as a read-only stream (a measurement
+    utility); ``sink`` (one int32 on the device) receives the XOR of its 32-bit words."""
+    nbytes = buf.numel() * buf.element_size()
+    _check(_lib.pa_hbm_read(_dev_ptr(buf, "buf"), nbytes, _dev_ptr(sink, "sink"),
+                            int(ctas_per_sm), _stream(stream)), "pa_hbm_read")
 
 
 def pa_device_status(stream=None) -> int:
