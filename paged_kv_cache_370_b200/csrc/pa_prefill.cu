@@ -979,9 +979,12 @@ __global__ void __launch_bounds__(t5::kThreads, 1) pa_prefill_tc_kernel(
           // (after the TMA copies into this V slot have landed)
           wait_bounded(&v_full[gv % NV], (gv / NV) & 1, abort_flag);
           unsigned char *vz = smem + L::kVRingOff + (gv % NV) * L::kSlotBytes;
-          for (int c = r; c < kN * 8 * L::kPanels; c += 128) {
-            const int vr = c / (8 * L::kPanels), pn = (c / 8) % L::kPanels, ch = c % 8;
-            if (vr >= nskip && vr < nvalid) continue;
+          // rows [0, nskip) and [max(nvalid, nskip), kN): only those rows are visited
+          const int hi0 = max(nvalid, nskip);
+          const int nrows = nskip + (kN - hi0);
+          for (int c = r; c < nrows * 8 * L::kPanels; c += 128) {
+            const int i = c / (8 * L::kPanels), pn = (c / 8) % L::kPanels, ch = c % 8;
+            const int vr = i < nskip ? i : hi0 + (i - nskip);
             *reinterpret_cast<uint4 *>(vz + pn * L::kKVPanel + vr * 128 + (ch << 4)) =
                 make_uint4(0u, 0u, 0u, 0u);
           }
