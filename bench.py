@@ -251,13 +251,16 @@ class ClockSampler:
 
         def poll():
             while not stop.is_set():
+                ts = time.time()
                 try:
                     sm = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
                     r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
                 except Exception:
                     return
+                # (time, SM MHz, max MHz, reasons, start of the query): a query that
+                # overlaps the timed region counts as taken in it
                 self.samples.append((time.time(), sm, max_sm,
-                                     ["Active" if r & b else "Not Active" for b in bits]))
+                                     ["Active" if r & b else "Not Active" for b in bits], ts))
                 time.sleep(2e-4)
 
         self._fast = (threading.Thread(target=poll, daemon=True), stop)
@@ -280,7 +283,8 @@ class ClockSampler:
     def summary(self, t0: float, t1: float, t_end: float | None = None) -> dict:
         """Clocks over the timed region [t0, t1]; when it is too short for a sample
         (50 ms apart), over it and the kernel-timing loop that follows, up to t_end."""
-        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        inside = [s for s in self.samples
+                  if (s[4] if len(s) > 4 else s[0]) <= t1 and s[0] >= t0]
         end = max(t1, t_end or t1)
         used = inside or [s for s in self.samples if t0 - 0.1 <= s[0] <= end + 0.1]
         if not used:
@@ -291,7 +295,7 @@ class ClockSampler:
         return {"sm_mhz": float(np.median([s[1] for s in used])),
                 "sm_max_mhz": float(max(s[2] for s in used)), "reasons": reasons,
                 "samples": len(used), "samples_in_timed_region": len(inside),
-                "window": ("the timed region (NVML, every ~0.2 ms)" if inside else
+                "window": ("the timed region (NVML queries that overlap it)" if inside else
                            f"the timed region ({1e3 * (t1 - t0):.1f} ms) and the kernel-timing "
                            f"loop after it ({1e3 * (end - t1):.0f} ms), sampled every 50 ms")}
 
