@@ -1,5 +1,6 @@
 """The C-ABI library on the CPU: exports, host block manager, slot helper and
 host-side argument checks. No device work is launched here."""
+import ctypes
 import os
 import re
 
@@ -396,6 +397,15 @@ def test_decode_rejects_bad_arguments_before_launch():
     # swap: a null space or unaligned pools are refused before any launch
     assert L.pa_swap_out(None, None, None, 8, None, 0, None) == abi.PA_ERR_INVALID
     assert L.pa_swap_in(None, None, None, 8, None, 0, None) == abi.PA_ERR_INVALID
+    # the read-rate probe: sizes, pointers and CTA counts are checked before any launch
+    buf, sink = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 12)
+    assert L.pa_hbm_read(None, 16, sink, 4, None) == abi.PA_ERR_INVALID
+    assert L.pa_hbm_read(buf, 16, None, 4, None) == abi.PA_ERR_INVALID
+    assert L.pa_hbm_read(buf, 0, sink, 4, None) == abi.PA_ERR_INVALID
+    assert L.pa_hbm_read(buf, 24, sink, 4, None) == abi.PA_ERR_INVALID      # not 16-byte units
+    assert L.pa_hbm_read(ctypes.c_void_p((1 << 20) + 8), 16, sink, 4, None) == abi.PA_ERR_INVALID
+    assert L.pa_hbm_read(buf, 16, sink, 0, None) == abi.PA_ERR_INVALID
+    assert L.pa_hbm_read(buf, 16, sink, 5, None) == abi.PA_ERR_INVALID
 
 
 def test_workspace_size():
